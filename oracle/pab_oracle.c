@@ -1,0 +1,259 @@
+/*
+ * pab_oracle.c -- plain, slow, fp64 CPU oracle for the Pyramid Attention
+ * Broadcast (PAB) attention stack.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path (the CUDA library
+ * under step_reuse_b200/) links, loads or calls this file; only the tests,
+ * the smoke check and the benchmark's CPU-baseline leg do.  It shares no
+ * code, header, table or constant with the CUDA path.
+ *
+ * Sources (the PAB pages):
+ *  - "Real-Time Video Generation with Pyramid Attention Broadcast"
+ *    (chatpaper.ai abstract): attention outputs are broadcast to later
+ *    diffusion steps in a pyramid style, a different strategy per attention.
+ *  - m.sbmmt.com PAB report, section "Implementation" and Fig. 2: the three
+ *    attention kinds (spatial, temporal, cross); the U-shaped attention
+ *    difference (first and last 15% of steps change a lot, the middle 70% is
+ *    stable); in the middle segment one step's attention output is broadcast
+ *    to the next few steps, with a wider range for kinds that change less.
+ *  - same report, Fig. 1: the difference between the attention outputs of
+ *    consecutive diffusion steps is quantified by MSE.
+ *
+ * Readings where the pages are silent (each is listed in the design notes):
+ *  - attention is the textbook softmax(Q K^T / sqrt(d)) V per head, no mask,
+ *    no bias, no output projection; head h owns channels [h*d, (h+1)*d);
+ *  - the 15% edge is rounded up: e = ceil(edge_pct * steps / 100);
+ *  - in the middle [e, steps - e) a compute serves itself plus the next
+ *    (range - 1) steps; windows are anchored at the first middle step and the
+ *    last one is cut at the end of the middle segment;
+ *  - MSE is the mean over all elements of (a - b)^2.
+ *
+ * Every function works in double precision.  The attention inputs are the
+ * bf16 values the GPU consumes, widened to double by the caller.
+ */
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+/* ------------------------------------------------------------------------ */
+/* Attention: one query row against Lk keys (the textbook definition).       */
+/*   s_j = (q . k_j) / sqrt(d);  m = max_j s_j;  p_j = exp(s_j - m);         */
+/*   o   = sum_j p_j v_j / sum_j p_j                                         */
+/* k_j starts at kbase + j*kstride (d contiguous doubles), likewise v_j.     */
+/* ------------------------------------------------------------------------ */
+static void attend_one_query(const double *q, const double *kbase, long kstride,
+                             const double *vbase, long vstride, int Lk, int d,
+                             double *o, double *p /* Lk scratch */)
+{
+    const double scale = 1.0 / sqrt((double)d);
+    double m = -INFINITY;
+    for (int j = 0; j < Lk; ++j) {
+        const double *kj = kbase + (long)j * kstride;
+        double s = 0.0;
+        for (int c = 0; c < d; ++c)
+            s += q[c] * kj[c];
+        s *= scale;
+        p[j] = s;
+        if (s > m)
+            m = s;
+    }
+    double denom = 0.0;
+    for (int j = 0; j < Lk; ++j) {
+        p[j] = exp(p[j] - m);
+        denom += p[j];
+    }
+    for (int c = 0; c < d; ++c) {
+        double acc = 0.0;
+        for (int j = 0; j < Lk; ++j)
+            acc += p[j] * vbase[(long)j * vstride + c];
+        o[c] = acc / denom;
+    }
+}
+
+/* Spatial attention (attention within a frame).
+ * q, k, v, o: [T][N][C] with C = heads*d.  For every frame t and head h the
+ * N tokens of frame t attend to each other. */
+int oracle_spatial_attention(const double *q, const double *k, const double *v,
+                             double *o, int T, int N, int heads, int d)
+{
+    if (T < 0 || N < 0 || heads <= 0 || d <= 0)
+        return -1;
+    const long C = (long)heads * d;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (N > 0 ? N : 1));
+        if (!p) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for collapse(2) schedule(dynamic)
+            for (int t = 0; t < T; ++t)
+                for (int h = 0; h < heads; ++h) {
+                    const long frame = (long)t * N * C;
+                    for (int n = 0; n < N; ++n)
+                        attend_one_query(q + frame + (long)n * C + (long)h * d,
+                                         k + frame + (long)h * d, C,
+                                         v + frame + (long)h * d, C, N, d,
+                                         o + frame + (long)n * C + (long)h * d, p);
+                }
+            free(p);
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/* Temporal attention (attention across frames at one spatial position).
+ * q, k, v, o: [N][T][C].  For every position n and head h the T frames at
+ * position n attend to each other. */
+int oracle_temporal_attention(const double *q, const double *k, const double *v,
+                              double *o, int N, int T, int heads, int d)
+{
+    if (T < 0 || N < 0 || heads <= 0 || d <= 0)
+        return -1;
+    const long C = (long)heads * d;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (T > 0 ? T : 1));
+        if (!p) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for collapse(2) schedule(dynamic, 64)
+            for (int n = 0; n < N; ++n)
+                for (int h = 0; h < heads; ++h) {
+                    const long pos = (long)n * T * C;
+                    for (int t = 0; t < T; ++t)
+                        attend_one_query(q + pos + (long)t * C + (long)h * d,
+                                         k + pos + (long)h * d, C,
+                                         v + pos + (long)h * d, C, T, d,
+                                         o + pos + (long)t * C + (long)h * d, p);
+                }
+            free(p);
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/* Cross attention (video tokens attend to text tokens).
+ * q, o: [R][C] (R video tokens, any order); kt, vt: [Lt][C] text tokens. */
+int oracle_cross_attention(const double *q, const double *kt, const double *vt,
+                           double *o, long R, int Lt, int heads, int d)
+{
+    if (R < 0 || Lt < 0 || heads <= 0 || d <= 0)
+        return -1;
+    const long C = (long)heads * d;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (Lt > 0 ? Lt : 1));
+        if (!p) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for schedule(dynamic, 256)
+            for (long r = 0; r < R; ++r)
+                for (int h = 0; h < heads; ++h)
+                    attend_one_query(q + r * C + (long)h * d, kt + (long)h * d, C,
+                                     vt + (long)h * d, C, Lt, d,
+                                     o + r * C + (long)h * d, p);
+            free(p);
+        }
+    }
+    return bad ? -2 : 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* PAB schedule, walked step by step in execution order (noisiest first).    */
+/*   edge steps (first and last edge_pct%): always compute;                  */
+/*   middle steps: a compute makes its output servable for the next          */
+/*   (range - 1) steps; while that budget lasts the step is a broadcast hit  */
+/*   (served from the cache), else it computes.                              */
+/* Outputs, per step i: is_compute[i] in {0,1} and source[i] = the step      */
+/* whose computed output step i uses (i itself when it computes).            */
+/* ------------------------------------------------------------------------ */
+int oracle_pab_edge_steps(int steps, int edge_pct)
+{
+    if (steps < 0 || edge_pct < 0 || edge_pct > 50)
+        return -1;
+    return (edge_pct * steps + 99) / 100; /* ceil(edge_pct% of steps) */
+}
+
+int oracle_pab_schedule(int steps, int edge_pct, int range, int *is_compute, int *source)
+{
+    if (steps < 0 || range < 1)
+        return -1;
+    const int e = oracle_pab_edge_steps(steps, edge_pct);
+    if (e < 0)
+        return -1;
+    const int lo = e, hi = steps - e;
+    int budget = 0;  /* further steps the cached output may still serve */
+    int cached = -1; /* step whose output is in the cache */
+    for (int i = 0; i < steps; ++i) {
+        const int middle = (i >= lo && i < hi);
+        if (middle && budget > 0 && cached >= 0) {
+            is_compute[i] = 0;
+            source[i] = cached;
+            budget -= 1;
+        } else {
+            is_compute[i] = 1;
+            source[i] = i;
+            cached = i;
+            budget = middle ? range - 1 : 0;
+        }
+    }
+    return 0;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Attention-difference diagnostic: mean over all n elements of (a - b)^2.   */
+/* ------------------------------------------------------------------------ */
+double oracle_mse(const double *a, const double *b, long n)
+{
+    if (n <= 0)
+        return 0.0;
+    double acc = 0.0;
+    for (long i = 0; i < n; ++i) {
+        const double diff = a[i] - b[i];
+        acc += diff * diff;
+    }
+    return acc / (double)n;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Layout change between the spatial view [T][N][C] and the temporal view    */
+/* [N][T][C]; elements are moved as opaque elem_size-byte units.             */
+/* ------------------------------------------------------------------------ */
+int oracle_layout(int to_temporal, const void *src, void *dst, int T, int N, int C,
+                  int elem_size)
+{
+    if (T < 0 || N < 0 || C < 0 || elem_size <= 0)
+        return -1;
+    const char *s = (const char *)src;
+    char *o = (char *)dst;
+    const size_t row = (size_t)C * elem_size;
+    for (int t = 0; t < T; ++t)
+        for (int n = 0; n < N; ++n) {
+            const size_t spatial_off = ((size_t)t * N + n) * row;
+            const size_t temporal_off = ((size_t)n * T + t) * row;
+            if (to_temporal)
+                memcpy(o + temporal_off, s + spatial_off, row);
+            else
+                memcpy(o + spatial_off, s + temporal_off, row);
+        }
+    return 0;
+}
+
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
