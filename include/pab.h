@@ -1,0 +1,196 @@
+/*
+ * pab.h -- C ABI of the B200 (sm_100a) Pyramid Attention Broadcast library.
+ *
+ * A video diffusion transformer block runs three attention kinds: spatial
+ * (tokens of one frame attend to each other), temporal (the frames at one
+ * spatial position attend to each other) and cross (video tokens attend to
+ * text tokens) -- PAB report (m.sbmmt.com), section "Implementation".
+ * Pyramid Attention Broadcast computes every attention in the first and last
+ * 15% of diffusion steps and, in the stable middle 70%, computes each kind
+ * once per window of r_kind steps and serves ("broadcasts") that output to
+ * the rest of the window -- same report, Fig. 2; paper abstract
+ * "Real-Time Video Generation with Pyramid Attention Broadcast".
+ *
+ * Conventions shared by every entry point
+ *  - Return value: PAB_OK (0) or a negative PAB_ERR_* code.  Nothing aborts,
+ *    throws or traps; pab_last_error_string() describes the last failure of
+ *    the calling thread.
+ *  - Pointers named q, k, v, out, src, dst, a, b are DEVICE pointers (CUDA
+ *    global memory of the current device) unless stated otherwise; the
+ *    caller owns them.  cuda_stream is a cudaStream_t (NULL = legacy default
+ *    stream); all device work is ordered on it and no call synchronises the
+ *    device unless its comment says so.
+ *  - Layouts are row-major with the last index contiguous.  C = heads * d and
+ *    head h occupies channels [h*d, (h+1)*d) of every token row.  N = H * W.
+ *  - Attention is softmax(Q K^T / sqrt(d)) V per head: no mask, no bias, no
+ *    output projection.  bf16 storage, fp32 accumulation, bf16 output.  With
+ *    dtype PAB_FP32 the inputs are rounded to bf16 (round to nearest even)
+ *    before the same bf16 kernels run, and the output is written as fp32.
+ *  - Alignment: every device pointer must be 16-byte aligned.
+ *  - Limits: 8 <= d <= 128 and d % 8 == 0; temporal length T <= 128;
+ *    1 <= text_len <= 512; spatial T <= 65535 frames; sizes must fit the
+ *    device; otherwise PAB_ERR_ARG or PAB_ERR_UNSUPPORTED.
+ */
+#ifndef PAB_H
+#define PAB_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* status codes */
+#define PAB_OK 0
+#define PAB_ERR_ARG (-1)         /* bad argument (null pointer, bad size, bad kind)   */
+#define PAB_ERR_STEP_ORDER (-2)  /* steps of one kind not strictly increasing          */
+#define PAB_ERR_NO_CACHE (-3)    /* broadcast step whose source output was never made  */
+#define PAB_ERR_CUDA (-4)        /* CUDA runtime error (incl. no device present)       */
+#define PAB_ERR_OOM (-5)         /* device allocation failed                           */
+#define PAB_ERR_UNSUPPORTED (-6) /* shape outside the kernels' documented limits       */
+
+/* attention kinds */
+enum { PAB_SPATIAL = 0, PAB_TEMPORAL = 1, PAB_CROSS = 2 };
+/* element types at the boundary */
+enum { PAB_BF16 = 0, PAB_FP32 = 1 };
+
+/* Broadcast ranges per kind (each >= 1; 1 = never broadcast) and the edge
+ * share in percent (0 -> the pages' 15).  The pages order the ranges
+ * r_cross >= r_temporal >= r_spatial (Fig. 2); that order is not enforced. */
+typedef struct {
+    int spatial;
+    int temporal;
+    int cross;
+    int edge_pct;
+} pab_ranges;
+
+typedef struct pab_plan pab_plan; /* opaque; owns the broadcast cache */
+
+/* Library version, (major << 16) | minor. */
+int pab_version(void);
+
+/* Text of the calling thread's last error ("" if none).  Owned by the
+ * library; valid until the thread's next failing call. */
+const char* pab_last_error_string(void);
+
+/* ---------------------------------------------------------------------- */
+/* Stateless attention kernels (each writes into caller memory).           */
+/* ---------------------------------------------------------------------- */
+
+/* Spatial attention (PAB report, "Implementation": attention within a frame).
+ * q, k, v, out: [T, N, C].  For each frame t and head h:
+ *   out[t, n, h] = sum_m softmax_m(q[t, n, h] . k[t, m, h] / sqrt(d)) v[t, m, h].
+ * dtype: PAB_BF16 only (the plan handles PAB_FP32 by conversion). */
+int pab_spatial_attention(const void* q, const void* k, const void* v, void* out,
+                          int T, int N, int heads, int d, void* cuda_stream);
+
+/* Temporal attention (same section: attention across frames).
+ * q, k, v, out: [N, T, C] (the temporal view).  For each position n, head h:
+ *   out[n, t, h] = sum_s softmax_s(q[n, t, h] . k[n, s, h] / sqrt(d)) v[n, s, h].
+ * T <= 128.  PAB_BF16 only. */
+int pab_temporal_attention(const void* q, const void* k, const void* v, void* out,
+                           int N, int T, int heads, int d, void* cuda_stream);
+
+/* Cross attention (same section: video tokens to text tokens).
+ * q, out: [R, C] (R video tokens in any order; out keeps it);
+ * kt, vt: [text_len, C].  Every text token is attended (no text mask).
+ *   out[r, h] = sum_j softmax_j(q[r, h] . kt[j, h] / sqrt(d)) vt[j, h].
+ * 1 <= text_len <= 512.  PAB_BF16 only. */
+int pab_cross_attention(const void* q, const void* kt, const void* vt, void* out,
+                        long long R, int text_len, int heads, int d, void* cuda_stream);
+
+/* ---------------------------------------------------------------------- */
+/* Layout change between the two views of a video token tensor.            */
+/* ---------------------------------------------------------------------- */
+
+/* to_temporal = 1: src [T, N, C] (spatial view) -> dst [N, T, C];
+ * to_temporal = 0: src [N, T, C] -> dst [T, N, C].
+ * dtype PAB_BF16 or PAB_FP32; bytes are moved unchanged.  src and dst must
+ * not overlap.  C * element size must be a multiple of 16 bytes. */
+int pab_layout(int to_temporal, const void* src, void* dst, int T, int N, int C,
+               int dtype, void* cuda_stream);
+
+/* ---------------------------------------------------------------------- */
+/* Attention-difference diagnostic (PAB report, Fig. 1: the difference      */
+/* between consecutive diffusion steps' attention outputs, as MSE).        */
+/* ---------------------------------------------------------------------- */
+
+/* *result (HOST pointer) = mean over n elements of (a - b)^2, accumulated in
+ * fp64 in a fixed order (bitwise reproducible for a given n).  a and b hold n
+ * elements of dtype (PAB_BF16 or PAB_FP32).  n == 0 gives 0.  Uses a
+ * per-device scratch buffer of fp64 partial sums that the library allocates
+ * on first use.  SYNCHRONISES cuda_stream before returning. */
+int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype,
+                      double* result, void* cuda_stream);
+
+/* As pab_attn_diff_mse, but writes the fp64 result to the DEVICE pointer
+ * result_dev (8-byte aligned) and does not synchronise.  Calls that run
+ * concurrently on different streams of one device share the scratch buffer
+ * and must be serialised by the caller. */
+int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype,
+                            double* result_dev, void* cuda_stream);
+
+/* Device status word of the kernels that wait on asynchronous copies: bit 0
+ * is set when a bounded wait gave up (the kernel then returns early and its
+ * output is incomplete).  Synchronises the device to read it; clear != 0
+ * resets it.  A healthy run reads 0. */
+int pab_device_errors(int clear, unsigned int* flags);
+
+/* ---------------------------------------------------------------------- */
+/* PAB plan: schedule + broadcast cache.                                   */
+/* ---------------------------------------------------------------------- */
+
+/* Create a plan for one video shape.  N = H * W tokens per frame, C = heads*d.
+ * steps >= 1 diffusion steps indexed 0..steps-1 in execution order.
+ * Schedule (per kind with range r; e = ceil(edge_pct * steps / 100)):
+ *   step i computes iff i < e, or i >= steps - e, or (i - e) % r == 0;
+ *   otherwise it is a broadcast hit served by the latest compute of the kind.
+ * No device memory is allocated here (see pab_plan_prepare).
+ * *out_plan receives the handle; destroy it with pab_plan_destroy. */
+int pab_plan_create(int T, int H, int W, int heads, int d, int text_len, int steps,
+                    pab_ranges ranges, int dtype, pab_plan** out_plan);
+
+/* Free the plan and its cache (device memory freed; no pointer returned by
+ * pab_attention stays valid).  NULL is accepted. */
+int pab_plan_destroy(pab_plan* plan);
+
+/* Start a new sampling run: the cache is invalidated and step order restarts.
+ * Device memory is kept. */
+int pab_plan_reset(pab_plan* plan);
+
+/* Allocate the cache (2 output slots per kind, plus bf16 staging for
+ * PAB_FP32 plans) on the current device now instead of at each kind's first
+ * compute.  Idempotent. */
+int pab_plan_prepare(pab_plan* plan);
+
+/* *is_compute = 1 if (kind, step) computes, 0 if it is a broadcast hit.
+ * Host only, no GPU needed. */
+int pab_schedule_query(const pab_plan* plan, int kind, int step, int* is_compute);
+
+/* *source_step = the step whose computed output (kind, step) uses (step
+ * itself when it computes).  Host only. */
+int pab_schedule_source(const pab_plan* plan, int kind, int step, int* source_step);
+
+/* Number of computing steps of `kind` over the whole run.  Host only. */
+int pab_schedule_count(const pab_plan* plan, int kind, int* computes);
+
+/* Run attention `kind` for diffusion step `step` under the schedule.
+ *  Compute step: runs the kind's kernel on cuda_stream into one of the
+ *    plan's two output slots of that kind and sets *out to it.
+ *    Shapes: SPATIAL q,k,v [T, N, C]; TEMPORAL q,k,v [N, T, C];
+ *    CROSS q [T*N, C], k,v [text_len, C].  *out has q's layout.
+ *  Broadcast hit: launches nothing, copies nothing, ignores q, k, v (which
+ *    may be NULL) and sets *out to the slot that holds the output of the
+ *    kind's latest compute (bit-identical to it).
+ * Element type: the plan's dtype.  Steps of one kind must be strictly
+ * increasing (else PAB_ERR_STEP_ORDER); a hit whose source step was not the
+ * kind's latest compute returns PAB_ERR_NO_CACHE.
+ * Lifetime: the pointer stays valid and unchanged until the SECOND following
+ * compute of the same kind is launched, or reset/destroy -- long enough to
+ * compare step i with step i-1. */
+int pab_attention(pab_plan* plan, int kind, int step, const void* q, const void* k,
+                  const void* v, const void** out, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAB_H */

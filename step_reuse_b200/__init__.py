@@ -1,0 +1,264 @@
+"""Python binding of libpab.so -- the B200 (sm_100a) Pyramid Attention
+Broadcast attention library.
+
+Argument marshalling only: every step of the attention stack runs in the
+library's CUDA kernels.  Tensors are torch CUDA tensors (PyTorch supplies the
+device memory and the stream); the calls go through the C ABI declared in
+include/pab.h with ctypes.  Importing this package fails loudly if
+libpab.so has not been built (python -m step_reuse_b200.build); there is no
+CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpab.so")
+
+PAB_OK = 0
+PAB_ERR_ARG = -1
+PAB_ERR_STEP_ORDER = -2
+PAB_ERR_NO_CACHE = -3
+PAB_ERR_CUDA = -4
+PAB_ERR_OOM = -5
+PAB_ERR_UNSUPPORTED = -6
+
+SPATIAL, TEMPORAL, CROSS = 0, 1, 2
+KIND = {"spatial": SPATIAL, "temporal": TEMPORAL, "cross": CROSS}
+BF16, FP32 = 0, 1
+
+# every symbol include/pab.h declares
+EXPORTS = (
+    "pab_version", "pab_last_error_string", "pab_spatial_attention", "pab_temporal_attention",
+    "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async",
+    "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
+    "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
+    "pab_attention",
+)
+
+
+class PabError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"[{code}] {msg}")
+        self.code = code
+
+
+class pab_ranges(ctypes.Structure):
+    _fields_ = [("spatial", ctypes.c_int), ("temporal", ctypes.c_int), ("cross", ctypes.c_int),
+                ("edge_pct", ctypes.c_int)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m step_reuse_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
+    sig = {
+        "pab_version": ([], i),
+        "pab_last_error_string": ([], ctypes.c_char_p),
+        "pab_spatial_attention": ([vp, vp, vp, vp, i, i, i, i, vp], i),
+        "pab_temporal_attention": ([vp, vp, vp, vp, i, i, i, i, vp], i),
+        "pab_cross_attention": ([vp, vp, vp, vp, ll, i, i, i, vp], i),
+        "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
+        "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
+        "pab_attn_diff_mse_async": ([vp, vp, ll, i, vp, vp], i),
+        "pab_device_errors": ([i, ctypes.POINTER(ctypes.c_uint)], i),
+        "pab_plan_create": ([i, i, i, i, i, i, i, pab_ranges, i, ctypes.POINTER(vp)], i),
+        "pab_plan_destroy": ([vp], i),
+        "pab_plan_reset": ([vp], i),
+        "pab_plan_prepare": ([vp], i),
+        "pab_schedule_query": ([vp, i, i, ctypes.POINTER(i)], i),
+        "pab_schedule_source": ([vp, i, i, ctypes.POINTER(i)], i),
+        "pab_schedule_count": ([vp, i, ctypes.POINTER(i)], i),
+        "pab_attention": ([vp, i, i, vp, vp, vp, ctypes.POINTER(vp), vp], i),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    return lib
+
+
+lib = _load()
+
+
+def _check(rc: int):
+    if rc != PAB_OK:
+        raise PabError(rc, lib.pab_last_error_string().decode(errors="replace"))
+
+
+def _stream(stream=None):
+    if stream is None:
+        if not torch.cuda.is_available():
+            return None
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def version() -> int:
+    return lib.pab_version()
+
+
+def spatial_attention(q, k, v, heads: int, out=None, stream=None):
+    """q, k, v: [T, N, C] bf16 CUDA tensors -> [T, N, C]."""
+    T, N, C = q.shape
+    out = torch.empty_like(q) if out is None else out
+    _check(lib.pab_spatial_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), T, N, heads, C // heads,
+                                     _stream(stream)))
+    return out
+
+
+def temporal_attention(q, k, v, heads: int, out=None, stream=None):
+    """q, k, v: [N, T, C] bf16 CUDA tensors -> [N, T, C]."""
+    N, T, C = q.shape
+    out = torch.empty_like(q) if out is None else out
+    _check(lib.pab_temporal_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), N, T, heads, C // heads,
+                                      _stream(stream)))
+    return out
+
+
+def cross_attention(q, kt, vt, heads: int, out=None, stream=None):
+    """q: [..., C] video tokens; kt, vt: [text_len, C] -> like q."""
+    C = q.shape[-1]
+    R = q.numel() // C
+    out = torch.empty_like(q) if out is None else out
+    _check(lib.pab_cross_attention(_ptr(q), _ptr(kt), _ptr(vt), _ptr(out), R, kt.shape[0], heads,
+                                   C // heads, _stream(stream)))
+    return out
+
+
+def layout(x, to_temporal: bool, out=None, stream=None):
+    """[T, N, C] -> [N, T, C] when to_temporal, else [N, T, C] -> [T, N, C]."""
+    A, B, C = x.shape
+    out = x.new_empty((B, A, C)) if out is None else out
+    T, N = (A, B) if to_temporal else (B, A)
+    _check(lib.pab_layout(1 if to_temporal else 0, _ptr(x), _ptr(out), T, N, C, _dtype_code(x),
+                          _stream(stream)))
+    return out
+
+
+def attn_diff_mse(a, b, stream=None) -> float:
+    """mean((a - b)^2) over all elements, fp64; synchronises the stream."""
+    assert a.shape == b.shape and a.dtype == b.dtype
+    res = ctypes.c_double(0.0)
+    _check(lib.pab_attn_diff_mse(_ptr(a), _ptr(b), a.numel(), _dtype_code(a), ctypes.byref(res),
+                                 _stream(stream)))
+    return res.value
+
+
+def attn_diff_mse_async(a, b, result_dev, stream=None):
+    """Writes mean((a - b)^2) into the fp64 device scalar `result_dev`."""
+    assert a.shape == b.shape and a.dtype == b.dtype and result_dev.dtype == torch.float64
+    _check(lib.pab_attn_diff_mse_async(_ptr(a), _ptr(b), a.numel(), _dtype_code(a),
+                                       ctypes.c_void_p(result_dev.data_ptr()), _stream(stream)))
+    return result_dev
+
+
+def device_errors(clear: bool = True) -> int:
+    flags = ctypes.c_uint(0)
+    _check(lib.pab_device_errors(1 if clear else 0, ctypes.byref(flags)))
+    return flags.value
+
+
+class _DeviceView:
+    """__cuda_array_interface__ wrapper so torch can view library-owned memory."""
+
+    def __init__(self, ptr: int, shape, typestr: str):
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr,
+                                         "data": (ptr, False), "version": 3, "strides": None}
+
+
+def _wrap(ptr: int, shape, dtype, device) -> torch.Tensor:
+    if dtype == torch.bfloat16:
+        t = torch.as_tensor(_DeviceView(ptr, shape, "<i2"), device=device)
+        return t.view(torch.bfloat16)
+    return torch.as_tensor(_DeviceView(ptr, shape, "<f4"), device=device)
+
+
+class Plan:
+    """A PAB plan: the broadcast schedule of one sampling run plus the
+    broadcast cache (two output slots per kind, owned by the library).
+
+    Tensors returned by attention() VIEW library memory: they stay valid until
+    the second following compute of the same kind, reset() or close()."""
+
+    def __init__(self, T, H, W, heads, d, text_len, steps, ranges, dtype=torch.bfloat16,
+                 edge_pct: int = 0):
+        self.T, self.H, self.W, self.heads, self.d = T, H, W, heads, d
+        self.N, self.C, self.text_len, self.steps = H * W, heads * d, text_len, steps
+        self.dtype = dtype
+        r = pab_ranges(int(ranges[0]), int(ranges[1]), int(ranges[2]), int(edge_pct))
+        h = ctypes.c_void_p()
+        _check(lib.pab_plan_create(T, H, W, heads, d, text_len, steps, r,
+                                   FP32 if dtype == torch.float32 else BF16, ctypes.byref(h)))
+        self._h = h
+
+    def close(self):
+        if self._h:
+            lib.pab_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def reset(self):
+        _check(lib.pab_plan_reset(self._h))
+
+    def prepare(self):
+        _check(lib.pab_plan_prepare(self._h))
+
+    def is_compute(self, kind, step: int) -> bool:
+        kind = KIND.get(kind, kind)
+        out = ctypes.c_int(0)
+        _check(lib.pab_schedule_query(self._h, kind, step, ctypes.byref(out)))
+        return bool(out.value)
+
+    def source(self, kind, step: int) -> int:
+        kind = KIND.get(kind, kind)
+        out = ctypes.c_int(0)
+        _check(lib.pab_schedule_source(self._h, kind, step, ctypes.byref(out)))
+        return out.value
+
+    def count(self, kind) -> int:
+        kind = KIND.get(kind, kind)
+        out = ctypes.c_int(0)
+        _check(lib.pab_schedule_count(self._h, kind, ctypes.byref(out)))
+        return out.value
+
+    def attention_ptr(self, kind, step: int, q=None, k=None, v=None, stream=None) -> int:
+        """Raw device pointer of the step's output (compute or broadcast hit)."""
+        kind = KIND.get(kind, kind)
+        out = ctypes.c_void_p()
+        _check(lib.pab_attention(self._h, kind, step, _ptr(q), _ptr(k), _ptr(v), ctypes.byref(out),
+                                 _stream(stream)))
+        return out.value
+
+    def attention(self, kind, step: int, q=None, k=None, v=None, stream=None) -> torch.Tensor:
+        kind = KIND.get(kind, kind)
+        ptr = self.attention_ptr(kind, step, q, k, v, stream)
+        shape = {SPATIAL: (self.T, self.N, self.C), TEMPORAL: (self.N, self.T, self.C),
+                 CROSS: (self.T * self.N, self.C)}[kind]
+        dev = q.device if q is not None else torch.device("cuda", torch.cuda.current_device())
+        return _wrap(ptr, shape, self.dtype, dev)

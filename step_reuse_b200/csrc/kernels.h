@@ -1,0 +1,40 @@
+// kernels.h -- host-side launchers of the sm_100a kernels (internal to the
+// library; the public ABI is include/pab.h).  Each launcher validates nothing
+// beyond what its kernel needs: argument checks live in pab_api.cu.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace pab {
+
+// Streaming multiprocessors of the current device (cached per device).
+int device_sm_count();
+
+// --- attention-difference MSE (two passes, fp64, deterministic) ----------
+// Number of first-pass partial sums used for n elements on this device.
+int mse_num_partials(long long n, int elem_size);
+cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, double* partials,
+                       int num_partials, double* result_dev, cudaStream_t s);
+
+// --- layout change [T,N,C] <-> [N,T,C] (bulk-copy engine) ----------------
+cudaError_t launch_layout(int to_temporal, const void* src, void* dst, int T, int N,
+                          int row_bytes, cudaStream_t s);
+unsigned int layout_device_errors(bool clear);
+
+// --- temporal short-sequence attention ([N,T,C], L = T) -------------------
+cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
+                            int heads, int d, cudaStream_t s);
+
+// --- flash attention for spatial (per frame) and cross (shared text K/V) --
+// Rows of batch b, head h: q + b*q_bstride + i*C + h*d (elements); likewise
+// k/v with kv_bstride (0 = shared K/V).  out has q's layout.
+cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches,
+                         long long Lq, int Lk, int heads, int d, long long q_bstride,
+                         long long kv_bstride, cudaStream_t s);
+
+// --- dtype conversion for fp32 plans --------------------------------------
+cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t s);
+cudaError_t launch_bf16_to_f32(const void* src, float* dst, long long n, cudaStream_t s);
+
+}  // namespace pab

@@ -1,0 +1,157 @@
+// mse.cu -- attention-difference diagnostic: mean over all elements of
+// (a - b)^2 between two attention outputs (PAB report, Fig. 1: the
+// difference between consecutive diffusion steps' attention outputs,
+// quantified by MSE).
+//
+// HBM-bound: each element is read once from each tensor (2 x size bytes).
+// Pass 1: a grid of (SM count x 4) blocks streams 16-byte vectors with a
+// grid-stride loop, accumulates (a - b)^2 in fp64 per thread, reduces each
+// warp with shuffles and each block through shared memory, and writes one
+// fp64 partial per block.  Pass 2: one block sums the partials in a fixed
+// order and divides by n.  The split depends only on n and the SM count, so
+// the result is bitwise reproducible on a given device.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pab {
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kUnroll = 4;
+
+template <typename T>
+struct Vec;  // 16 bytes of T
+template <>
+struct Vec<__nv_bfloat16> {
+    static constexpr int kElems = 8;
+    PAB_DEV static double sq_sum(const uint4& a, const uint4& b) {
+        const __nv_bfloat162* pa = reinterpret_cast<const __nv_bfloat162*>(&a);
+        const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&b);
+        double acc = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float2 fa = __bfloat1622float2(pa[i]);
+            const float2 fb = __bfloat1622float2(pb[i]);
+            const double d0 = (double)(fa.x - fb.x);
+            const double d1 = (double)(fa.y - fb.y);
+            acc = fma(d0, d0, acc);
+            acc = fma(d1, d1, acc);
+        }
+        return acc;
+    }
+    PAB_DEV static double sq_one(const __nv_bfloat16* a, const __nv_bfloat16* b, long long i) {
+        const double d = (double)(__bfloat162float(a[i]) - __bfloat162float(b[i]));
+        return d * d;
+    }
+};
+template <>
+struct Vec<float> {
+    static constexpr int kElems = 4;
+    PAB_DEV static double sq_sum(const uint4& a, const uint4& b) {
+        const float* fa = reinterpret_cast<const float*>(&a);
+        const float* fb = reinterpret_cast<const float*>(&b);
+        double acc = 0.0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const double d = (double)fa[i] - (double)fb[i];
+            acc = fma(d, d, acc);
+        }
+        return acc;
+    }
+    PAB_DEV static double sq_one(const float* a, const float* b, long long i) {
+        const double d = (double)a[i] - (double)b[i];
+        return d * d;
+    }
+};
+
+PAB_DEV double warp_sum(double x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Fixed-order block reduction; every thread passes its value, thread 0 gets the sum.
+PAB_DEV double block_sum(double x, double* red) {
+    x = warp_sum(x);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) red[warp] = x;
+    __syncthreads();
+    double s = 0.0;
+    if (warp == 0) {
+        s = (lane < (int)(blockDim.x >> 5)) ? red[lane] : 0.0;
+        s = warp_sum(s);
+    }
+    return s;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) mse_partials_kernel(const T* __restrict__ a,
+                                                                const T* __restrict__ b,
+                                                                long long n,
+                                                                double* __restrict__ partials) {
+    __shared__ double red[kThreads / 32];
+    constexpr int E = Vec<T>::kElems;
+    const long long nvec = n / E;
+    const uint4* va = reinterpret_cast<const uint4*>(a);
+    const uint4* vb = reinterpret_cast<const uint4*>(b);
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    double acc = 0.0;
+    // unrolled body: kUnroll independent 16-byte loads per tensor in flight
+    for (; i + (kUnroll - 1) * stride < nvec; i += kUnroll * stride) {
+        uint4 ra[kUnroll], rb[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+            ra[u] = __ldcs(va + i + u * stride);
+            rb[u] = __ldcs(vb + i + u * stride);
+        }
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) acc += Vec<T>::sq_sum(ra[u], rb[u]);
+    }
+    for (; i < nvec; i += stride) acc += Vec<T>::sq_sum(__ldcs(va + i), __ldcs(vb + i));
+    // scalar tail (n not a multiple of the vector width): block 0 only
+    if (blockIdx.x == 0) {
+        const long long t = nvec * E + threadIdx.x;
+        if (t < n) acc += Vec<T>::sq_one(a, b, t);
+    }
+    const double s = block_sum(acc, red);
+    if (threadIdx.x == 0) partials[blockIdx.x] = s;
+}
+
+__global__ void __launch_bounds__(kThreads) mse_final_kernel(const double* __restrict__ partials,
+                                                             int count, long long n,
+                                                             double* __restrict__ result) {
+    __shared__ double red[kThreads / 32];
+    double acc = 0.0;
+    for (int i = threadIdx.x; i < count; i += blockDim.x) acc += partials[i];
+    const double s = block_sum(acc, red);
+    if (threadIdx.x == 0) *result = (n > 0) ? s / (double)n : 0.0;
+}
+
+}  // namespace
+
+int mse_num_partials(long long n, int elem_size) {
+    const long long nvec = n * elem_size / 16;
+    const long long per_block = (long long)kThreads * kUnroll;
+    long long blocks = (nvec + per_block - 1) / per_block;
+    const long long cap = (long long)device_sm_count() * 4;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    return (int)blocks;
+}
+
+cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, double* partials,
+                       int num_partials, double* result_dev, cudaStream_t s) {
+    if (dtype == 1)
+        mse_partials_kernel<float><<<num_partials, kThreads, 0, s>>>(
+            static_cast<const float*>(a), static_cast<const float*>(b), n, partials);
+    else
+        mse_partials_kernel<__nv_bfloat16><<<num_partials, kThreads, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(a), static_cast<const __nv_bfloat16*>(b), n, partials);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    mse_final_kernel<<<1, kThreads, 0, s>>>(partials, num_partials, n, result_dev);
+    return cudaGetLastError();
+}
+
+}  // namespace pab

@@ -1,0 +1,517 @@
+// pab_api.cu -- the C ABI of include/pab.h: argument checks, error
+// reporting, the Pyramid Attention Broadcast plan (schedule + broadcast
+// cache) and dispatch to the sm_100a kernels.
+//
+// Schedule (PAB report, "Implementation" and Fig. 2; paper abstract): the
+// first and last edge_pct% of the diffusion steps compute every attention;
+// in the middle segment each kind computes at the first step of every window
+// of r_kind steps and the other r_kind - 1 steps are broadcast hits.  With
+// e = ceil(edge_pct * steps / 100), lo = e, hi = steps - e:
+//     compute(i)  <=>  i < lo  or  i >= hi  or  (i - lo) % r == 0
+//     source(i)   =    i if compute(i) else lo + ((i - lo) / r) * r.
+// Broadcast cache: two output slots per kind.  A compute writes the slot
+// that does not hold the latest output, then becomes the latest; a hit
+// returns the latest slot's pointer (no launch, no copy).
+#include <mutex>
+#include <new>
+#include <string>
+#include <vector>
+
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "../../include/pab.h"
+#include "kernels.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
+int cuda_fail(cudaError_t e, const char* what) {
+    const int code = (e == cudaErrorMemoryAllocation) ? PAB_ERR_OOM : PAB_ERR_CUDA;
+    return fail(code, "%s: %s (%s)", what, cudaGetErrorString(e), cudaGetErrorName(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr int kMaxDevices = 64;
+
+// Per-device scratch for the MSE first pass: fp64 partials + one result slot.
+struct MseScratch {
+    double* buf = nullptr;
+    int capacity = 0;  // doubles
+};
+std::mutex g_scratch_mu;
+MseScratch g_mse_scratch[kMaxDevices];
+
+int current_device(int* dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    if (*dev < 0 || *dev >= kMaxDevices) return fail(PAB_ERR_UNSUPPORTED, "device index %d", *dev);
+    return PAB_OK;
+}
+
+int mse_scratch(int need, double** out) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lk(g_scratch_mu);
+    MseScratch& s = g_mse_scratch[dev];
+    if (s.capacity < need) {
+        if (s.buf) cudaFree(s.buf);
+        s.buf = nullptr;
+        s.capacity = 0;
+        cudaError_t e = cudaMalloc(&s.buf, sizeof(double) * (size_t)need);
+        if (e != cudaSuccess) return cuda_fail(e, "MSE scratch allocation");
+        s.capacity = need;
+    }
+    *out = s.buf;
+    return PAB_OK;
+}
+
+int check_dims(int heads, int d) {
+    if (heads <= 0 || d <= 0) return fail(PAB_ERR_ARG, "heads (%d) and d (%d) must be positive", heads, d);
+    if (d % 8 != 0 || d > 128)
+        return fail(PAB_ERR_UNSUPPORTED, "head dim %d unsupported (need d %% 8 == 0, d <= 128)", d);
+    return PAB_OK;
+}
+
+int check_ptrs(const char* names, const void* a, const void* b, const void* c, const void* o) {
+    const void* ps[4] = {a, b, c, o};
+    for (int i = 0; i < 4; ++i) {
+        if (!ps[i]) return fail(PAB_ERR_ARG, "null device pointer among (%s)", names);
+        if (!aligned16(ps[i])) return fail(PAB_ERR_ARG, "device pointer among (%s) not 16-byte aligned", names);
+    }
+    return PAB_OK;
+}
+
+int run_spatial(const void* q, const void* k, const void* v, void* out, int T, int N, int heads,
+                int d, cudaStream_t s) {
+    const long long C = (long long)heads * d;
+    cudaError_t e = pab::launch_flash(q, k, v, out, T, N, N, heads, d, (long long)N * C,
+                                      (long long)N * C, s);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "spatial attention launch");
+}
+
+int run_temporal(const void* q, const void* k, const void* v, void* out, int N, int T, int heads,
+                 int d, cudaStream_t s) {
+    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, s);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "temporal attention launch");
+}
+
+int run_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lt,
+              int heads, int d, cudaStream_t s) {
+    cudaError_t e = pab::launch_flash(q, kt, vt, out, 1, R, Lt, heads, d, 0, 0, s);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "cross attention launch");
+}
+
+}  // namespace
+
+namespace pab {
+int device_sm_count() {
+    static int cache[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+    if (cache[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+}  // namespace pab
+
+// ============================================================== plan
+struct pab_plan {
+    int T, H, W, N, heads, d, text_len, steps, dtype;
+    long long C;
+    int range[3];
+    int edge_pct, lo, hi;
+    // cache
+    int device;
+    void* slot[3][2];
+    size_t slot_bytes[3];
+    int cur[3];          // slot holding the latest computed output, -1 = none
+    int cached_step[3];  // step of that compute
+    int last_step[3];    // last step seen (order check)
+    // bf16 staging for fp32 plans
+    void* stage_in[3];
+    void* stage_out;
+    size_t stage_in_bytes, stage_out_bytes;
+};
+
+namespace {
+
+bool sched_compute(const pab_plan* p, int kind, int i) {
+    if (i < p->lo || i >= p->hi) return true;
+    return ((i - p->lo) % p->range[kind]) == 0;
+}
+int sched_source(const pab_plan* p, int kind, int i) {
+    if (sched_compute(p, kind, i)) return i;
+    return p->lo + ((i - p->lo) / p->range[kind]) * p->range[kind];
+}
+
+void plan_free_device(pab_plan* p) {
+    for (int k = 0; k < 3; ++k)
+        for (int j = 0; j < 2; ++j) {
+            if (p->slot[k][j]) cudaFree(p->slot[k][j]);
+            p->slot[k][j] = nullptr;
+        }
+    for (int j = 0; j < 3; ++j) {
+        if (p->stage_in[j]) cudaFree(p->stage_in[j]);
+        p->stage_in[j] = nullptr;
+    }
+    if (p->stage_out) cudaFree(p->stage_out);
+    p->stage_out = nullptr;
+    p->device = -1;
+}
+
+int plan_alloc_kind(pab_plan* p, int kind) {
+    int dev;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    if (p->device >= 0 && p->device != dev)
+        return fail(PAB_ERR_ARG, "plan's cache lives on device %d, current device is %d", p->device, dev);
+    p->device = dev;
+    for (int j = 0; j < 2; ++j)
+        if (!p->slot[kind][j] && p->slot_bytes[kind] > 0) {
+            cudaError_t e = cudaMalloc(&p->slot[kind][j], p->slot_bytes[kind]);
+            if (e != cudaSuccess) return cuda_fail(e, "broadcast cache allocation");
+        }
+    if (p->dtype == PAB_FP32) {
+        for (int j = 0; j < 3; ++j)
+            if (!p->stage_in[j] && p->stage_in_bytes > 0) {
+                cudaError_t e = cudaMalloc(&p->stage_in[j], p->stage_in_bytes);
+                if (e != cudaSuccess) return cuda_fail(e, "bf16 staging allocation");
+            }
+        if (!p->stage_out && p->stage_out_bytes > 0) {
+            cudaError_t e = cudaMalloc(&p->stage_out, p->stage_out_bytes);
+            if (e != cudaSuccess) return cuda_fail(e, "bf16 staging allocation");
+        }
+    }
+    return PAB_OK;
+}
+
+int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void* v, void* out,
+                 cudaStream_t s) {
+    const long long qn = (long long)p->T * p->N * p->C;
+    const long long kvn = (kind == PAB_CROSS) ? (long long)p->text_len * p->C : qn;
+    const void *qq = q, *kk = k, *vv = v;
+    void* oo = out;
+    if (p->dtype == PAB_FP32) {
+        const float* src[3] = {static_cast<const float*>(q), static_cast<const float*>(k),
+                               static_cast<const float*>(v)};
+        const long long cnt[3] = {qn, kvn, kvn};
+        for (int j = 0; j < 3; ++j) {
+            cudaError_t e = pab::launch_f32_to_bf16(src[j], p->stage_in[j], cnt[j], s);
+            if (e != cudaSuccess) return cuda_fail(e, "fp32 -> bf16 conversion");
+        }
+        qq = p->stage_in[0];
+        kk = p->stage_in[1];
+        vv = p->stage_in[2];
+        oo = p->stage_out;
+    }
+    int rc;
+    if (kind == PAB_SPATIAL)
+        rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s);
+    else if (kind == PAB_TEMPORAL)
+        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, s);
+    else
+        rc = run_cross(qq, kk, vv, oo, (long long)p->T * p->N, p->text_len, p->heads, p->d, s);
+    if (rc) return rc;
+    if (p->dtype == PAB_FP32) {
+        cudaError_t e = pab::launch_bf16_to_f32(p->stage_out, static_cast<float*>(out), qn, s);
+        if (e != cudaSuccess) return cuda_fail(e, "bf16 -> fp32 conversion");
+    }
+    return PAB_OK;
+}
+
+}  // namespace
+
+#define PAB_GUARD_BEGIN try {
+#define PAB_GUARD_END                                                   \
+    }                                                                   \
+    catch (const std::bad_alloc&) {                                     \
+        return fail(PAB_ERR_OOM, "host allocation failed");             \
+    }                                                                   \
+    catch (...) {                                                       \
+        return fail(PAB_ERR_ARG, "unexpected host exception");          \
+    }
+
+extern "C" {
+
+int pab_version(void) { return (0 << 16) | 1; }
+
+const char* pab_last_error_string(void) { return g_last_error.c_str(); }
+
+int pab_spatial_attention(const void* q, const void* k, const void* v, void* out, int T, int N,
+                          int heads, int d, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || N < 0) return fail(PAB_ERR_ARG, "T (%d) and N (%d) must be >= 0", T, N);
+    if ((long long)T * N == 0) return PAB_OK;
+    if (T > 65535) return fail(PAB_ERR_UNSUPPORTED, "T=%d frames exceeds 65535", T);
+    rc = check_ptrs("q, k, v, out", q, k, v, out);
+    if (rc) return rc;
+    return run_spatial(q, k, v, out, T, N, heads, d, static_cast<cudaStream_t>(cuda_stream));
+    PAB_GUARD_END
+}
+
+int pab_temporal_attention(const void* q, const void* k, const void* v, void* out, int N, int T,
+                           int heads, int d, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || N < 0) return fail(PAB_ERR_ARG, "T (%d) and N (%d) must be >= 0", T, N);
+    if (T > 128) return fail(PAB_ERR_UNSUPPORTED, "temporal length T=%d exceeds 128", T);
+    if ((long long)T * N == 0) return PAB_OK;
+    rc = check_ptrs("q, k, v, out", q, k, v, out);
+    if (rc) return rc;
+    return run_temporal(q, k, v, out, N, T, heads, d, static_cast<cudaStream_t>(cuda_stream));
+    PAB_GUARD_END
+}
+
+int pab_cross_attention(const void* q, const void* kt, const void* vt, void* out, long long R,
+                        int text_len, int heads, int d, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (R < 0) return fail(PAB_ERR_ARG, "R=%lld must be >= 0", R);
+    if (text_len < 1 || text_len > 512)
+        return fail(PAB_ERR_UNSUPPORTED, "text_len=%d outside [1, 512]", text_len);
+    if (R == 0) return PAB_OK;
+    rc = check_ptrs("q, kt, vt, out", q, kt, vt, out);
+    if (rc) return rc;
+    return run_cross(q, kt, vt, out, R, text_len, heads, d, static_cast<cudaStream_t>(cuda_stream));
+    PAB_GUARD_END
+}
+
+int pab_layout(int to_temporal, const void* src, void* dst, int T, int N, int C, int dtype,
+               void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (dtype != PAB_BF16 && dtype != PAB_FP32) return fail(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (T < 0 || N < 0 || C < 0) return fail(PAB_ERR_ARG, "negative size");
+    const int elem = dtype == PAB_FP32 ? 4 : 2;
+    const long long row = (long long)C * elem;
+    if ((long long)T * N * C == 0) return PAB_OK;
+    if (row % 16 != 0) return fail(PAB_ERR_UNSUPPORTED, "row of %lld bytes is not a multiple of 16", row);
+    if (row > 48 * 1024) return fail(PAB_ERR_UNSUPPORTED, "row of %lld bytes exceeds 48 KiB", row);
+    if (!src || !dst) return fail(PAB_ERR_ARG, "null src/dst");
+    if (!aligned16(src) || !aligned16(dst)) return fail(PAB_ERR_ARG, "src/dst not 16-byte aligned");
+    const char* s0 = static_cast<const char*>(src);
+    const char* d0 = static_cast<const char*>(dst);
+    const long long bytes = (long long)T * N * row;
+    if (s0 < d0 + bytes && d0 < s0 + bytes) return fail(PAB_ERR_ARG, "src and dst overlap");
+    cudaError_t e = pab::launch_layout(to_temporal ? 1 : 0, src, dst, T, N, (int)row,
+                                       static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "layout launch");
+    PAB_GUARD_END
+}
+
+int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype, double* result_dev,
+                            void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (dtype != PAB_BF16 && dtype != PAB_FP32) return fail(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (n < 0) return fail(PAB_ERR_ARG, "n=%lld must be >= 0", n);
+    if (!result_dev || (reinterpret_cast<uintptr_t>(result_dev) & 7u))
+        return fail(PAB_ERR_ARG, "result_dev null or not 8-byte aligned");
+    if (n > 0 && (!a || !b)) return fail(PAB_ERR_ARG, "null input");
+    if (n > 0 && (!aligned16(a) || !aligned16(b))) return fail(PAB_ERR_ARG, "inputs not 16-byte aligned");
+    const int elem = dtype == PAB_FP32 ? 4 : 2;
+    const int parts = pab::mse_num_partials(n, elem);
+    double* scratch = nullptr;
+    int rc = mse_scratch(parts + 1, &scratch);
+    if (rc) return rc;
+    cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, result_dev,
+                                    static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "MSE launch");
+    PAB_GUARD_END
+}
+
+int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype, double* result,
+                      void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (!result) return fail(PAB_ERR_ARG, "null result pointer");
+    if (dtype != PAB_BF16 && dtype != PAB_FP32) return fail(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (n < 0) return fail(PAB_ERR_ARG, "n=%lld must be >= 0", n);
+    if (n > 0 && (!a || !b)) return fail(PAB_ERR_ARG, "null input");
+    if (n > 0 && (!aligned16(a) || !aligned16(b))) return fail(PAB_ERR_ARG, "inputs not 16-byte aligned");
+    const int elem = dtype == PAB_FP32 ? 4 : 2;
+    const int parts = pab::mse_num_partials(n, elem);
+    double* scratch = nullptr;
+    int rc = mse_scratch(parts + 1, &scratch);
+    if (rc) return rc;
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, scratch + parts, s);
+    if (e != cudaSuccess) return cuda_fail(e, "MSE launch");
+    e = cudaMemcpyAsync(result, scratch + parts, sizeof(double), cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return cuda_fail(e, "MSE result copy");
+    e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return cuda_fail(e, "MSE stream synchronise");
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+int pab_device_errors(int clear, unsigned int* flags) {
+    PAB_GUARD_BEGIN
+    if (!flags) return fail(PAB_ERR_ARG, "null flags pointer");
+    const unsigned int v = pab::layout_device_errors(clear != 0);
+    if (v == 0xffffffffu) return fail(PAB_ERR_CUDA, "could not read the device status word");
+    *flags = v;
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+int pab_plan_create(int T, int H, int W, int heads, int d, int text_len, int steps,
+                    pab_ranges ranges, int dtype, pab_plan** out_plan) {
+    PAB_GUARD_BEGIN
+    if (!out_plan) return fail(PAB_ERR_ARG, "null out_plan");
+    *out_plan = nullptr;
+    if (T < 1 || H < 1 || W < 1) return fail(PAB_ERR_ARG, "T, H, W must be >= 1 (got %d, %d, %d)", T, H, W);
+    if (steps < 1) return fail(PAB_ERR_ARG, "steps=%d must be >= 1", steps);
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (text_len < 1 || text_len > 512) return fail(PAB_ERR_UNSUPPORTED, "text_len=%d outside [1, 512]", text_len);
+    if (T > 128) return fail(PAB_ERR_UNSUPPORTED, "T=%d frames exceeds the temporal limit 128", T);
+    if (dtype != PAB_BF16 && dtype != PAB_FP32) return fail(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (ranges.spatial < 1 || ranges.temporal < 1 || ranges.cross < 1)
+        return fail(PAB_ERR_ARG, "broadcast ranges must be >= 1 (got %d, %d, %d)", ranges.spatial,
+                    ranges.temporal, ranges.cross);
+    const int edge = ranges.edge_pct == 0 ? 15 : ranges.edge_pct;
+    if (edge < 0 || edge > 50) return fail(PAB_ERR_ARG, "edge_pct=%d outside [0, 50]", ranges.edge_pct);
+    const long long N = (long long)H * W;
+    if (N > (1LL << 30)) return fail(PAB_ERR_UNSUPPORTED, "H*W too large");
+    pab_plan* p = new pab_plan;
+    memset(p, 0, sizeof(*p));
+    p->T = T;
+    p->H = H;
+    p->W = W;
+    p->N = (int)N;
+    p->heads = heads;
+    p->d = d;
+    p->C = (long long)heads * d;
+    p->text_len = text_len;
+    p->steps = steps;
+    p->dtype = dtype;
+    p->range[PAB_SPATIAL] = ranges.spatial;
+    p->range[PAB_TEMPORAL] = ranges.temporal;
+    p->range[PAB_CROSS] = ranges.cross;
+    p->edge_pct = edge;
+    const int e = (edge * steps + 99) / 100;
+    p->lo = e;
+    p->hi = steps - e;
+    p->device = -1;
+    const size_t elem = dtype == PAB_FP32 ? 4 : 2;
+    const size_t video = (size_t)T * N * p->C;
+    for (int k = 0; k < 3; ++k) {
+        p->slot_bytes[k] = video * elem;
+        p->cur[k] = -1;
+        p->cached_step[k] = -1;
+        p->last_step[k] = -1;
+    }
+    p->stage_in_bytes = video * 2;
+    p->stage_out_bytes = video * 2;
+    *out_plan = p;
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+int pab_plan_destroy(pab_plan* plan) {
+    if (!plan) return PAB_OK;
+    plan_free_device(plan);
+    delete plan;
+    return PAB_OK;
+}
+
+int pab_plan_reset(pab_plan* plan) {
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    for (int k = 0; k < 3; ++k) {
+        plan->cur[k] = -1;
+        plan->cached_step[k] = -1;
+        plan->last_step[k] = -1;
+    }
+    return PAB_OK;
+}
+
+int pab_plan_prepare(pab_plan* plan) {
+    PAB_GUARD_BEGIN
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    for (int k = 0; k < 3; ++k) {
+        int rc = plan_alloc_kind(plan, k);
+        if (rc) return rc;
+    }
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+int pab_schedule_query(const pab_plan* plan, int kind, int step, int* is_compute) {
+    if (!plan || !is_compute) return fail(PAB_ERR_ARG, "null argument");
+    if (kind < 0 || kind > 2) return fail(PAB_ERR_ARG, "bad kind %d", kind);
+    if (step < 0 || step >= plan->steps) return fail(PAB_ERR_ARG, "step %d outside [0, %d)", step, plan->steps);
+    *is_compute = sched_compute(plan, kind, step) ? 1 : 0;
+    return PAB_OK;
+}
+
+int pab_schedule_source(const pab_plan* plan, int kind, int step, int* source_step) {
+    if (!plan || !source_step) return fail(PAB_ERR_ARG, "null argument");
+    if (kind < 0 || kind > 2) return fail(PAB_ERR_ARG, "bad kind %d", kind);
+    if (step < 0 || step >= plan->steps) return fail(PAB_ERR_ARG, "step %d outside [0, %d)", step, plan->steps);
+    *source_step = sched_source(plan, kind, step);
+    return PAB_OK;
+}
+
+int pab_schedule_count(const pab_plan* plan, int kind, int* computes) {
+    if (!plan || !computes) return fail(PAB_ERR_ARG, "null argument");
+    if (kind < 0 || kind > 2) return fail(PAB_ERR_ARG, "bad kind %d", kind);
+    int c = 0;
+    for (int i = 0; i < plan->steps; ++i) c += sched_compute(plan, kind, i) ? 1 : 0;
+    *computes = c;
+    return PAB_OK;
+}
+
+int pab_attention(pab_plan* plan, int kind, int step, const void* q, const void* k, const void* v,
+                  const void** out, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (!plan || !out) return fail(PAB_ERR_ARG, "null plan or out");
+    if (kind < 0 || kind > 2) return fail(PAB_ERR_ARG, "bad kind %d", kind);
+    if (step < 0 || step >= plan->steps) return fail(PAB_ERR_ARG, "step %d outside [0, %d)", step, plan->steps);
+    if (step <= plan->last_step[kind])
+        return fail(PAB_ERR_STEP_ORDER, "kind %d: step %d after step %d", kind, step, plan->last_step[kind]);
+    if (!sched_compute(plan, kind, step)) {
+        const int src = sched_source(plan, kind, step);
+        if (plan->cur[kind] < 0 || plan->cached_step[kind] != src)
+            return fail(PAB_ERR_NO_CACHE, "kind %d step %d needs the output of step %d, which was not computed",
+                        kind, step, src);
+        plan->last_step[kind] = step;
+        *out = plan->slot[kind][plan->cur[kind]];
+        return PAB_OK;
+    }
+    int rc = check_ptrs("q, k, v", q, k, v, q);
+    if (rc) return rc;
+    rc = plan_alloc_kind(plan, kind);
+    if (rc) return rc;
+    const int slot = plan->cur[kind] < 0 ? 0 : 1 - plan->cur[kind];
+    rc = plan_compute(plan, kind, q, k, v, plan->slot[kind][slot], static_cast<cudaStream_t>(cuda_stream));
+    if (rc) return rc;
+    plan->cur[kind] = slot;
+    plan->cached_step[kind] = step;
+    plan->last_step[kind] = step;
+    *out = plan->slot[kind][slot];
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+}  // extern "C"

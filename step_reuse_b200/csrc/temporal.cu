@@ -1,0 +1,291 @@
+// temporal.cu -- temporal attention: at every spatial position n and head h
+// the T frames attend to each other (PAB report, "Implementation": temporal
+// attention, the mid-frequency kind).  q, k, v, out: [N, T, C] (temporal
+// view), bf16.  L = T is short (16..64 in the workloads), the batch
+// (N * heads) is in the tens of thousands, so the kernel is HBM-bound
+// (2 * T * d * 2 flop per loaded byte ~ 8-32 flop/B).
+//
+// Design:
+//  - persistent grid; a unit of work is (position n, group of G heads); the
+//    unit's q, k, v rows (T rows of G*d contiguous channels each) stream into
+//    shared memory with 16-byte cp.async, double-buffered across units, so
+//    the next unit's loads overlap this unit's math;
+//  - one warp per (head, 16-query tile): QK^T and PV run on warp-level bf16
+//    MMA (m16n8k16, fp32 accumulate) from ldmatrix fragments; the softmax is
+//    an online (streaming) softmax over 16-key blocks with quad shuffles;
+//  - shared-memory rows have a pitch of P elements with P/8 odd, so the eight
+//    16-byte rows an ldmatrix phase reads hit distinct banks;
+//  - outputs are staged in the q buffer and written back with coalesced
+//    16-byte stores.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace pab {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxStageBytes = 56 * 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct TemporalArgs {
+    const __nv_bfloat16* q;
+    const __nv_bfloat16* k;
+    const __nv_bfloat16* v;
+    __nv_bfloat16* out;
+    int N, T, heads, d;
+    int G;       // heads per unit
+    int P;       // smem row pitch (elements)
+    int RT;      // rows per head block in smem (T rounded up to 16)
+    long long units;
+    float scale_log2;  // log2(e) / sqrt(d)
+};
+
+PAB_DEV float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// smem layout of one stage: [3 tensors][G heads][RT rows][P cols] bf16
+template <int DN>
+__global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs p) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    constexpr int DK = (DN + 1) / 2;  // 16-wide k chunks covering d
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int G = p.G, P = p.P, RT = p.RT, T = p.T, d = p.d;
+    const long long C = (long long)p.heads * d;
+    const int head_elems = RT * P;
+    const int tensor_elems = G * head_elems;
+    const int stage_elems = 3 * tensor_elems;
+    const int chunks_per_row = d / 8;
+    const int hg_count = p.heads / G;
+
+    // zero both stages once: padding rows/cols are never written afterwards
+    {
+        uint4* z = reinterpret_cast<uint4*>(smem);
+        const int n16 = (2 * stage_elems * 2 + 256) / 16;
+        for (int i = tid; i < n16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    __syncthreads();
+
+    __nv_bfloat16* sbase = reinterpret_cast<__nv_bfloat16*>(smem);
+    auto issue_unit = [&](long long unit, int stage) {
+        const long long n = unit / hg_count;
+        const int h0 = (int)(unit - n * hg_count) * G;
+        __nv_bfloat16* st = sbase + stage * stage_elems;
+        const int per_tensor = T * G * chunks_per_row;
+        for (int c = tid; c < 3 * per_tensor; c += kThreads) {
+            const int tsr = c / per_tensor;
+            int r = c - tsr * per_tensor;
+            const int t = r / (G * chunks_per_row);
+            r -= t * (G * chunks_per_row);
+            const int g = r / chunks_per_row;
+            const int ch = r - g * chunks_per_row;
+            const __nv_bfloat16* src = (tsr == 0 ? p.q : (tsr == 1 ? p.k : p.v)) +
+                                       ((n * T + t) * C + (long long)(h0 + g) * d + ch * 8);
+            __nv_bfloat16* dst = st + tsr * tensor_elems + g * head_elems + t * P + ch * 8;
+            cp_async16(smem_u32(dst), src, 16);
+        }
+    };
+
+    const long long first = blockIdx.x, step = gridDim.x;
+    if (first < p.units) issue_unit(first, 0);
+    cp_async_commit();
+
+    const int mtiles = RT / 16;
+    const int tasks = G * mtiles;
+    for (long long i = 0;; ++i) {
+        const long long u = first + i * step;
+        if (u >= p.units) break;
+        const int stage = (int)(i & 1);
+        const long long nu = u + step;
+        if (nu < p.units) issue_unit(nu, stage ^ 1);
+        cp_async_commit();
+        cp_async_wait<1>();
+        __syncthreads();
+
+        __nv_bfloat16* st = sbase + stage * stage_elems;
+        for (int task = warp; task < tasks; task += kWarps) {
+            const int g = task / mtiles, mt = task - (task / mtiles) * mtiles;
+            __nv_bfloat16* qs = st + g * head_elems + mt * 16 * P;
+            const __nv_bfloat16* ks = st + tensor_elems + g * head_elems;
+            const __nv_bfloat16* vs = st + 2 * tensor_elems + g * head_elems;
+
+            // Q fragments for this 16-row tile
+            uint32_t qa[DK][4];
+#pragma unroll
+            for (int kc = 0; kc < DK; ++kc)
+                ldsm_x4(smem_u32(qs + (lane & 15) * P + kc * 16 + (lane >> 4) * 8), qa[kc][0],
+                        qa[kc][1], qa[kc][2], qa[kc][3]);
+            if (DN & 1) {  // d % 16 == 8: the last chunk's upper 8 columns are past d
+                qa[DK - 1][2] = 0u;
+                qa[DK - 1][3] = 0u;
+            }
+            float o[DN][4];
+#pragma unroll
+            for (int j = 0; j < DN; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
+            float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+            for (int kb = 0; kb < mtiles; ++kb) {
+                float s[2][4];
+#pragma unroll
+                for (int j = 0; j < 2; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+                for (int kc = 0; kc < DK; ++kc) {
+                    uint32_t b0, b1, b2, b3;
+                    const int krow = kb * 16 + (lane & 7) + ((lane >> 4) << 3);
+                    const int kcol = kc * 16 + ((lane >> 3) & 1) * 8;
+                    ldsm_x4(smem_u32(ks + krow * P + kcol), b0, b1, b2, b3);
+                    mma_bf16_16816(s[0], qa[kc][0], qa[kc][1], qa[kc][2], qa[kc][3], b0, b1);
+                    mma_bf16_16816(s[1], qa[kc][0], qa[kc][1], qa[kc][2], qa[kc][3], b2, b3);
+                }
+                // scale, mask keys >= T, online softmax (rows r and r+8)
+                float mx0 = m0, mx1 = m1;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int key = kb * 16 + j * 8 + 2 * (lane & 3);
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const bool valid = (key + e) < T;
+                        s[j][e] = valid ? s[j][e] * p.scale_log2 : -INFINITY;
+                        s[j][2 + e] = valid ? s[j][2 + e] * p.scale_log2 : -INFINITY;
+                        mx0 = fmaxf(mx0, s[j][e]);
+                        mx1 = fmaxf(mx1, s[j][2 + e]);
+                    }
+                }
+                mx0 = quad_max(mx0);
+                mx1 = quad_max(mx1);
+                const float c0 = ex2(m0 - mx0), c1 = ex2(m1 - mx1);
+                m0 = mx0;
+                m1 = mx1;
+                float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        s[j][e] = ex2(s[j][e] - mx0);
+                        s[j][2 + e] = ex2(s[j][2 + e] - mx1);
+                        ps0 += s[j][e];
+                        ps1 += s[j][2 + e];
+                    }
+                }
+                l0 = l0 * c0 + ps0;
+                l1 = l1 * c1 + ps1;
+#pragma unroll
+                for (int j = 0; j < DN; ++j) {
+                    o[j][0] *= c0;
+                    o[j][1] *= c0;
+                    o[j][2] *= c1;
+                    o[j][3] *= c1;
+                }
+                const uint32_t pa0 = pack_bf16x2(s[0][0], s[0][1]);
+                const uint32_t pa1 = pack_bf16x2(s[0][2], s[0][3]);
+                const uint32_t pa2 = pack_bf16x2(s[1][0], s[1][1]);
+                const uint32_t pa3 = pack_bf16x2(s[1][2], s[1][3]);
+                const int vrow = kb * 16 + (lane & 7) + (((lane >> 3) & 1) << 3);
+#pragma unroll
+                for (int j = 0; j < DN; j += 2) {
+                    if (j + 1 < DN) {
+                        uint32_t b0, b1, b2, b3;
+                        ldsm_x4_t(smem_u32(vs + vrow * P + j * 8 + (lane >> 4) * 8), b0, b1, b2, b3);
+                        mma_bf16_16816(o[j], pa0, pa1, pa2, pa3, b0, b1);
+                        mma_bf16_16816(o[j + 1], pa0, pa1, pa2, pa3, b2, b3);
+                    } else {
+                        uint32_t b0, b1;
+                        ldsm_x2_t(smem_u32(vs + vrow * P + j * 8), b0, b1);
+                        mma_bf16_16816(o[j], pa0, pa1, pa2, pa3, b0, b1);
+                    }
+                }
+            }
+            l0 = quad_sum(l0);
+            l1 = quad_sum(l1);
+            const float inv0 = 1.f / l0, inv1 = 1.f / l1;
+            // stage O (bf16) over this warp's own q rows
+            const int r0 = lane >> 2, cq = 2 * (lane & 3);
+#pragma unroll
+            for (int j = 0; j < DN; ++j) {
+                *reinterpret_cast<uint32_t*>(qs + r0 * P + j * 8 + cq) =
+                    pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
+                *reinterpret_cast<uint32_t*>(qs + (r0 + 8) * P + j * 8 + cq) =
+                    pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
+            }
+        }
+        __syncthreads();
+        // coalesced write-back of the unit's outputs
+        {
+            const long long n = u / hg_count;
+            const int h0 = (int)(u - n * hg_count) * G;
+            const int per = T * G * chunks_per_row;
+            for (int c = tid; c < per; c += kThreads) {
+                const int t = c / (G * chunks_per_row);
+                int r = c - t * (G * chunks_per_row);
+                const int g = r / chunks_per_row;
+                const int ch = r - g * chunks_per_row;
+                const uint4 val = *reinterpret_cast<const uint4*>(st + g * head_elems + t * P + ch * 8);
+                __stcs(reinterpret_cast<uint4*>(p.out + ((n * T + t) * C + (long long)(h0 + g) * d +
+                                                        ch * 8)),
+                       val);
+            }
+        }
+        __syncthreads();
+    }
+    cp_async_wait<0>();
+}
+
+template <int DN>
+cudaError_t launch_dn(const TemporalArgs& p, size_t smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(temporal_kernel<DN>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, temporal_kernel<DN>, kThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    long long grid = (long long)device_sm_count() * per_sm;
+    if (grid > p.units) grid = p.units;
+    temporal_kernel<DN><<<(unsigned)grid, kThreads, smem, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
+                            int heads, int d, cudaStream_t s) {
+    TemporalArgs p;
+    p.q = static_cast<const __nv_bfloat16*>(q);
+    p.k = static_cast<const __nv_bfloat16*>(k);
+    p.v = static_cast<const __nv_bfloat16*>(v);
+    p.out = static_cast<__nv_bfloat16*>(out);
+    p.N = N;
+    p.T = T;
+    p.heads = heads;
+    p.d = d;
+    p.P = ((d / 8) & 1) ? d : d + 8;
+    p.RT = (T + 15) / 16 * 16;
+    // largest divisor of heads whose stage fits the budget
+    int G = 1;
+    for (int g = heads; g >= 1; --g)
+        if (heads % g == 0 && 3 * g * p.RT * p.P * 2 <= kMaxStageBytes) {
+            G = g;
+            break;
+        }
+    p.G = G;
+    p.units = (long long)N * (heads / G);
+    p.scale_log2 = kLog2e / sqrtf((float)d);
+    if (p.units == 0) return cudaSuccess;
+    const size_t smem = (size_t)2 * 3 * G * p.RT * p.P * 2 + 256;
+    switch (d / 8) {
+#define PAB_T_CASE(DNV) \
+    case DNV:           \
+        return launch_dn<DNV>(p, smem, s);
+        PAB_T_CASE(1) PAB_T_CASE(2) PAB_T_CASE(3) PAB_T_CASE(4) PAB_T_CASE(5) PAB_T_CASE(6)
+        PAB_T_CASE(7) PAB_T_CASE(8) PAB_T_CASE(9) PAB_T_CASE(10) PAB_T_CASE(11) PAB_T_CASE(12)
+        PAB_T_CASE(13) PAB_T_CASE(14) PAB_T_CASE(15) PAB_T_CASE(16)
+#undef PAB_T_CASE
+        default:
+            return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace pab

@@ -1,0 +1,166 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/pab.h declares, and its PAB schedule and argument
+checks behave as documented.  The schedule is compared with the oracle's
+step-by-step walk (PAB report, "Implementation" / Fig. 2)."""
+import ctypes
+import os
+import re
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    names = set()
+    for f in os.listdir(os.path.join(ROOT, "include")):
+        if f.endswith(".h"):
+            text = open(os.path.join(ROOT, "include", f)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names.update(re.findall(r"\b(pab_\w+)\s*\(", text))
+    return names
+
+
+@pytest.fixture(scope="module")
+def pab():
+    import step_reuse_b200
+    return step_reuse_b200
+
+
+def test_library_exports_every_declared_symbol(pab):
+    declared = header_functions()
+    assert len(declared) >= 15
+    raw = ctypes.CDLL(pab.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert set(pab.EXPORTS) == declared
+    assert pab.version() >= 1
+
+
+def test_library_has_sm100a_code_only():
+    """The build targets sm_100a only (no PTX / other arch fallbacks)."""
+    src = open(os.path.join(ROOT, "step_reuse_b200", "build.py")).read()
+    assert "arch=compute_100a,code=sm_100a" in src
+    assert "sm_90" not in src and "compute_90" not in src
+
+
+@pytest.mark.parametrize("name", ["tiny", "480p", "720p", "temporal_heavy", "sweep"])
+def test_schedule_matches_oracle(pab, oracle_mod, name):
+    from synth import WORKLOADS
+    w = WORKLOADS[name]
+    range_sets = w.extra_ranges or (w.ranges,)
+    for ranges in range_sets:
+        plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, ranges)
+        for kind, r in zip(("spatial", "temporal", "cross"), ranges):
+            comp, src = oracle_mod.schedule(w.steps, r)
+            got = [plan.is_compute(kind, i) for i in range(w.steps)]
+            assert got == [bool(c) for c in comp], (name, ranges, kind)
+            assert [plan.source(kind, i) for i in range(w.steps)] == list(src)
+            assert plan.count(kind) == int(comp.sum())
+        plan.close()
+
+
+def test_schedule_exhaustive_small(pab, oracle_mod):
+    for steps in range(1, 61):
+        for r in (1, 2, 3, 5, 7):
+            plan = pab.Plan(2, 2, 2, 1, 8, 4, steps, (r, r, r))
+            comp, src = oracle_mod.schedule(steps, r)
+            assert [plan.is_compute(0, i) for i in range(steps)] == [bool(c) for c in comp]
+            assert [plan.source(2, i) for i in range(steps)] == list(src)
+            plan.close()
+
+
+def test_edge_pct_parameter(pab, oracle_mod):
+    for edge in (5, 15, 25, 50):
+        plan = pab.Plan(2, 2, 2, 1, 8, 4, 40, (3, 3, 3), edge_pct=edge)
+        comp, _ = oracle_mod.schedule(40, 3, edge_pct=edge)
+        assert [plan.is_compute(1, i) for i in range(40)] == [bool(c) for c in comp]
+        plan.close()
+
+
+def test_argument_errors(pab):
+    P = pab.Plan
+    with pytest.raises(pab.PabError) as e:
+        P(4, 8, 8, 2, 30, 16, 10, (2, 3, 4))  # d % 8 != 0
+    assert e.value.code == pab.PAB_ERR_UNSUPPORTED
+    with pytest.raises(pab.PabError) as e:
+        P(4, 8, 8, 2, 32, 16, 10, (0, 3, 4))
+    assert e.value.code == pab.PAB_ERR_ARG
+    with pytest.raises(pab.PabError) as e:
+        P(4, 8, 8, 2, 32, 16, 0, (2, 3, 4))
+    assert e.value.code == pab.PAB_ERR_ARG
+    with pytest.raises(pab.PabError) as e:
+        P(200, 8, 8, 2, 32, 16, 10, (2, 3, 4))  # T > 128
+    assert e.value.code == pab.PAB_ERR_UNSUPPORTED
+    with pytest.raises(pab.PabError) as e:
+        P(4, 8, 8, 2, 32, 0, 10, (2, 3, 4))
+    assert e.value.code == pab.PAB_ERR_UNSUPPORTED
+    with pytest.raises(pab.PabError) as e:
+        P(4, 8, 8, 2, 32, 16, 10, (2, 3, 4), edge_pct=60)
+    assert e.value.code == pab.PAB_ERR_ARG
+    plan = P(4, 8, 8, 2, 32, 16, 10, (2, 3, 4))
+    with pytest.raises(pab.PabError) as e:
+        plan.is_compute(3, 0)
+    assert e.value.code == pab.PAB_ERR_ARG
+    with pytest.raises(pab.PabError) as e:
+        plan.is_compute(0, 10)
+    assert e.value.code == pab.PAB_ERR_ARG
+    plan.close()
+
+
+def test_hit_before_compute_and_step_order(pab):
+    """Host-side cache rules, exercised on broadcast steps (no device work)."""
+    plan = pab.Plan(4, 8, 8, 2, 32, 16, 10, (2, 3, 4))
+    assert not plan.is_compute("spatial", 3)
+    with pytest.raises(pab.PabError) as e:
+        plan.attention_ptr("spatial", 3)  # hit, but step 2 was never computed
+    assert e.value.code == pab.PAB_ERR_NO_CACHE
+    with pytest.raises(pab.PabError) as e:
+        plan.attention_ptr("spatial", 3)  # the failed call did not advance the order
+    assert e.value.code == pab.PAB_ERR_NO_CACHE
+    plan.reset()
+    plan.close()
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device error path")
+def test_compute_without_device_fails_loudly(pab):
+    """No GPU: a compute step reports PAB_ERR_CUDA instead of falling back."""
+    plan = pab.Plan(4, 8, 8, 2, 32, 16, 10, (2, 3, 4))
+    buf = ctypes.create_string_buffer(1 << 16)
+    addr = (ctypes.addressof(buf) + 15) // 16 * 16
+    out = ctypes.c_void_p()
+    rc = pab.lib.pab_attention(plan._h, 0, 0, ctypes.c_void_p(addr), ctypes.c_void_p(addr),
+                               ctypes.c_void_p(addr), ctypes.byref(out), None)
+    assert rc in (pab.PAB_ERR_CUDA, pab.PAB_ERR_OOM)
+    assert pab.lib.pab_last_error_string()
+    with pytest.raises(pab.PabError) as e:
+        plan.prepare()
+    assert e.value.code in (pab.PAB_ERR_CUDA, pab.PAB_ERR_OOM)
+    plan.close()
+    res = ctypes.c_double()
+    rc = pab.lib.pab_attn_diff_mse(ctypes.c_void_p(addr), ctypes.c_void_p(addr), 64, 0,
+                                   ctypes.byref(res), None)
+    assert rc in (pab.PAB_ERR_CUDA, pab.PAB_ERR_OOM)
+
+
+def test_stateless_argument_checks(pab):
+    lib = pab.lib
+    vp = ctypes.c_void_p
+    assert lib.pab_spatial_attention(None, None, None, None, 1, 16, 2, 32, None) == pab.PAB_ERR_ARG
+    assert lib.pab_spatial_attention(None, None, None, None, 1, 16, 2, 36, None) == pab.PAB_ERR_UNSUPPORTED
+    assert lib.pab_temporal_attention(None, None, None, None, 16, 200, 2, 32, None) == pab.PAB_ERR_UNSUPPORTED
+    assert lib.pab_cross_attention(None, None, None, None, 10, 0, 2, 32, None) == pab.PAB_ERR_UNSUPPORTED
+    assert lib.pab_cross_attention(None, None, None, None, 10, 600, 2, 32, None) == pab.PAB_ERR_UNSUPPORTED
+    # empty problems are no-ops
+    assert lib.pab_spatial_attention(None, None, None, None, 0, 16, 2, 32, None) == pab.PAB_OK
+    assert lib.pab_layout(1, None, None, 4, 0, 64, 0, None) == pab.PAB_OK
+    # misaligned pointers
+    assert lib.pab_layout(1, vp(8), vp(1 << 20), 4, 4, 64, 0, None) == pab.PAB_ERR_ARG
+    assert lib.pab_layout(1, vp(1 << 20), vp(1 << 21), 4, 4, 60, 0, None) == pab.PAB_ERR_UNSUPPORTED
+    # overlap
+    assert lib.pab_layout(1, vp(1 << 20), vp((1 << 20) + 64), 4, 4, 64, 0, None) == pab.PAB_ERR_ARG
+    res = ctypes.c_double(1.0)
+    assert lib.pab_attn_diff_mse(None, None, 10, 0, ctypes.byref(res), None) == pab.PAB_ERR_ARG
+    assert lib.pab_attn_diff_mse(None, None, 10, 7, ctypes.byref(res), None) == pab.PAB_ERR_ARG
+    assert lib.pab_attn_diff_mse(None, None, 10, 0, None, None) == pab.PAB_ERR_ARG
