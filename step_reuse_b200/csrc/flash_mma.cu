@@ -224,7 +224,7 @@ cudaError_t launch_dn(const FlashArgs& p, dim3 grid, size_t smem, cudaStream_t s
 
 }  // namespace
 
-cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches,
+cudaError_t launch_flash_mma(const void* q, const void* k, const void* v, void* out, int batches,
                          long long Lq, int Lk, int heads, int d, long long q_bstride,
                          long long kv_bstride, cudaStream_t s) {
     FlashArgs p;

@@ -1,0 +1,421 @@
+// flash_tc.cu -- flash (online-softmax) attention on the 5th-generation
+// tensor cores (tcgen05 + TMEM) for the long-sequence PAB kinds: spatial
+// attention (the tokens of one frame, L = H*W) and cross attention (video
+// tokens against one shared set of text keys/values) -- PAB report,
+// "Implementation".  softmax(Q K^T / sqrt(d)) V per (batch, head).
+//
+// One CTA owns a 128-row query tile of one (batch, head) and runs three roles:
+//   warp 4 (one thread)  TMA producer: Q once, then K_j / V_j tiles of 128
+//                         keys into a STAGES-deep shared-memory ring;
+//   warp 5 (one thread)  MMA issuer: S_j = Q K_j^T (SS form, fp32 in TMEM,
+//                         double-buffered S_0 / S_1), then O += P_j V_j
+//                         (TS form: P read from TMEM, V from shared memory);
+//                         warp 5 also owns the TMEM allocation;
+//   warps 0-3            softmax: thread i owns query row i = TMEM lane i; it
+//                         reads its row of S_j with tcgen05.ld, applies the
+//                         online softmax (row max / sum in registers, no
+//                         shuffles), writes P_j as bf16 over S_j's columns and
+//                         rescales O in TMEM only when the running max grew by
+//                         more than 2^8 (the final O / l is exact either way);
+//                         at the end it normalises O and stores it through
+//                         shared memory with a TMA tensor store.
+// S_{j+1} is computed on the tensor cores while the softmax warps work on S_j.
+//
+// Operand layouts (128-byte swizzle, TMA-written):
+//   Q, K: [128 rows][64 cols] boxes, K-major (d contiguous); a 16-wide K step
+//         advances the descriptor start by 32 bytes inside the box.
+//   V:    the same boxes read MN-major (B of the PV product has N = d
+//         contiguous); a 16-key K step advances by 16 rows = 2048 bytes, the
+//         next 64 columns of d are one box (16 KB) further (LBO).
+// Head dims that are not a multiple of 64 read zero-filled columns past d
+// (the tensor map's innermost extent is d); keys past Lk are masked to -inf;
+// query rows past Lq are zero-filled on load and clipped by the TMA store.
+// Every wait on an mbarrier is bounded; on time-out the CTA raises the error
+// word, lets its own asynchronous copies and MMAs drain, frees TMEM and exits.
+#include <cuda.h>
+
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace pab {
+namespace {
+
+constexpr int kBM = 128;          // query rows per CTA
+constexpr int kBN = 128;          // keys per tile
+constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
+constexpr int kThreads = 192;     // 4 softmax warps + producer warp + MMA warp
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;  // TMEM column bases
+constexpr float kRescaleLog2 = 8.0f;
+
+__device__ unsigned int g_flash_err = 0;
+
+struct FlashTcArgs {
+    int Lq;            // query rows per batch
+    int Lk;            // keys per batch
+    int kv_batched;    // 1: K/V have a batch coordinate (spatial); 0: shared (cross)
+    float scale_log2;  // log2(e) / sqrt(d)
+};
+
+struct Bars {
+    unsigned long long q_full;
+    unsigned long long k_full[4];
+    unsigned long long v_full[4];
+    unsigned long long kv_empty[4];
+    unsigned long long s_full[2];
+    unsigned long long p_full[2];
+    unsigned long long o_done;
+    unsigned long long mma_done;
+    uint32_t tmem_base;
+    int abort;
+};
+
+PAB_DEV float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// bounded wait that gives up at once when the CTA has already aborted
+PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
+    if (*(volatile int*)&b->abort) return false;
+    if (!mbar_wait_bounded(smem_u32(bar), parity, &g_flash_err)) {
+        *(volatile int*)&b->abort = 1;
+        return false;
+    }
+    return true;
+}
+
+template <int KSTEPS, int STAGES>
+__global__ void __launch_bounds__(kThreads, 1)
+    flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                    FlashTcArgs a) {
+    constexpr int NB = (KSTEPS + 3) / 4;  // 64-column boxes covering d
+    constexpr int NO = KSTEPS * 16;       // N of the PV product (d rounded up to 16)
+    constexpr uint32_t kTileBytes = NB * kBox;
+
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    __shared__ Bars bars;
+    // 1024-byte aligned base for the swizzled tiles
+    const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
+    const uint32_t q_s = sbase;
+    const uint32_t k_s = q_s + kTileBytes;
+    const uint32_t v_s = k_s + STAGES * kTileBytes;
+    unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int nkv = (a.Lk + kBN - 1) / kBN;
+
+    if (threadIdx.x == 128) {
+        mbar_init(smem_u32(&bars.q_full), 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&bars.k_full[s]), 1);
+            mbar_init(smem_u32(&bars.v_full[s]), 1);
+            mbar_init(smem_u32(&bars.kv_empty[s]), 1);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&bars.s_full[s]), 1);
+            mbar_init(smem_u32(&bars.p_full[s]), 128);
+        }
+        mbar_init(smem_u32(&bars.o_done), 1);
+        mbar_init(smem_u32(&bars.mma_done), 1);
+        bars.abort = 0;
+        fence_mbar_init();
+        tc::prefetch_tmap(&tm_q);
+        tc::prefetch_tmap(&tm_k);
+        tc::prefetch_tmap(&tm_v);
+        tc::prefetch_tmap(&tm_o);
+    }
+    if (warp == 5) {
+        tc::tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
+        tc::tmem_relinquish();
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = bars.tmem_base;
+    const int kvb = a.kv_batched ? b : 0;
+
+    if (warp == 4) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            int issued[4] = {0, 0, 0, 0};
+            mbar_arrive_expect_tx(smem_u32(&bars.q_full), kTileBytes);
+            for (int bx = 0; bx < NB; ++bx)
+                tc::tma_load_4d(q_s + bx * kBox, &tm_q, bx * 64, h, qt * kBM, b, smem_u32(&bars.q_full));
+            bool ok = true;
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int st = j % STAGES;
+                if (j >= STAGES) ok = wait_bar(&bars, &bars.kv_empty[st], ((j / STAGES) - 1) & 1);
+                if (!ok) break;
+                mbar_arrive_expect_tx(smem_u32(&bars.k_full[st]), kTileBytes);
+                for (int bx = 0; bx < NB; ++bx)
+                    tc::tma_load_4d(k_s + st * kTileBytes + bx * kBox, &tm_k, bx * 64, h, j * kBN, kvb,
+                                    smem_u32(&bars.k_full[st]));
+                mbar_arrive_expect_tx(smem_u32(&bars.v_full[st]), kTileBytes);
+                for (int bx = 0; bx < NB; ++bx)
+                    tc::tma_load_4d(v_s + st * kTileBytes + bx * kBox, &tm_v, bx * 64, h, j * kBN, kvb,
+                                    smem_u32(&bars.v_full[st]));
+                issued[st] += 1;
+            }
+            if (!ok || *(volatile int*)&bars.abort) {
+                // drain: let this CTA's loads land before it exits (bounded)
+                for (int s = 0; s < STAGES; ++s)
+                    if (issued[s] > 0) {
+                        mbar_wait_bounded(smem_u32(&bars.k_full[s]), (issued[s] - 1) & 1, &g_flash_err);
+                        mbar_wait_bounded(smem_u32(&bars.v_full[s]), (issued[s] - 1) & 1, &g_flash_err);
+                    }
+                mbar_wait_bounded(smem_u32(&bars.q_full), 0, &g_flash_err);
+            }
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
+            constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
+            bool ok = wait_bar(&bars, &bars.q_full, 0);
+            auto issue_pv = [&](int j) -> bool {
+                const int st = j % STAGES;
+                if (!wait_bar(&bars, &bars.p_full[j & 1], (j >> 1) & 1)) return false;
+                if (!wait_bar(&bars, &bars.v_full[st], (j / STAGES) & 1)) return false;
+                tc::fence_after_sync();
+                const uint32_t p_tmem = tmem + ((j & 1) ? kS1 : kS0);
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    const uint64_t bdesc =
+                        tc::smem_desc(v_s + st * kTileBytes + kk * 2048, kBox, 1024, 2);
+                    tc::mma_ts(tmem + kO, p_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                }
+                tc::commit(smem_u32(&bars.kv_empty[st]));
+                tc::commit(smem_u32(&bars.o_done));
+                return true;
+            };
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int st = j % STAGES;
+                ok = wait_bar(&bars, &bars.k_full[st], (j / STAGES) & 1);
+                if (!ok) break;
+                tc::fence_after_sync();
+                const uint32_t s_tmem = tmem + ((j & 1) ? kS1 : kS0);
+#pragma unroll
+                for (int ks = 0; ks < KSTEPS; ++ks) {
+                    const uint32_t off = (ks >> 2) * kBox + (ks & 3) * 32;
+                    const uint64_t adesc = tc::smem_desc(q_s + off, 16, 1024, 2);
+                    const uint64_t bdesc = tc::smem_desc(k_s + st * kTileBytes + off, 16, 1024, 2);
+                    tc::mma_ss(s_tmem, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+                }
+                tc::commit(smem_u32(&bars.s_full[j & 1]));
+                if (j > 0) ok = issue_pv(j - 1);
+            }
+            if (ok && nkv > 0) ok = issue_pv(nkv - 1);
+            // all MMAs this thread issued complete before TMEM is released
+            tc::commit(smem_u32(&bars.mma_done));
+            mbar_wait_bounded(smem_u32(&bars.mma_done), 0, &g_flash_err);
+        }
+    } else {
+        // ------------------------------------------------ softmax warps
+        const int row = warp * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        float m_ref = -INFINITY, l = 0.f;
+        bool ok = true;
+        for (int j = 0; j < nkv; ++j) {
+            ok = wait_bar(&bars, &bars.s_full[j & 1], (j >> 1) & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint32_t s_addr = lane_addr + ((j & 1) ? kS1 : kS0);
+            float s[kBN];
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t r[32];
+                tc::ld_32col(s_addr + c * 32, r);
+                tc::wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+            }
+            const int valid = a.Lk - j * kBN;  // keys of this tile that exist
+            float mt = -INFINITY;
+#pragma unroll
+            for (int i = 0; i < kBN; ++i) {
+                s[i] = (i < valid) ? s[i] * a.scale_log2 : -INFINITY;
+                mt = fmaxf(mt, s[i]);
+            }
+            if (j == 0) {
+                m_ref = mt;
+            } else {
+                const bool need = mt > m_ref + kRescaleLog2;
+                if (__any_sync(0xffffffffu, need)) {
+                    const float m_new = need ? mt : m_ref;
+                    const float f = ex2(m_ref - m_new);
+                    // O must hold PV_{j-1} before it is rescaled
+                    ok = wait_bar(&bars, &bars.o_done, (j - 1) & 1);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+#pragma unroll
+                    for (int c = 0; c < NO / 16; ++c) {
+                        uint32_t r[16];
+                        tc::ld_16col(lane_addr + kO + c * 16, r);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+                        tc::st_16col(lane_addr + kO + c * 16, r);
+                    }
+                    l *= f;
+                    m_ref = m_new;
+                }
+            }
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < kBN / 32; ++c) {
+                uint32_t r[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const float p0 = ex2(s[c * 32 + 2 * i] - m_ref);
+                    const float p1 = ex2(s[c * 32 + 2 * i + 1] - m_ref);
+                    rs += p0 + p1;
+                    r[i] = pack_bf16x2(p0, p1);
+                }
+                tc::st_16col(s_addr + c * 16, r);
+            }
+            l += rs;
+            tc::wait_st();
+            tc::fence_before_sync();
+            mbar_arrive(smem_u32(&bars.p_full[j & 1]));
+        }
+        // ---------------- epilogue: O / l -> bf16 -> swizzled smem -> TMA store
+        if (ok && nkv > 0) ok = wait_bar(&bars, &bars.o_done, (nkv - 1) & 1);
+        if (ok) {
+            tc::fence_after_sync();
+            const float inv = 1.f / l;
+            unsigned char* stage = gen_base;  // reuse the Q tile (all S MMAs are done)
+#pragma unroll
+            for (int c = 0; c < NO / 16; ++c) {
+                uint32_t r[16];
+                tc::ld_16col(lane_addr + kO + c * 16, r);
+                tc::wait_ld();
+                uint32_t w[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                // columns c*16 .. c*16+15 = two 16-byte chunks of box (c*16)/64
+                const int col = c * 16;
+                const int bx = col >> 6;
+                const int ch = (col & 63) >> 3;
+                unsigned char* rowp = stage + bx * kBox + row * 128;
+                *reinterpret_cast<uint4*>(rowp + (((ch) ^ (row & 7)) << 4)) =
+                    make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
+                    make_uint4(w[4], w[5], w[6], w[7]);
+            }
+            fence_proxy_async_smem();
+        }
+        tc::named_bar_sync(1, 128);
+        if (ok && row == 0) {
+            for (int bx = 0; bx < NB; ++bx) tc::tma_store_4d(&tm_o, q_s + bx * kBox, bx * 64, h, qt * kBM, b);
+            bulk_commit();
+            bulk_wait<0>();
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    if (warp == 5) {
+        __syncwarp();
+        tc::fence_after_sync();
+        tc::tmem_dealloc(tmem, kTmemCols);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 4-D map over a [batches][rows][heads][d] bf16 view (row stride C elements):
+// dims (d, heads, rows, batches), box (64, 1, 128, 1), 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows, long long batches,
+              long long row_stride_elems, long long batch_stride_elems) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows, (cuuint64_t)batches};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)row_stride_elems * 2,
+                             (cuuint64_t)(batch_stride_elems > 0 ? batch_stride_elems : rows * row_stride_elems) * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int KSTEPS>
+cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                      const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
+    constexpr int NB = (KSTEPS + 3) / 4;
+    constexpr int STAGES = NB == 1 ? 3 : 2;
+    const size_t smem = (size_t)(1 + 2 * STAGES) * NB * kBox + 1024;
+    const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
+    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, STAGES>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
+    if (e != cudaSuccess) return e;
+    flash_tc_kernel<KSTEPS, STAGES><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches, long long Lq,
+                         int Lk, int heads, int d, long long q_bstride, long long kv_bstride, cudaStream_t s) {
+    if (Lq == 0 || batches == 0) return cudaSuccess;
+    const long long C = (long long)heads * d;
+    const long long qtiles = (Lq + kBM - 1) / kBM;
+    if (qtiles > 0x7fffffffLL || batches > 65535 || heads > 65535 || Lq > 0x7fffffffLL)
+        return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mo;
+    const long long kv_batches = kv_bstride > 0 ? batches : 1;
+    if (!make_map(&mq, q, d, heads, Lq, batches, C, q_bstride) ||
+        !make_map(&mk, k, d, heads, Lk, kv_batches, C, kv_bstride) ||
+        !make_map(&mv, v, d, heads, Lk, kv_batches, C, kv_bstride) ||
+        !make_map(&mo, out, d, heads, Lq, batches, C, q_bstride))
+        return cudaErrorInvalidValue;
+    FlashTcArgs a;
+    a.Lq = (int)Lq;
+    a.Lk = Lk;
+    a.kv_batched = kv_bstride > 0 ? 1 : 0;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+    dim3 grid((unsigned)qtiles, (unsigned)heads, (unsigned)batches);
+    switch ((d + 15) / 16) {
+        case 1: return launch_ks<1>(mq, mk, mv, mo, a, grid, s);
+        case 2: return launch_ks<2>(mq, mk, mv, mo, a, grid, s);
+        case 3: return launch_ks<3>(mq, mk, mv, mo, a, grid, s);
+        case 4: return launch_ks<4>(mq, mk, mv, mo, a, grid, s);
+        case 5: return launch_ks<5>(mq, mk, mv, mo, a, grid, s);
+        case 6: return launch_ks<6>(mq, mk, mv, mo, a, grid, s);
+        case 7: return launch_ks<7>(mq, mk, mv, mo, a, grid, s);
+        case 8: return launch_ks<8>(mq, mk, mv, mo, a, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+unsigned int flash_device_errors(bool clear) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_flash_err, sizeof(v)) != cudaSuccess) return 0xffffffffu;
+    if (clear && v) {
+        unsigned int z = 0;
+        cudaMemcpyToSymbol(g_flash_err, &z, sizeof(z));
+    }
+    return v;
+}
+
+}  // namespace pab

@@ -33,6 +33,11 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
                          long long Lq, int Lk, int heads, int d, long long q_bstride,
                          long long kv_bstride, cudaStream_t s);
 
+cudaError_t launch_flash_mma(const void* q, const void* k, const void* v, void* out, int batches,
+                             long long Lq, int Lk, int heads, int d, long long q_bstride,
+                             long long kv_bstride, cudaStream_t s);
+unsigned int flash_device_errors(bool clear);
+
 // --- dtype conversion for fp32 plans --------------------------------------
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t s);
 cudaError_t launch_bf16_to_f32(const void* src, float* dst, long long n, cudaStream_t s);
