@@ -50,13 +50,15 @@ MEASURED_TRAFFIC = {}
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--input-sets", type=int, default=8,
+                    help="distinct drifted input sets cycled over the diffusion steps")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0,
                     help="target seconds of oracle work for the CPU baseline sample")
     return ap.parse_args(argv)
@@ -133,7 +135,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
+                 "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except (OSError, ValueError):
             self.proc = None
@@ -376,7 +378,7 @@ def run_ours(args):
     exec_flops = sum(counts[k] * flops[k] for k in synth.KINDS)
     abytes = algorithmic_bytes(w)
 
-    n_sets = min(w.steps, 8)
+    n_sets = max(1, min(w.steps, args.input_sets))
     inputs = make_inputs(w, device, n_sets, seed=rank)
     stack = AttentionStack(pab, w, device)
     stream = torch.cuda.current_stream(device)
@@ -417,7 +419,7 @@ def run_ours(args):
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
     sp_ms = per_kind_ms["spatial"]
     achieved = flops["spatial"] / (sp_ms * 1e-3) / 1e12
-    src_hash = kernel_source_hash("flash_mma.cu")
+    src_hash = kernel_source_hash("flash_tc.cu")
     traffic = MEASURED_TRAFFIC.get(src_hash)
     roofline = {"kernel": "spatial flash attention", "bound": "tensor", "achieved": achieved,
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,

@@ -5,7 +5,7 @@ Argument marshalling only: every step of the attention stack runs in the
 library's CUDA kernels.  Tensors are torch CUDA tensors (PyTorch supplies the
 device memory and the stream); the calls go through the C ABI declared in
 include/pab.h with ctypes.  Importing this package fails loudly if
-libpab.so has not been built (python -m step_reuse_b200.build); there is no
+libpab.so has not been built (python step_reuse_b200/build.py); there is no
 CPU fallback.
 """
 from __future__ import annotations
@@ -53,7 +53,7 @@ class pab_ranges(ctypes.Structure):
 
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m step_reuse_b200.build`")
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python step_reuse_b200/build.py`")
     lib = ctypes.CDLL(LIB_PATH)
     vp, i, ll = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong
     sig = {

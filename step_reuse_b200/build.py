@@ -1,6 +1,6 @@
 """Build libpab.so (the sm_100a kernels + C ABI) in-tree with nvcc.
 
-    python -m step_reuse_b200.build [--force] [-v]
+    python step_reuse_b200/build.py [--force] [-v]
 
 Every .cu under csrc/ is compiled for sm_100a only
 (-gencode arch=compute_100a,code=sm_100a) and linked into

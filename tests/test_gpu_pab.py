@@ -39,23 +39,27 @@ def oracle_kind(oracle_mod, kind, q, k, v, heads):
 
 def sampled_check(oracle_mod, kind, w, x, out, rng, what):
     """Compare seeded samples of the output with the oracle computed on just
-    those rows (each query row's result depends only on its keys)."""
-    q, k, v = (to_f64(x[n]) for n in ("q", "k", "v"))
-    o = to_f64(out)
+    those rows (each query row's result depends only on its keys).  Rows are
+    gathered on the device first, so only the samples cross to the host."""
+    q, k, v = x["q"], x["k"], x["v"]
+    dev = q.device
     if kind == "spatial":
         for t in rng.choice(w.T, size=min(2, w.T), replace=False):
-            rows = np.sort(rng.choice(w.N, size=min(256, w.N), replace=False))
+            rows = torch.from_numpy(np.sort(rng.choice(w.N, size=min(256, w.N), replace=False))).to(dev)
+            t = int(t)
             # rows of frame t against all keys of frame t
-            want = oracle_mod.cross_attention(q[t, rows], k[t], v[t], w.heads)
-            assert_attn_close(o[t, rows], want, f"{what} frame {t}")
+            want = oracle_mod.cross_attention(to_f64(q[t].index_select(0, rows)), to_f64(k[t]),
+                                              to_f64(v[t]), w.heads)
+            assert_attn_close(out[t].index_select(0, rows), want, f"{what} frame {t}")
     elif kind == "temporal":
-        pos = np.sort(rng.choice(w.N, size=min(512, w.N), replace=False))
-        want = oracle_mod.temporal_attention(q[pos], k[pos], v[pos], w.heads)
-        assert_attn_close(o[pos], want, what)
+        pos = torch.from_numpy(np.sort(rng.choice(w.N, size=min(512, w.N), replace=False))).to(dev)
+        want = oracle_mod.temporal_attention(to_f64(q.index_select(0, pos)), to_f64(k.index_select(0, pos)),
+                                             to_f64(v.index_select(0, pos)), w.heads)
+        assert_attn_close(out.index_select(0, pos), want, what)
     else:
-        rows = np.sort(rng.choice(w.T * w.N, size=min(4096, w.T * w.N), replace=False))
-        want = oracle_mod.cross_attention(q[rows], k, v, w.heads)
-        assert_attn_close(o[rows], want, what)
+        rows = torch.from_numpy(np.sort(rng.choice(w.T * w.N, size=min(4096, w.T * w.N), replace=False))).to(dev)
+        want = oracle_mod.cross_attention(to_f64(q.index_select(0, rows)), to_f64(k), to_f64(v), w.heads)
+        assert_attn_close(out.index_select(0, rows), want, what)
 
 
 def run_pab(pab, oracle_mod, w, ranges, check_steps, full_steps=(), mse_steps=None, seed=0):
