@@ -128,6 +128,23 @@ int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype,
 int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype,
                             double* result_dev, void* cuda_stream);
 
+/* Allocation-free variant of pab_attn_diff_mse_async, for callers that
+ * cannot call cudaMalloc (code inside a framework whose memory pool owns all
+ * device memory, or latency-critical loops that must not allocate).  The
+ * paper has no counterpart: this is a property of the library, not of PAB.
+ * Same arguments and result as pab_attn_diff_mse_async (result_dev is a
+ * DEVICE pointer; no synchronisation), but the fp64 partial sums live in a
+ * static device array of 4096 doubles (32 KiB) that every GPU loading the
+ * library holds until exit; the call allocates nothing.  A call that would
+ * need more than 4096 partial sums (only on devices with more than 1024 SMs)
+ * returns PAB_ERR_UNSUPPORTED.  The first call on each device looks up the
+ * array's device address (cudaGetSymbolAddress) and caches it; make that
+ * first call before any stream capture.  All calls share the array: calls
+ * whose kernels overlap on the GPU race and must be serialised by the
+ * caller. */
+int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long n, int dtype,
+                              double* result_dev, void* cuda_stream);
+
 /* Device status word of the kernels that wait on asynchronous copies: bit 0
  * is set when a bounded wait gave up (the kernel then returns early and its
  * output is incomplete).  Synchronises the device to read it; clear != 0

@@ -33,7 +33,7 @@ BF16, FP32 = 0, 1
 # every symbol include/pab.h declares
 EXPORTS = (
     "pab_version", "pab_last_error_string", "pab_spatial_attention", "pab_temporal_attention",
-    "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async",
+    "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
     "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
     "pab_attention",
@@ -65,6 +65,7 @@ def _load() -> ctypes.CDLL:
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
         "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
         "pab_attn_diff_mse_async": ([vp, vp, ll, i, vp, vp], i),
+        "pab_attn_diff_mse_noalloc": ([vp, vp, ll, i, vp, vp], i),
         "pab_device_errors": ([i, ctypes.POINTER(ctypes.c_uint)], i),
         "pab_plan_create": ([i, i, i, i, i, i, i, pab_ranges, i, ctypes.POINTER(vp)], i),
         "pab_plan_destroy": ([vp], i),

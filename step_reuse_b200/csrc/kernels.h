@@ -11,6 +11,9 @@ namespace pab {
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
+// Record `code` and a message as the calling thread's last error; returns code.
+int report_error(int code, const char* fmt, ...);
+
 // --- attention-difference MSE (two passes, fp64, deterministic) ----------
 // Number of first-pass partial sums used for n elements on this device.
 int mse_num_partials(long long n, int elem_size);

@@ -10,6 +10,9 @@
 // fp64 partial per block.  Pass 2: one block sums the partials in a fixed
 // order and divides by n.  The split depends only on n and the SM count, so
 // the result is bitwise reproducible on a given device.
+#include <mutex>
+
+#include "../../include/pab.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -155,3 +158,83 @@ cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, dou
 }
 
 }  // namespace pab
+
+// ===========================================================================
+// Allocation-free variant of the MSE diagnostic.
+//
+// Some callers cannot call cudaMalloc: code that runs inside a host framework
+// whose memory pool owns all device memory and must account for every byte,
+// or latency-critical loops where a device allocation (and the implicit
+// synchronisation it may bring) is not acceptable.  For them,
+// pab_attn_diff_mse_noalloc keeps its fp64 partial sums in a fixed,
+// file-scope device array instead of the lazily allocated per-device buffer
+// that pab_attn_diff_mse / pab_attn_diff_mse_async use.
+//
+// The array holds kNoAllocMaxPartials doubles (32 KiB).  Every GPU that loads
+// this library keeps it until the process exits.  Every call shares it and
+// it keeps the last call's contents; nothing in it has to start at zero,
+// because each first-pass block overwrites its own slot and the second pass
+// reads only the slots this call wrote.  Calls whose kernels overlap on the
+// GPU (different streams, or different host threads on one device) race on
+// the array and must be serialised by the caller.
+// ===========================================================================
+namespace {
+
+constexpr int kNoAllocMaxPartials = 4096;
+static __device__ __align__(256) double g_mse_noalloc_scratch[kNoAllocMaxPartials];
+
+constexpr int kNoAllocMaxDevices = 64;
+std::mutex g_noalloc_mu;
+double* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
+
+// Device address of the array on the current device.  Host code cannot use
+// the array's name as a device pointer (it names a host-side stand-in), so
+// the address is looked up once per device with cudaGetSymbolAddress while
+// that device is current, and cached.
+int noalloc_scratch(double** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return pab::report_error(PAB_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= kNoAllocMaxDevices)
+        return pab::report_error(PAB_ERR_UNSUPPORTED, "device index %d", dev);
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_mse_noalloc_scratch);
+        if (e != cudaSuccess || !p)
+            return pab::report_error(PAB_ERR_CUDA, "cudaGetSymbolAddress of the MSE scratch array: %s",
+                                     cudaGetErrorString(e));
+        g_noalloc_ptr[dev] = static_cast<double*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return PAB_OK;
+}
+
+}  // namespace
+
+extern "C" int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long n, int dtype,
+                                         double* result_dev, void* cuda_stream) {
+    if (dtype != PAB_BF16 && dtype != PAB_FP32)
+        return pab::report_error(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (n < 0) return pab::report_error(PAB_ERR_ARG, "n=%lld must be >= 0", n);
+    if (!result_dev || (reinterpret_cast<uintptr_t>(result_dev) & 7u))
+        return pab::report_error(PAB_ERR_ARG, "result_dev null or not 8-byte aligned");
+    if (n > 0 && (!a || !b)) return pab::report_error(PAB_ERR_ARG, "null input");
+    if (n > 0 && ((reinterpret_cast<uintptr_t>(a) | reinterpret_cast<uintptr_t>(b)) & 15u))
+        return pab::report_error(PAB_ERR_ARG, "inputs not 16-byte aligned");
+    const int elem = dtype == PAB_FP32 ? 4 : 2;
+    const int parts = pab::mse_num_partials(n, elem);
+    if (parts > kNoAllocMaxPartials)
+        return pab::report_error(PAB_ERR_UNSUPPORTED,
+                                 "this call needs %d partial sums; the static scratch array holds %d",
+                                 parts, kNoAllocMaxPartials);
+    double* scratch = nullptr;
+    const int rc = noalloc_scratch(&scratch);
+    if (rc != PAB_OK) return rc;
+    const cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, result_dev,
+                                          static_cast<cudaStream_t>(cuda_stream));
+    if (e != cudaSuccess)
+        return pab::report_error(PAB_ERR_CUDA, "MSE launch: %s", cudaGetErrorString(e));
+    return PAB_OK;
+}

@@ -119,6 +119,16 @@ int run_cross(const void* q, const void* kt, const void* vt, void* out, long lon
 }  // namespace
 
 namespace pab {
+int report_error(int code, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof(buf), fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return code;
+}
+
 int device_sm_count() {
     static int cache[kMaxDevices] = {0};
     int dev = 0;
