@@ -4,23 +4,30 @@
 // tokens against one shared set of text keys/values) -- PAB report,
 // "Implementation".  softmax(Q K^T / sqrt(d)) V per (batch, head).
 //
-// One CTA owns a 128-row query tile of one (batch, head) and runs three roles:
-//   warp 4 (one thread)  TMA producer: Q once, then K_j / V_j tiles of 128
-//                         keys into a STAGES-deep shared-memory ring;
-//   warp 5 (one thread)  MMA issuer: S_j = Q K_j^T (SS form, fp32 in TMEM,
-//                         double-buffered S_0 / S_1), then O += P_j V_j
-//                         (TS form: P read from TMEM, V from shared memory);
-//                         warp 5 also owns the TMEM allocation;
-//   warps 0-3            softmax: thread i owns query row i = TMEM lane i; it
-//                         reads its row of S_j with tcgen05.ld, applies the
-//                         online softmax (row max / sum in registers, no
-//                         shuffles), writes P_j as bf16 over S_j's columns and
-//                         rescales O in TMEM only when the running max grew by
-//                         more than 2^8 (the final O / l is exact either way);
-//                         at the end it normalises O and stores it through
-//                         shared memory with a TMA tensor store.
-// S_{j+1} is computed on the tensor cores while the softmax warps work on S_j.
+// A CTA owns 256 query rows of one (batch, head) as two 128-row tiles A and B
+// that share every K/V tile, and runs four roles:
+//   warp 8 (one thread)   TMA producer: Q_A, Q_B once, then K_j / V_j tiles of
+//                          128 keys into a STAGES-deep shared-memory ring;
+//   warp 9 (one thread)   MMA issuer: S_X = Q_X K_j^T (SS form, fp32 in TMEM)
+//                          and O_X += P_X V_j (TS form: P from TMEM, V from
+//                          shared memory), ping-ponging between the tiles:
+//                          PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ... so the
+//                          tensor cores work on one tile while the other
+//                          tile's softmax runs; warp 9 also owns TMEM;
+//   warps 0-3 / 4-7       softmax of tile A / B: thread i owns query row i =
+//                          TMEM lane i.  It reads its row of S with tcgen05.ld,
+//                          keeps the running max and sum in registers (tree
+//                          reductions, no shuffles), writes P as bf16 over S's
+//                          columns and rescales O in TMEM only when the running
+//                          max grew by more than 2^8 (the final O / l is exact
+//                          either way).  Exponentials: most on the MUFU ex2
+//                          unit, a fixed share on the FMA pipes (exp2_poly).
+//                          At the end it normalises O and writes it through
+//                          shared memory with a TMA tensor store.
+// When S_X(j) completes, every earlier MMA of the issuing thread -- PV_X(j-1)
+// in particular -- has completed too, so the softmax may rescale O_X then.
 //
+// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+NO), O_B [384,384+NO).
 // Operand layouts (128-byte swizzle, TMA-written):
 //   Q, K: [128 rows][64 cols] boxes, K-major (d contiguous); a 16-wide K step
 //         advances the descriptor start by 32 bytes inside the box.
@@ -29,7 +36,8 @@
 //         next 64 columns of d are one box (16 KB) further (LBO).
 // Head dims that are not a multiple of 64 read zero-filled columns past d
 // (the tensor map's innermost extent is d); keys past Lk are masked to -inf;
-// query rows past Lq are zero-filled on load and clipped by the TMA store.
+// query rows past Lq are zero-filled on load and clipped by the TMA store; a
+// B tile that lies wholly past Lq is skipped.
 // Every wait on an mbarrier is bounded; on time-out the CTA raises the error
 // word, lets its own asynchronous copies and MMAs drain, frees TMEM and exits.
 #include <cuda.h>
@@ -40,13 +48,15 @@
 namespace pab {
 namespace {
 
-constexpr int kBM = 128;          // query rows per CTA
-constexpr int kBN = 128;          // keys per tile
+constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
+constexpr int kBN = 128;          // keys per K/V tile
 constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
-constexpr int kThreads = 192;     // 4 softmax warps + producer warp + MMA warp
+constexpr int kThreads = 320;     // 2 softmax warpgroups + producer warp + MMA warp
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kS0 = 0, kS1 = 128, kO = 256;  // TMEM column bases
 constexpr float kRescaleLog2 = 8.0f;
+// Of every 8 consecutive scores of a row, this many take exp2_poly (FMA
+// pipes), the rest the MUFU ex2 unit.
+constexpr int kPolyOf8 = 3;
 
 __device__ unsigned int g_flash_err = 0;
 
@@ -58,13 +68,13 @@ struct FlashTcArgs {
 };
 
 struct Bars {
-    unsigned long long q_full;
+    unsigned long long q_full[2];
     unsigned long long k_full[4];
     unsigned long long v_full[4];
     unsigned long long kv_empty[4];
     unsigned long long s_full[2];
     unsigned long long p_full[2];
-    unsigned long long o_done;
+    unsigned long long o_done[2];
     unsigned long long mma_done;
     uint32_t tmem_base;
     int abort;
@@ -74,6 +84,27 @@ PAB_DEV float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// 2^x on the FMA/ALU pipes, for x <= 8 (the lazily rescaled softmax never
+// exceeds 2^8).  Cody-Waite style range reduction: x = n + f with n = rint(x)
+// (the 1.5*2^23 rounding trick) and f in [-0.5, 0.5]; 2^f from a degree-3
+// polynomial fitted here by minimising the maximum relative error on
+// [-0.5, 0.5] (linear-programming minimax fit; max relative error 7.5e-5,
+// far below the bf16 rounding of P); 2^n is added to the exponent field.
+// x below -120 is clamped (the result, ~1e-36, is negligible next to the
+// row maximum's weight 1).
+PAB_DEV float exp2_poly(float x) {
+    x = fmaxf(x, -120.0f);
+    const float y = x + 12582912.0f;  // 1.5 * 2^23
+    const float n = y - 12582912.0f;  // rint(x)
+    const float f = x - n;
+    float p = fmaf(0.0551716685f, f, 0.242611125f);
+    p = fmaf(p, f, 0.693260968f);
+    p = fmaf(p, f, 0.999928057f);
+    // bits(y) << 23 == rint(x) << 23 (mod 2^32): the constant part of y's
+    // bit pattern has no bits below position 22.
+    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(y) << 23));
 }
 
 // bounded wait that gives up at once when the CTA has already aborted
@@ -97,29 +128,30 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ Bars bars;
-    // 1024-byte aligned base for the swizzled tiles
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t q_s = sbase;
-    const uint32_t k_s = q_s + kTileBytes;
+    const uint32_t q_s = sbase;                   // [2 tiles][NB boxes]
+    const uint32_t k_s = q_s + 2 * kTileBytes;    // [STAGES][NB boxes]
     const uint32_t v_s = k_s + STAGES * kTileBytes;
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    const int qblk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
     const int nkv = (a.Lk + kBN - 1) / kBN;
+    const bool has_b = qblk * 2 * kBM + kBM < a.Lq;
+    const int ntiles = has_b ? 2 : 1;
 
-    if (threadIdx.x == 128) {
-        mbar_init(smem_u32(&bars.q_full), 1);
+    if (threadIdx.x == 256) {
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&bars.q_full[x]), 1);
+            mbar_init(smem_u32(&bars.s_full[x]), 1);
+            mbar_init(smem_u32(&bars.p_full[x]), 128);
+            mbar_init(smem_u32(&bars.o_done[x]), 1);
+        }
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&bars.k_full[s]), 1);
             mbar_init(smem_u32(&bars.v_full[s]), 1);
             mbar_init(smem_u32(&bars.kv_empty[s]), 1);
         }
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(smem_u32(&bars.s_full[s]), 1);
-            mbar_init(smem_u32(&bars.p_full[s]), 128);
-        }
-        mbar_init(smem_u32(&bars.o_done), 1);
         mbar_init(smem_u32(&bars.mma_done), 1);
         bars.abort = 0;
         fence_mbar_init();
@@ -128,7 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::prefetch_tmap(&tm_v);
         tc::prefetch_tmap(&tm_o);
     }
-    if (warp == 5) {
+    if (warp == 9) {
         tc::tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -138,13 +170,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem = bars.tmem_base;
     const int kvb = a.kv_batched ? b : 0;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             int issued[4] = {0, 0, 0, 0};
-            mbar_arrive_expect_tx(smem_u32(&bars.q_full), kTileBytes);
-            for (int bx = 0; bx < NB; ++bx)
-                tc::tma_load_4d(q_s + bx * kBox, &tm_q, bx * 64, h, qt * kBM, b, smem_u32(&bars.q_full));
+            for (int x = 0; x < ntiles; ++x) {
+                mbar_arrive_expect_tx(smem_u32(&bars.q_full[x]), kTileBytes);
+                for (int bx = 0; bx < NB; ++bx)
+                    tc::tma_load_4d(q_s + x * kTileBytes + bx * kBox, &tm_q, bx * 64, h,
+                                    (qblk * 2 + x) * kBM, b, smem_u32(&bars.q_full[x]));
+            }
             bool ok = true;
             for (int j = 0; j < nkv && ok; ++j) {
                 const int st = j % STAGES;
@@ -167,158 +202,191 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait_bounded(smem_u32(&bars.k_full[s]), (issued[s] - 1) & 1, &g_flash_err);
                         mbar_wait_bounded(smem_u32(&bars.v_full[s]), (issued[s] - 1) & 1, &g_flash_err);
                     }
-                mbar_wait_bounded(smem_u32(&bars.q_full), 0, &g_flash_err);
+                for (int x = 0; x < ntiles; ++x)
+                    mbar_wait_bounded(smem_u32(&bars.q_full[x]), 0, &g_flash_err);
             }
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
-            bool ok = wait_bar(&bars, &bars.q_full, 0);
-            auto issue_pv = [&](int j) -> bool {
+            auto issue_s = [&](int x, int j) {
                 const int st = j % STAGES;
-                if (!wait_bar(&bars, &bars.p_full[j & 1], (j >> 1) & 1)) return false;
-                if (!wait_bar(&bars, &bars.v_full[st], (j / STAGES) & 1)) return false;
-                tc::fence_after_sync();
-                const uint32_t p_tmem = tmem + ((j & 1) ? kS1 : kS0);
-#pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t bdesc =
-                        tc::smem_desc(v_s + st * kTileBytes + kk * 2048, kBox, 1024, 2);
-                    tc::mma_ts(tmem + kO, p_tmem + kk * 8, bdesc, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                }
-                tc::commit(smem_u32(&bars.kv_empty[st]));
-                tc::commit(smem_u32(&bars.o_done));
-                return true;
-            };
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j % STAGES;
-                ok = wait_bar(&bars, &bars.k_full[st], (j / STAGES) & 1);
-                if (!ok) break;
-                tc::fence_after_sync();
-                const uint32_t s_tmem = tmem + ((j & 1) ? kS1 : kS0);
+                const uint32_t qx = q_s + x * kTileBytes;
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const uint32_t off = (ks >> 2) * kBox + (ks & 3) * 32;
-                    const uint64_t adesc = tc::smem_desc(q_s + off, 16, 1024, 2);
+                    const uint64_t adesc = tc::smem_desc(qx + off, 16, 1024, 2);
                     const uint64_t bdesc = tc::smem_desc(k_s + st * kTileBytes + off, 16, 1024, 2);
-                    tc::mma_ss(s_tmem, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+                    tc::mma_ss(tmem + x * 128, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
                 }
-                tc::commit(smem_u32(&bars.s_full[j & 1]));
-                if (j > 0) ok = issue_pv(j - 1);
+                tc::commit(smem_u32(&bars.s_full[x]));
+            };
+            auto issue_pv = [&](int x, int j) {
+                const int st = j % STAGES;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk) {
+                    const uint64_t bdesc = tc::smem_desc(v_s + st * kTileBytes + kk * 2048, kBox, 1024, 2);
+                    tc::mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, idesc_o,
+                               (j > 0 || kk > 0) ? 1u : 0u);
+                }
+            };
+            bool ok = true;
+            for (int x = 0; x < ntiles && ok; ++x) ok = wait_bar(&bars, &bars.q_full[x], 0);
+            if (ok && nkv > 0) ok = wait_bar(&bars, &bars.k_full[0], 0);
+            if (ok && nkv > 0) {
+                tc::fence_after_sync();
+                for (int x = 0; x < ntiles; ++x) issue_s(x, 0);
             }
-            if (ok && nkv > 0) ok = issue_pv(nkv - 1);
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int st = j % STAGES;
+                const bool more = j + 1 < nkv;
+                ok = wait_bar(&bars, &bars.v_full[st], (j / STAGES) & 1);
+                if (ok && more) ok = wait_bar(&bars, &bars.k_full[(j + 1) % STAGES], ((j + 1) / STAGES) & 1);
+                for (int x = 0; x < ntiles && ok; ++x) {
+                    ok = wait_bar(&bars, &bars.p_full[x], j & 1);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    issue_pv(x, j);
+                    if (more)
+                        issue_s(x, j + 1);
+                    else
+                        tc::commit(smem_u32(&bars.o_done[x]));
+                }
+                if (ok) tc::commit(smem_u32(&bars.kv_empty[st]));
+            }
             // all MMAs this thread issued complete before TMEM is released
             tc::commit(smem_u32(&bars.mma_done));
             mbar_wait_bounded(smem_u32(&bars.mma_done), 0, &g_flash_err);
         }
     } else {
-        // ------------------------------------------------ softmax warps
-        const int row = warp * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)(warp * 32) << 16);
+        // ------------------------------------------------ softmax warpgroups
+        const int x = warp >> 2;  // tile
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        const uint32_t s_col = x * 128, o_col = 256 + x * 128;
         float m_ref = -INFINITY, l = 0.f;
-        bool ok = true;
-        for (int j = 0; j < nkv; ++j) {
-            ok = wait_bar(&bars, &bars.s_full[j & 1], (j >> 1) & 1);
+        bool ok = x < ntiles;
+        for (int j = 0; j < nkv && ok; ++j) {
+            ok = wait_bar(&bars, &bars.s_full[x], j & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            const uint32_t s_addr = lane_addr + ((j & 1) ? kS1 : kS0);
             float s[kBN];
-#pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[32];
-                tc::ld_32col(s_addr + c * 32, r);
+            {
+                uint32_t r0[32], r1[32], r2[32], r3[32];
+                tc::ld_32col(lane_addr + s_col + 0, r0);
+                tc::ld_32col(lane_addr + s_col + 32, r1);
+                tc::ld_32col(lane_addr + s_col + 64, r2);
+                tc::ld_32col(lane_addr + s_col + 96, r3);
                 tc::wait_ld();
 #pragma unroll
-                for (int i = 0; i < 32; ++i) s[c * 32 + i] = __uint_as_float(r[i]);
+                for (int i = 0; i < 32; ++i) {
+                    s[i] = __uint_as_float(r0[i]);
+                    s[32 + i] = __uint_as_float(r1[i]);
+                    s[64 + i] = __uint_as_float(r2[i]);
+                    s[96 + i] = __uint_as_float(r3[i]);
+                }
             }
             const int valid = a.Lk - j * kBN;  // keys of this tile that exist
-            float mt = -INFINITY;
+            if (valid < kBN) {
 #pragma unroll
-            for (int i = 0; i < kBN; ++i) {
-                s[i] = (i < valid) ? s[i] * a.scale_log2 : -INFINITY;
-                mt = fmaxf(mt, s[i]);
+                for (int i = 0; i < kBN; ++i)
+                    if (i >= valid) s[i] = -INFINITY;
             }
+            // row max of the raw scores (scale > 0 commutes with max): 8-way tree
+            float mx[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx[k] = s[k];
+#pragma unroll
+            for (int i = 8; i < kBN; i += 8)
+#pragma unroll
+                for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[i + k]);
+            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * a.scale_log2;
             if (j == 0) {
                 m_ref = mt;
             } else {
                 const bool need = mt > m_ref + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
+                    // PV_X(j-1) completed before S_X(j) did: O_X is stable here
                     const float m_new = need ? mt : m_ref;
                     const float f = ex2(m_ref - m_new);
-                    // O must hold PV_{j-1} before it is rescaled
-                    ok = wait_bar(&bars, &bars.o_done, (j - 1) & 1);
-                    if (!ok) break;
-                    tc::fence_after_sync();
 #pragma unroll
                     for (int c = 0; c < NO / 16; ++c) {
                         uint32_t r[16];
-                        tc::ld_16col(lane_addr + kO + c * 16, r);
+                        tc::ld_16col(lane_addr + o_col + c * 16, r);
                         tc::wait_ld();
 #pragma unroll
                         for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-                        tc::st_16col(lane_addr + kO + c * 16, r);
+                        tc::st_16col(lane_addr + o_col + c * 16, r);
                     }
                     l *= f;
                     m_ref = m_new;
                 }
             }
-            float rs = 0.f;
+            const float neg_m = -m_ref;
+            float acc[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
 #pragma unroll
             for (int c = 0; c < kBN / 32; ++c) {
                 uint32_t r[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const float p0 = ex2(s[c * 32 + 2 * i] - m_ref);
-                    const float p1 = ex2(s[c * 32 + 2 * i + 1] - m_ref);
-                    rs += p0 + p1;
-                    r[i] = pack_bf16x2(p0, p1);
+                    float p[2];
+#pragma unroll
+                    for (int e = 0; e < 2; ++e) {
+                        const int idx = c * 32 + 2 * i + e;
+                        const float t = fmaf(s[idx], a.scale_log2, neg_m);
+                        p[e] = ((idx & 7) < kPolyOf8) ? exp2_poly(t) : ex2(t);
+                        acc[idx & 7] += p[e];
+                    }
+                    r[i] = pack_bf16x2(p[0], p[1]);
                 }
-                tc::st_16col(s_addr + c * 16, r);
+                tc::st_16col(lane_addr + s_col + c * 16, r);
             }
-            l += rs;
+            l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
             tc::wait_st();
             tc::fence_before_sync();
-            mbar_arrive(smem_u32(&bars.p_full[j & 1]));
+            mbar_arrive(smem_u32(&bars.p_full[x]));
         }
         // ---------------- epilogue: O / l -> bf16 -> swizzled smem -> TMA store
-        if (ok && nkv > 0) ok = wait_bar(&bars, &bars.o_done, (nkv - 1) & 1);
+        if (ok && nkv > 0) ok = wait_bar(&bars, &bars.o_done[x], 0);
         if (ok) {
             tc::fence_after_sync();
             const float inv = 1.f / l;
-            unsigned char* stage = gen_base;  // reuse the Q tile (all S MMAs are done)
+            unsigned char* stage = gen_base + x * kTileBytes;  // this tile's Q buffer (all S MMAs done)
 #pragma unroll
             for (int c = 0; c < NO / 16; ++c) {
                 uint32_t r[16];
-                tc::ld_16col(lane_addr + kO + c * 16, r);
+                tc::ld_16col(lane_addr + o_col + c * 16, r);
                 tc::wait_ld();
                 uint32_t w[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
                     w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                // columns c*16 .. c*16+15 = two 16-byte chunks of box (c*16)/64
                 const int col = c * 16;
                 const int bx = col >> 6;
                 const int ch = (col & 63) >> 3;
                 unsigned char* rowp = stage + bx * kBox + row * 128;
-                *reinterpret_cast<uint4*>(rowp + (((ch) ^ (row & 7)) << 4)) =
-                    make_uint4(w[0], w[1], w[2], w[3]);
+                *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
                 *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
                     make_uint4(w[4], w[5], w[6], w[7]);
             }
             fence_proxy_async_smem();
         }
-        tc::named_bar_sync(1, 128);
+        tc::named_bar_sync(1 + x, 128);
         if (ok && row == 0) {
-            for (int bx = 0; bx < NB; ++bx) tc::tma_store_4d(&tm_o, q_s + bx * kBox, bx * 64, h, qt * kBM, b);
+            for (int bx = 0; bx < NB; ++bx)
+                tc::tma_store_4d(&tm_o, q_s + x * kTileBytes + bx * kBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
             bulk_commit();
             bulk_wait<0>();
         }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 5) {
+    if (warp == 9) {
         __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
@@ -364,7 +432,7 @@ cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtens
                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
     constexpr int STAGES = NB == 1 ? 3 : 2;
-    const size_t smem = (size_t)(1 + 2 * STAGES) * NB * kBox + 1024;
+    const size_t smem = (size_t)(2 + 2 * STAGES) * NB * kBox + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
     cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, STAGES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
@@ -379,8 +447,8 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
                          int Lk, int heads, int d, long long q_bstride, long long kv_bstride, cudaStream_t s) {
     if (Lq == 0 || batches == 0) return cudaSuccess;
     const long long C = (long long)heads * d;
-    const long long qtiles = (Lq + kBM - 1) / kBM;
-    if (qtiles > 0x7fffffffLL || batches > 65535 || heads > 65535 || Lq > 0x7fffffffLL)
+    const long long qblocks = (Lq + 2 * kBM - 1) / (2 * kBM);
+    if (qblocks > 0x7fffffffLL || batches > 65535 || heads > 65535 || Lq > 0x7fffffffLL)
         return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
     const long long kv_batches = kv_bstride > 0 ? batches : 1;
@@ -394,7 +462,7 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
     a.Lk = Lk;
     a.kv_batched = kv_bstride > 0 ? 1 : 0;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
-    dim3 grid((unsigned)qtiles, (unsigned)heads, (unsigned)batches);
+    dim3 grid((unsigned)qblocks, (unsigned)heads, (unsigned)batches);
     switch ((d + 15) / 16) {
         case 1: return launch_ks<1>(mq, mk, mv, mo, a, grid, s);
         case 2: return launch_ks<2>(mq, mk, mv, mo, a, grid, s);

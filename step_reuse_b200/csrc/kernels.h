@@ -28,6 +28,7 @@ unsigned int layout_device_errors(bool clear);
 // --- temporal short-sequence attention ([N,T,C], L = T) -------------------
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
                             int heads, int d, cudaStream_t s);
+unsigned int temporal_device_errors(bool clear);
 
 // --- flash attention for spatial (per frame) and cross (shared text K/V) --
 // Rows of batch b, head h: q + b*q_bstride + i*C + h*d (elements); likewise
@@ -36,9 +37,6 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
                          long long Lq, int Lk, int heads, int d, long long q_bstride,
                          long long kv_bstride, cudaStream_t s);
 
-cudaError_t launch_flash_mma(const void* q, const void* k, const void* v, void* out, int batches,
-                             long long Lq, int Lk, int heads, int d, long long q_bstride,
-                             long long kv_bstride, cudaStream_t s);
 unsigned int flash_device_errors(bool clear);
 
 // --- dtype conversion for fp32 plans --------------------------------------

@@ -378,8 +378,13 @@ int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype, doub
 int pab_device_errors(int clear, unsigned int* flags) {
     PAB_GUARD_BEGIN
     if (!flags) return fail(PAB_ERR_ARG, "null flags pointer");
-    const unsigned int v = pab::layout_device_errors(clear != 0);
-    if (v == 0xffffffffu) return fail(PAB_ERR_CUDA, "could not read the device status word");
+    const unsigned int words[3] = {pab::layout_device_errors(clear != 0), pab::flash_device_errors(clear != 0),
+                                   pab::temporal_device_errors(clear != 0)};
+    unsigned int v = 0;
+    for (unsigned int w : words) {
+        if (w == 0xffffffffu) return fail(PAB_ERR_CUDA, "could not read the device status words");
+        v |= w;
+    }
     *flags = v;
     return PAB_OK;
     PAB_GUARD_END

@@ -6,19 +6,24 @@
 // (2 * T * d * 2 flop per loaded byte ~ 8-32 flop/B).
 //
 // Design:
-//  - persistent grid; a unit of work is (position n, group of G heads); the
-//    unit's q, k, v rows (T rows of G*d contiguous channels each) stream into
-//    shared memory with 16-byte cp.async, double-buffered across units, so
-//    the next unit's loads overlap this unit's math;
+//  - persistent grid; a unit of work is (position n, group of G heads); one
+//    thread streams the unit's q, k, v into shared memory with TMA tensor
+//    loads (one [T rows][P cols] box per tensor and head), double-buffered
+//    across units so the next unit's loads overlap this unit's math, and
+//    writes the unit's output back with TMA tensor stores;
 //  - one warp per (head, 16-query tile): QK^T and PV run on warp-level bf16
 //    MMA (m16n8k16, fp32 accumulate) from ldmatrix fragments; the softmax is
 //    an online (streaming) softmax over 16-key blocks with quad shuffles;
-//  - shared-memory rows have a pitch of P elements with P/8 odd, so the eight
-//    16-byte rows an ldmatrix phase reads hit distinct banks;
-//  - outputs are staged in the q buffer and written back with coalesced
-//    16-byte stores.
-#include "common.cuh"
+//  - a head's rows have a pitch of P elements with P/8 odd (P = d or d + 8),
+//    so the eight 16-byte rows an ldmatrix phase reads hit distinct banks;
+//    the tensor map's innermost extent is d, so columns d..P-1 load as zero;
+//    rows T..RT-1 (RT = T rounded up to 16) stay zero from the start.
+// Waits on the stage barriers are bounded; on time-out the CTA raises the
+// error word and stops after its copies in flight have landed.
+#include <cuda.h>
+
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace pab {
 namespace {
@@ -28,14 +33,12 @@ constexpr int kThreads = kWarps * 32;
 constexpr int kMaxStageBytes = 56 * 1024;
 constexpr float kLog2e = 1.4426950408889634f;
 
+__device__ unsigned int g_temporal_err = 0;
+
 struct TemporalArgs {
-    const __nv_bfloat16* q;
-    const __nv_bfloat16* k;
-    const __nv_bfloat16* v;
-    __nv_bfloat16* out;
     int N, T, heads, d;
     int G;       // heads per unit
-    int P;       // smem row pitch (elements)
+    int P;       // smem row pitch (elements) = TMA box width
     int RT;      // rows per head block in smem (T rounded up to 16)
     long long units;
     float scale_log2;  // log2(e) / sqrt(d)
@@ -49,61 +52,85 @@ PAB_DEV float ex2(float x) {
 
 // smem layout of one stage: [3 tensors][G heads][RT rows][P cols] bf16
 template <int DN>
-__global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs p) {
+__global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constant__ CUtensorMap tm_q,
+                                                            const __grid_constant__ CUtensorMap tm_k,
+                                                            const __grid_constant__ CUtensorMap tm_v,
+                                                            const __grid_constant__ CUtensorMap tm_o,
+                                                            TemporalArgs p) {
     extern __shared__ __align__(128) unsigned char smem[];
+    __shared__ __align__(8) unsigned long long full_bar[2];
+    __shared__ int abort_flag;
     constexpr int DK = (DN + 1) / 2;  // 16-wide k chunks covering d
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int G = p.G, P = p.P, RT = p.RT, T = p.T, d = p.d;
-    const long long C = (long long)p.heads * d;
+    const int G = p.G, P = p.P, RT = p.RT, T = p.T;
     const int head_elems = RT * P;
     const int tensor_elems = G * head_elems;
     const int stage_elems = 3 * tensor_elems;
-    const int chunks_per_row = d / 8;
     const int hg_count = p.heads / G;
+    const uint32_t unit_bytes = 3u * G * T * P * 2;
 
-    // zero both stages once: padding rows/cols are never written afterwards
+    // zero both stages once: padding rows are never written afterwards
     {
         uint4* z = reinterpret_cast<uint4*>(smem);
         const int n16 = (2 * stage_elems * 2 + 256) / 16;
         for (int i = tid; i < n16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
     }
+    if (tid == 0) {
+        mbar_init(smem_u32(&full_bar[0]), 1);
+        mbar_init(smem_u32(&full_bar[1]), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+        tc::prefetch_tmap(&tm_q);
+        tc::prefetch_tmap(&tm_k);
+        tc::prefetch_tmap(&tm_v);
+        tc::prefetch_tmap(&tm_o);
+    }
+    // generic-proxy zeroing must be visible to the async proxy (TMA writes)
+    fence_proxy_async_smem();
     __syncthreads();
 
     __nv_bfloat16* sbase = reinterpret_cast<__nv_bfloat16*>(smem);
+    const uint32_t sbase_u32 = smem_u32(smem);
     auto issue_unit = [&](long long unit, int stage) {
-        const long long n = unit / hg_count;
-        const int h0 = (int)(unit - n * hg_count) * G;
-        __nv_bfloat16* st = sbase + stage * stage_elems;
-        const int per_tensor = T * G * chunks_per_row;
-        for (int c = tid; c < 3 * per_tensor; c += kThreads) {
-            const int tsr = c / per_tensor;
-            int r = c - tsr * per_tensor;
-            const int t = r / (G * chunks_per_row);
-            r -= t * (G * chunks_per_row);
-            const int g = r / chunks_per_row;
-            const int ch = r - g * chunks_per_row;
-            const __nv_bfloat16* src = (tsr == 0 ? p.q : (tsr == 1 ? p.k : p.v)) +
-                                       ((n * T + t) * C + (long long)(h0 + g) * d + ch * 8);
-            __nv_bfloat16* dst = st + tsr * tensor_elems + g * head_elems + t * P + ch * 8;
-            cp_async16(smem_u32(dst), src, 16);
-        }
+        const int n = (int)(unit / hg_count);
+        const int h0 = (int)(unit - (long long)n * hg_count) * G;
+        const uint32_t bar = smem_u32(&full_bar[stage]);
+        mbar_arrive_expect_tx(bar, unit_bytes);
+        const CUtensorMap* maps[3] = {&tm_q, &tm_k, &tm_v};
+        for (int tsr = 0; tsr < 3; ++tsr)
+            for (int g = 0; g < G; ++g)
+                tc::tma_load_4d(sbase_u32 + 2u * (stage * stage_elems + tsr * tensor_elems + g * head_elems),
+                                maps[tsr], 0, h0 + g, 0, n, bar);
     };
 
     const long long first = blockIdx.x, step = gridDim.x;
-    if (first < p.units) issue_unit(first, 0);
-    cp_async_commit();
+    int issued[2] = {0, 0};
+    if (tid == 0 && first < p.units) {
+        issue_unit(first, 0);
+        issued[0] = 1;
+    }
 
     const int mtiles = RT / 16;
     const int tasks = G * mtiles;
+    int waited[2] = {0, 0};
     for (long long i = 0;; ++i) {
         const long long u = first + i * step;
         if (u >= p.units) break;
         const int stage = (int)(i & 1);
-        const long long nu = u + step;
-        if (nu < p.units) issue_unit(nu, stage ^ 1);
-        cp_async_commit();
-        cp_async_wait<1>();
+        if (tid == 0) {
+            const long long nu = u + step;
+            if (nu < p.units) {
+                // the other stage held unit i-1: its output store must have read it
+                bulk_wait_read<0>();
+                issue_unit(nu, stage ^ 1);
+                issued[stage ^ 1] += 1;
+            }
+        }
+        if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), (uint32_t)(waited[stage] & 1), &g_temporal_err))
+            abort_flag = 1;
+        waited[stage] += 1;
         __syncthreads();
+        if (abort_flag) break;
 
         __nv_bfloat16* st = sbase + stage * stage_elems;
         for (int task = warp; task < tasks; task += kWarps) {
@@ -112,12 +139,11 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs p) {
             const __nv_bfloat16* ks = st + tensor_elems + g * head_elems;
             const __nv_bfloat16* vs = st + 2 * tensor_elems + g * head_elems;
 
-            // Q fragments for this 16-row tile
             uint32_t qa[DK][4];
 #pragma unroll
             for (int kc = 0; kc < DK; ++kc)
-                ldsm_x4(smem_u32(qs + (lane & 15) * P + kc * 16 + (lane >> 4) * 8), qa[kc][0],
-                        qa[kc][1], qa[kc][2], qa[kc][3]);
+                ldsm_x4(smem_u32(qs + (lane & 15) * P + kc * 16 + (lane >> 4) * 8), qa[kc][0], qa[kc][1],
+                        qa[kc][2], qa[kc][3]);
             if (DN & 1) {  // d % 16 == 8: the last chunk's upper 8 columns are past d
                 qa[DK - 1][2] = 0u;
                 qa[DK - 1][3] = 0u;
@@ -140,7 +166,6 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs p) {
                     mma_bf16_16816(s[0], qa[kc][0], qa[kc][1], qa[kc][2], qa[kc][3], b0, b1);
                     mma_bf16_16816(s[1], qa[kc][0], qa[kc][1], qa[kc][2], qa[kc][3], b2, b3);
                 }
-                // scale, mask keys >= T, online softmax (rows r and r+8)
                 float mx0 = m0, mx1 = m1;
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
@@ -205,38 +230,62 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(TemporalArgs p) {
             const int r0 = lane >> 2, cq = 2 * (lane & 3);
 #pragma unroll
             for (int j = 0; j < DN; ++j) {
-                *reinterpret_cast<uint32_t*>(qs + r0 * P + j * 8 + cq) =
-                    pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
+                *reinterpret_cast<uint32_t*>(qs + r0 * P + j * 8 + cq) = pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
                 *reinterpret_cast<uint32_t*>(qs + (r0 + 8) * P + j * 8 + cq) =
                     pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
             }
         }
+        fence_proxy_async_smem();
         __syncthreads();
-        // coalesced write-back of the unit's outputs
-        {
-            const long long n = u / hg_count;
-            const int h0 = (int)(u - n * hg_count) * G;
-            const int per = T * G * chunks_per_row;
-            for (int c = tid; c < per; c += kThreads) {
-                const int t = c / (G * chunks_per_row);
-                int r = c - t * (G * chunks_per_row);
-                const int g = r / chunks_per_row;
-                const int ch = r - g * chunks_per_row;
-                const uint4 val = *reinterpret_cast<const uint4*>(st + g * head_elems + t * P + ch * 8);
-                __stcs(reinterpret_cast<uint4*>(p.out + ((n * T + t) * C + (long long)(h0 + g) * d +
-                                                        ch * 8)),
-                       val);
-            }
+        if (tid == 0) {
+            const int n = (int)(u / hg_count);
+            const int h0 = (int)(u - (long long)n * hg_count) * G;
+            for (int g = 0; g < G; ++g)
+                tc::tma_store_4d(&tm_o, sbase_u32 + 2u * (stage * stage_elems + g * head_elems), 0, h0 + g, 0, n);
+            bulk_commit();
         }
-        __syncthreads();
     }
-    cp_async_wait<0>();
+    if (tid == 0) {
+        if (abort_flag) {
+            // let every load this CTA issued land before it exits (bounded)
+            for (int s = 0; s < 2; ++s)
+                if (issued[s] > waited[s])
+                    mbar_wait_bounded(smem_u32(&full_bar[s]), (uint32_t)((issued[s] - 1) & 1), &g_temporal_err);
+        }
+        bulk_wait<0>();
+    }
+}
+
+// 4-D map over [N][T][heads][d] (row stride C): dims (d, heads, T, N),
+// box (P, 1, T, 1), no swizzle; columns d..P-1 of the box read as zero.
+bool make_map(CUtensorMap* m, const void* base, int d, int heads, int T, int N, int P) {
+    typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                      const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
+                                      CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
+                                      CUtensorMapFloatOOBfill);
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return false;
+        fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    const long long C = (long long)heads * d;
+    cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)N};
+    cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)C * 2, (cuuint64_t)T * C * 2};
+    cuuint32_t box[4] = {(cuuint32_t)P, 1, (cuuint32_t)T, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int DN>
-cudaError_t launch_dn(const TemporalArgs& p, size_t smem, cudaStream_t s) {
-    cudaError_t e = cudaFuncSetAttribute(temporal_kernel<DN>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+cudaError_t launch_dn(const CUtensorMap* maps, const TemporalArgs& p, size_t smem, cudaStream_t s) {
+    cudaError_t e = cudaFuncSetAttribute(temporal_kernel<DN>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, temporal_kernel<DN>, kThreads, smem);
@@ -244,7 +293,7 @@ cudaError_t launch_dn(const TemporalArgs& p, size_t smem, cudaStream_t s) {
     if (per_sm < 1) per_sm = 1;
     long long grid = (long long)device_sm_count() * per_sm;
     if (grid > p.units) grid = p.units;
-    temporal_kernel<DN><<<(unsigned)grid, kThreads, smem, s>>>(p);
+    temporal_kernel<DN><<<(unsigned)grid, kThreads, smem, s>>>(maps[0], maps[1], maps[2], maps[3], p);
     return cudaGetLastError();
 }
 
@@ -253,10 +302,6 @@ cudaError_t launch_dn(const TemporalArgs& p, size_t smem, cudaStream_t s) {
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
                             int heads, int d, cudaStream_t s) {
     TemporalArgs p;
-    p.q = static_cast<const __nv_bfloat16*>(q);
-    p.k = static_cast<const __nv_bfloat16*>(k);
-    p.v = static_cast<const __nv_bfloat16*>(v);
-    p.out = static_cast<__nv_bfloat16*>(out);
     p.N = N;
     p.T = T;
     p.heads = heads;
@@ -274,11 +319,15 @@ cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* o
     p.units = (long long)N * (heads / G);
     p.scale_log2 = kLog2e / sqrtf((float)d);
     if (p.units == 0) return cudaSuccess;
+    CUtensorMap maps[4];
+    const void* bases[4] = {q, k, v, out};
+    for (int i = 0; i < 4; ++i)
+        if (!make_map(&maps[i], bases[i], d, heads, T, N, p.P)) return cudaErrorInvalidValue;
     const size_t smem = (size_t)2 * 3 * G * p.RT * p.P * 2 + 256;
     switch (d / 8) {
 #define PAB_T_CASE(DNV) \
     case DNV:           \
-        return launch_dn<DNV>(p, smem, s);
+        return launch_dn<DNV>(maps, p, smem, s);
         PAB_T_CASE(1) PAB_T_CASE(2) PAB_T_CASE(3) PAB_T_CASE(4) PAB_T_CASE(5) PAB_T_CASE(6)
         PAB_T_CASE(7) PAB_T_CASE(8) PAB_T_CASE(9) PAB_T_CASE(10) PAB_T_CASE(11) PAB_T_CASE(12)
         PAB_T_CASE(13) PAB_T_CASE(14) PAB_T_CASE(15) PAB_T_CASE(16)
@@ -286,6 +335,16 @@ cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* o
         default:
             return cudaErrorInvalidValue;
     }
+}
+
+unsigned int temporal_device_errors(bool clear) {
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_temporal_err, sizeof(v)) != cudaSuccess) return 0xffffffffu;
+    if (clear && v) {
+        unsigned int z = 0;
+        cudaMemcpyToSymbol(g_temporal_err, &z, sizeof(z));
+    }
+    return v;
 }
 
 }  // namespace pab

@@ -1,0 +1,60 @@
+"""The flash kernel's software exp2 (exp2_poly in flash_tc.cu), emulated bit
+for bit in numpy float32 with the coefficients read from the kernel source,
+against numpy's exp2 in float64 over the whole input range the softmax
+produces (x <= 8; x < -120 clamped).  The kernel moves part of the softmax
+exponentials from the MUFU unit to the FMA pipes with it; its error must stay
+far below the bf16 rounding (2^-9) that P receives right after."""
+import os
+import re
+
+import numpy as np
+
+SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
+                   "step_reuse_b200", "csrc", "flash_tc.cu")
+
+
+def kernel_coefficients():
+    text = open(SRC).read()
+    body = text[text.index("PAB_DEV float exp2_poly"):]
+    body = body[:body.index("\n}\n")]
+    c3, c2 = re.search(r"fmaf\(([-0-9.e]+)f, f, ([-0-9.e]+)f\)", body).groups()
+    c1 = re.search(r"fmaf\(p, f, ([-0-9.e]+)f\);\s*p = fmaf\(p, f", body).group(1)
+    c0 = re.findall(r"fmaf\(p, f, ([-0-9.e]+)f\)", body)[-1]
+    return [np.float32(c) for c in (c0, c1, c2, c3)]
+
+
+def exp2_poly_emulated(x):
+    c0, c1, c2, c3 = kernel_coefficients()
+    x = np.maximum(np.asarray(x, np.float32), np.float32(-120.0))
+    magic = np.float32(12582912.0)
+    y = (x + magic).astype(np.float32)
+    n = (y - magic).astype(np.float32)
+    f = (x - n).astype(np.float32)
+    # fmaf is fused: emulate each step in float64 then round to float32
+    p = np.float32(np.float64(c3) * f + np.float64(c2))
+    p = np.float32(np.float64(p) * f + np.float64(c1))
+    p = np.float32(np.float64(p) * f + np.float64(c0))
+    bits = (p.view(np.uint32).astype(np.uint64) + (y.view(np.uint32).astype(np.uint64) << 23)) & 0xFFFFFFFF
+    return bits.astype(np.uint32).view(np.float32)
+
+
+def test_exp2_poly_relative_error():
+    x = np.concatenate([np.linspace(-120.0, 8.0, 2_000_001, dtype=np.float64),
+                        np.arange(-120, 9, dtype=np.float64) + 0.5,
+                        np.arange(-120, 9, dtype=np.float64)]).astype(np.float32)
+    got = exp2_poly_emulated(x).astype(np.float64)
+    want = np.exp2(x.astype(np.float64))
+    rel = np.abs(got / want - 1.0)
+    assert rel.max() < 1e-4, rel.max()
+    assert rel.max() < 2.0 ** -9 / 20
+
+
+def test_exp2_poly_clamps_and_orders():
+    v = exp2_poly_emulated(np.array([-np.inf, -1000.0, -121.0, -120.0, 0.0, 8.0], np.float32))
+    assert np.isfinite(v).all() and (v >= 0).all()
+    assert v[0] == v[1] == v[2] == v[3] and v[3] < 1e-35
+    assert abs(v[4] - 1.0) < 1e-4 and abs(v[5] / 256.0 - 1.0) < 1e-4
+    # monotone on a fine grid (no jumps at the integer boundaries of the reduction)
+    x = np.linspace(-20.0, 8.0, 200_001, dtype=np.float32)
+    y = exp2_poly_emulated(x)
+    assert (np.diff(y.astype(np.float64)) >= -1e-6 * y[1:]).all()
