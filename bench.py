@@ -50,7 +50,7 @@ MEASURED_TRAFFIC = {}
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny"))
@@ -121,7 +121,7 @@ def kernel_source_hash(name: str) -> str:
 class ClockSampler:
     """nvidia-smi clocks / throttle reasons sampled during the timed region."""
 
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -130,6 +130,13 @@ class ClockSampler:
         self.proc = None
         self.lines = []
         self._t = None
+        self.t_start = self.t_end = None
+
+    def mark_start(self):
+        self.t_start = time.time()
+
+    def mark_end(self):
+        self.t_end = time.time()
 
     def start(self):
         try:
@@ -145,7 +152,7 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
 
     def stop(self):
         if self.proc is None:
@@ -159,7 +166,11 @@ class ClockSampler:
             self._t.join(timeout=2)
         sm, mx, reasons = [], None, set()
         names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
-        for ln in self.lines:
+        lo = (self.t_start or 0.0) - 0.05
+        hi = (self.t_end or 1e30) + 0.25  # a sample is printed up to one period late
+        for ts, ln in self.lines:
+            if not (lo <= ts <= hi):
+                continue
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 9:
                 continue
@@ -211,48 +222,50 @@ class AttentionStack:
         return n
 
     def run(self, inputs, stream, events=None):
-        """inputs[i][kind] -> dict q,k,v (spatial view for temporal)."""
+        """inputs[i][kind] -> dict q,k,v (spatial view for temporal).  With
+        `events` (name -> ([starts], [ends])), every launch is bracketed by
+        CUDA events on `stream`, grouped by kernel."""
         pab, w, plan = self.pab, self.w, self.plan
         plan.reset()
         prev = {}
         T, N, C = w.T, w.N, w.C
+
+        def timed(name, fn):
+            if events is None:
+                return fn()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            r = fn()
+            b.record(stream)
+            events.setdefault(name, ([], []))
+            events[name][0].append(a)
+            events[name][1].append(b)
+            return r
+
         for i in range(w.steps):
             x = inputs[i % len(inputs)]
             for ki, k in enumerate(synth.KINDS):
-                comp = self.sched[k][i]
-                if not comp:
+                if not self.sched[k][i]:
                     self.last_ptr[k] = plan.attention_ptr(k, i, None, None, None, stream)
                     continue
-                ev = events[k] if events is not None else None
-                if ev is not None:
-                    ev[0].append(torch.cuda.Event(enable_timing=True))
-                    ev[0][-1].record(stream)
                 if k == "temporal":
-                    pab.layout(x[k]["q"], True, out=self.tq, stream=stream)
-                    pab.layout(x[k]["k"], True, out=self.tk, stream=stream)
-                    pab.layout(x[k]["v"], True, out=self.tv, stream=stream)
-                    if events is not None:
-                        events["temporal_attn"][0].append(torch.cuda.Event(enable_timing=True))
-                        events["temporal_attn"][0][-1].record(stream)
-                    ptr = plan.attention_ptr(k, i, self.tq, self.tk, self.tv, stream)
+                    for src, dst in ((x[k]["q"], self.tq), (x[k]["k"], self.tk), (x[k]["v"], self.tv)):
+                        timed("layout", lambda: pab.layout(src, True, out=dst, stream=stream))
+                    ptr = timed("temporal", lambda: plan.attention_ptr(k, i, self.tq, self.tk, self.tv, stream))
                     self.last_ptr[k] = ptr
-                    if events is not None:
-                        events["temporal_attn"][1].append(torch.cuda.Event(enable_timing=True))
-                        events["temporal_attn"][1][-1].record(stream)
                     t_out = pab._wrap(ptr, (N, T, C), torch.bfloat16, self.dev)
                     self.tslot ^= 1
-                    pab.layout(t_out, False, out=self.tout[self.tslot], stream=stream)
+                    timed("layout", lambda: pab.layout(t_out, False, out=self.tout[self.tslot], stream=stream))
                     cur = self.tout[self.tslot]
                 else:
-                    ptr = plan.attention_ptr(k, i, x[k]["q"], x[k]["k"], x[k]["v"], stream)
+                    ptr = timed(k, lambda: plan.attention_ptr(k, i, x[k]["q"], x[k]["k"], x[k]["v"], stream))
                     self.last_ptr[k] = ptr
                     shape = (T, N, C) if k == "spatial" else (T * N, C)
                     cur = pab._wrap(ptr, shape, torch.bfloat16, self.dev)
-                if ev is not None:
-                    ev[1].append(torch.cuda.Event(enable_timing=True))
-                    ev[1][-1].record(stream)
                 if k in prev:
-                    pab.attn_diff_mse_async(cur, prev[k], self.mse[ki, i:i + 1], stream=stream)
+                    timed("mse", lambda: pab.attn_diff_mse_async(cur, prev[k], self.mse[ki, i:i + 1],
+                                                                stream=stream))
                 prev[k] = cur
 
     def close(self):
@@ -388,27 +401,27 @@ def run_ours(args):
     torch.cuda.synchronize(device)
     assert pab.device_errors() == 0
 
-    events = {k: ([], []) for k in synth.KINDS}
-    events["temporal_attn"] = ([], [])
+    events = {}
     clocks = ClockSampler(local)
     clocks.start()
+    time.sleep(0.5)  # let the sampler start before the timed region
     barrier(device)
     torch.cuda.synchronize(device)
     t0 = torch.cuda.Event(enable_timing=True)
     t1 = torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
     t0.record(stream)
     for _ in range(args.steps):
         stack.run(inputs, stream, events)
     t1.record(stream)
     torch.cuda.synchronize(device)
+    clocks.mark_end()
     barrier(device)
     clk = clocks.stop()
     ms = t0.elapsed_time(t1) / args.steps
     ms = max_over_ranks(ms, device)
     assert pab.device_errors() == 0
 
-    per_kind_ms = {k: mean_ms(events[k]) for k in synth.KINDS}
-    t_attn_ms = mean_ms(events["temporal_attn"])
     peaks = {}
     try:
         peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
@@ -417,27 +430,29 @@ def run_ours(args):
         peak_src = "fallback"
     tc_peak = peaks.get("bf16_tflops_sustained", 1400.0)
     hbm_peak = peaks.get("hbm_gbs", 6650.0)
-    sp_ms = per_kind_ms["spatial"]
+    kms = {name: mean_ms(ev) for name, ev in events.items()}
+    kernels = {}
+    for name in ("spatial", "cross", "temporal", "layout", "mse"):
+        t = kms.get(name)
+        if not t:
+            continue
+        fl = flops.get(name, 0.0) if name != "layout" and name != "mse" else 0.0
+        by = abytes[name]
+        ent = {"ms": t, "launches_per_run": len(events[name][0]) // args.steps,
+               "gbs": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
+        if fl:
+            ent["tflops"] = fl / (t * 1e-3) / 1e12
+            ent["frac_tc"] = ent["tflops"] / tc_peak
+        kernels[name] = ent
+    sp_ms = kms["spatial"]
     achieved = flops["spatial"] / (sp_ms * 1e-3) / 1e12
     src_hash = kernel_source_hash("flash_tc.cu")
     traffic = MEASURED_TRAFFIC.get(src_hash)
-    roofline = {"kernel": "spatial flash attention", "bound": "tensor", "achieved": achieved,
+    roofline = {"kernel": "spatial flash attention (flash_tc)", "bound": "tensor", "achieved": achieved,
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops_sustained",
-                "algorithmic_flops_per_launch": flops["spatial"]}
-    kernels = {
-        "spatial": {"ms": sp_ms, "tflops": achieved, "frac_tc": achieved / tc_peak},
-        "temporal_attention": {"ms": t_attn_ms,
-                               "gbs": abytes["temporal"] / (t_attn_ms * 1e-3) / 1e9 if t_attn_ms else None},
-        "temporal_with_layouts": {"ms": per_kind_ms["temporal"]},
-        "cross": {"ms": per_kind_ms["cross"],
-                  "gbs": abytes["cross"] / (per_kind_ms["cross"] * 1e-3) / 1e9,
-                  "tflops": flops["cross"] / (per_kind_ms["cross"] * 1e-3) / 1e12},
-    }
-    for name in ("temporal_attention", "cross"):
-        g = kernels[name].get("gbs")
-        if g:
-            kernels[name]["frac_hbm"] = g / hbm_peak
+                "algorithmic_flops_per_launch": flops["spatial"],
+                "algorithmic_bytes_per_launch": abytes["spatial"]}
 
     value = world * dense_flops / (ms * 1e-3) / 1e12
     line = {

@@ -7,7 +7,8 @@
 // A CTA owns 256 query rows of one (batch, head) as two 128-row tiles A and B
 // that share every K/V tile, and runs four roles:
 //   warp 8 (one thread)   TMA producer: Q_A, Q_B once, then K_j / V_j tiles of
-//                          128 keys into a STAGES-deep shared-memory ring;
+//                          128 keys into separate shared-memory rings, K two
+//                          tiles ahead of V (K is consumed one step earlier);
 //   warp 9 (one thread)   MMA issuer: S_X = Q_X K_j^T (SS form, fp32 in TMEM)
 //                          and O_X += P_X V_j (TS form: P from TMEM, V from
 //                          shared memory), ping-ponging between the tiles:
@@ -20,8 +21,8 @@
 //                          reductions, no shuffles), writes P as bf16 over S's
 //                          columns and rescales O in TMEM only when the running
 //                          max grew by more than 2^8 (the final O / l is exact
-//                          either way).  Exponentials: most on the MUFU ex2
-//                          unit, a fixed share on the FMA pipes (exp2_poly).
+//                          either way).  Exponentials: 5/8 on the MUFU ex2
+//                          unit, 3/8 on the FMA pipes (exp2_poly2).
 //                          At the end it normalises O and writes it through
 //                          shared memory with a TMA tensor store.
 // When S_X(j) completes, every earlier MMA of the issuing thread -- PV_X(j-1)
@@ -54,9 +55,15 @@ constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
 constexpr int kThreads = 320;     // 2 softmax warpgroups + producer warp + MMA warp
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
-// Of every 8 consecutive scores of a row, this many take exp2_poly (FMA
-// pipes), the rest the MUFU ex2 unit.
-constexpr int kPolyOf8 = 3;
+// Exponentials: of every 8 consecutive pairs of a row's scores, this many go
+// to exp2_poly2 on the FMA pipes and the rest to the MUFU ex2 unit, which
+// alone would bound the softmax (16 results per clock per SM).
+#ifndef PAB_POLY_PAIRS_OF_8
+#define PAB_POLY_PAIRS_OF_8 3
+#endif
+constexpr int kPolyPairsOf8 = PAB_POLY_PAIRS_OF_8;
+// 2^f ~ kP0 + kP1 f + kP2 f^2 + kP3 f^3 on [-0.5, 0.5] (see exp2_poly2)
+constexpr float kP0 = 0.999928057f, kP1 = 0.693260968f, kP2 = 0.242611125f, kP3 = 0.0551716685f;
 
 __device__ unsigned int g_flash_err = 0;
 
@@ -71,7 +78,8 @@ struct Bars {
     unsigned long long q_full[2];
     unsigned long long k_full[4];
     unsigned long long v_full[4];
-    unsigned long long kv_empty[4];
+    unsigned long long k_empty[4];
+    unsigned long long v_empty[4];
     unsigned long long s_full[2];
     unsigned long long p_full[2];
     unsigned long long o_done[2];
@@ -86,25 +94,29 @@ PAB_DEV float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA/ALU pipes, for x <= 8 (the lazily rescaled softmax never
-// exceeds 2^8).  Cody-Waite style range reduction: x = n + f with n = rint(x)
-// (the 1.5*2^23 rounding trick) and f in [-0.5, 0.5]; 2^f from a degree-3
-// polynomial fitted here by minimising the maximum relative error on
-// [-0.5, 0.5] (linear-programming minimax fit; max relative error 7.5e-5,
-// far below the bf16 rounding of P); 2^n is added to the exponent field.
-// x below -120 is clamped (the result, ~1e-36, is negligible next to the
-// row maximum's weight 1).
-PAB_DEV float exp2_poly(float x) {
-    x = fmaxf(x, -120.0f);
-    const float y = x + 12582912.0f;  // 1.5 * 2^23
-    const float n = y - 12582912.0f;  // rint(x)
-    const float f = x - n;
-    float p = fmaf(0.0551716685f, f, 0.242611125f);
-    p = fmaf(p, f, 0.693260968f);
-    p = fmaf(p, f, 0.999928057f);
+// 2^x on the FMA/ALU pipes for two values at once, for x <= 8 (the lazily
+// rescaled softmax never exceeds 2^8).  Cody-Waite style range reduction:
+// x = n + f with n = rint(x) (the 1.5*2^23 rounding trick) and f in
+// [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted here by minimising the
+// maximum relative error on [-0.5, 0.5] (linear-programming minimax fit; max
+// relative error 7.5e-5, far below the bf16 rounding of P); 2^n is added to
+// the exponent field.  x below -120 is clamped (the result, ~1e-36, is
+// negligible next to the row maximum's weight 1).
+PAB_DEV void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+    const tc::f32x2 x = tc::pack2(fmaxf(x0, -120.0f), fmaxf(x1, -120.0f));
+    const tc::f32x2 magic = tc::pack2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    const tc::f32x2 y = tc::add2(x, magic);
+    const tc::f32x2 f = tc::sub2(x, tc::sub2(y, magic));  // x - rint(x)
+    tc::f32x2 p = tc::fma2(tc::pack2(kP3, kP3), f, tc::pack2(kP2, kP2));
+    p = tc::fma2(p, f, tc::pack2(kP1, kP1));
+    p = tc::fma2(p, f, tc::pack2(kP0, kP0));
+    float q0, q1, y0, y1;
+    tc::unpack2(p, q0, q1);
+    tc::unpack2(y, y0, y1);
     // bits(y) << 23 == rint(x) << 23 (mod 2^32): the constant part of y's
     // bit pattern has no bits below position 22.
-    return __uint_as_float(__float_as_uint(p) + (__float_as_uint(y) << 23));
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(y0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(y1) << 23));
 }
 
 // bounded wait that gives up at once when the CTA has already aborted
@@ -117,7 +129,7 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
     return true;
 }
 
-template <int KSTEPS, int STAGES>
+template <int KSTEPS, int KST, int VST>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -130,8 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     __shared__ Bars bars;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
     const uint32_t q_s = sbase;                   // [2 tiles][NB boxes]
-    const uint32_t k_s = q_s + 2 * kTileBytes;    // [STAGES][NB boxes]
-    const uint32_t v_s = k_s + STAGES * kTileBytes;
+    const uint32_t k_s = q_s + 2 * kTileBytes;    // [KST][NB boxes]
+    const uint32_t v_s = k_s + KST * kTileBytes;  // [VST][NB boxes]
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -147,10 +159,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&bars.p_full[x]), 128);
             mbar_init(smem_u32(&bars.o_done[x]), 1);
         }
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < KST; ++s) {
             mbar_init(smem_u32(&bars.k_full[s]), 1);
+            mbar_init(smem_u32(&bars.k_empty[s]), 1);
+        }
+        for (int s = 0; s < VST; ++s) {
             mbar_init(smem_u32(&bars.v_full[s]), 1);
-            mbar_init(smem_u32(&bars.kv_empty[s]), 1);
+            mbar_init(smem_u32(&bars.v_empty[s]), 1);
         }
         mbar_init(smem_u32(&bars.mma_done), 1);
         bars.abort = 0;
@@ -173,35 +188,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            int issued[4] = {0, 0, 0, 0};
             for (int x = 0; x < ntiles; ++x) {
                 mbar_arrive_expect_tx(smem_u32(&bars.q_full[x]), kTileBytes);
                 for (int bx = 0; bx < NB; ++bx)
                     tc::tma_load_4d(q_s + x * kTileBytes + bx * kBox, &tm_q, bx * 64, h,
                                     (qblk * 2 + x) * kBM, b, smem_u32(&bars.q_full[x]));
             }
-            bool ok = true;
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j % STAGES;
-                if (j >= STAGES) ok = wait_bar(&bars, &bars.kv_empty[st], ((j / STAGES) - 1) & 1);
-                if (!ok) break;
+            // K runs two tiles ahead of V: K_{j+2} is requested as soon as
+            // V_j's slot is granted, so every K tile lands an iteration early
+            int nk = 0, nv = 0;  // K / V tiles whose loads were issued
+            auto load_k = [&](int j) -> bool {
+                const int st = j % KST;
+                if (j >= KST && !wait_bar(&bars, &bars.k_empty[st], ((j / KST) - 1) & 1)) return false;
                 mbar_arrive_expect_tx(smem_u32(&bars.k_full[st]), kTileBytes);
                 for (int bx = 0; bx < NB; ++bx)
                     tc::tma_load_4d(k_s + st * kTileBytes + bx * kBox, &tm_k, bx * 64, h, j * kBN, kvb,
                                     smem_u32(&bars.k_full[st]));
+                nk = j + 1;
+                return true;
+            };
+            auto load_v = [&](int j) -> bool {
+                const int st = j % VST;
+                if (j >= VST && !wait_bar(&bars, &bars.v_empty[st], ((j / VST) - 1) & 1)) return false;
                 mbar_arrive_expect_tx(smem_u32(&bars.v_full[st]), kTileBytes);
                 for (int bx = 0; bx < NB; ++bx)
                     tc::tma_load_4d(v_s + st * kTileBytes + bx * kBox, &tm_v, bx * 64, h, j * kBN, kvb,
                                     smem_u32(&bars.v_full[st]));
-                issued[st] += 1;
+                nv = j + 1;
+                return true;
+            };
+            bool ok = true;
+            for (int j = 0; j < 2 && j < nkv && ok; ++j) ok = load_k(j);
+            for (int j = 0; j < nkv && ok; ++j) {
+                ok = load_v(j);
+                if (ok && j + 2 < nkv) ok = load_k(j + 2);
             }
             if (!ok || *(volatile int*)&bars.abort) {
                 // drain: let this CTA's loads land before it exits (bounded)
-                for (int s = 0; s < STAGES; ++s)
-                    if (issued[s] > 0) {
-                        mbar_wait_bounded(smem_u32(&bars.k_full[s]), (issued[s] - 1) & 1, &g_flash_err);
-                        mbar_wait_bounded(smem_u32(&bars.v_full[s]), (issued[s] - 1) & 1, &g_flash_err);
-                    }
+                for (int st = 0; st < KST; ++st) {
+                    const int uses = (nk - st + KST - 1) / KST;  // loads issued into K slot st
+                    if (uses > 0) mbar_wait_bounded(smem_u32(&bars.k_full[st]), (uses - 1) & 1, &g_flash_err);
+                }
+                for (int st = 0; st < VST; ++st) {
+                    const int uses = (nv - st + VST - 1) / VST;
+                    if (uses > 0) mbar_wait_bounded(smem_u32(&bars.v_full[st]), (uses - 1) & 1, &g_flash_err);
+                }
                 for (int x = 0; x < ntiles; ++x)
                     mbar_wait_bounded(smem_u32(&bars.q_full[x]), 0, &g_flash_err);
             }
@@ -211,25 +242,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
+            // Descriptors are built once; a K step or stage only moves the start
+            // address (bits 0..13, in 16-byte units), which stays below 2^14
+            // because shared memory is smaller than 256 KB.
+            const uint64_t dq = tc::smem_desc(q_s, 16, 1024, 2);
+            const uint64_t dk = tc::smem_desc(k_s, 16, 1024, 2);
+            const uint64_t dv = tc::smem_desc(v_s, kBox, 1024, 2);
             auto issue_s = [&](int x, int j) {
-                const int st = j % STAGES;
-                const uint32_t qx = q_s + x * kTileBytes;
+                const uint64_t a0 = dq + (uint64_t)((x * kTileBytes) >> 4);
+                const uint64_t b0 = dk + (uint64_t)(((j % KST) * kTileBytes) >> 4);
+                const uint32_t d = tmem + x * 128;
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
-                    const uint32_t off = (ks >> 2) * kBox + (ks & 3) * 32;
-                    const uint64_t adesc = tc::smem_desc(qx + off, 16, 1024, 2);
-                    const uint64_t bdesc = tc::smem_desc(k_s + st * kTileBytes + off, 16, 1024, 2);
-                    tc::mma_ss(tmem + x * 128, adesc, bdesc, idesc_s, ks > 0 ? 1u : 0u);
+                    constexpr uint32_t kBox16 = kBox >> 4;
+                    const uint32_t off = (ks >> 2) * kBox16 + (ks & 3) * 2;
+                    tc::mma_ss(d, a0 + off, b0 + off, idesc_s, ks > 0 ? 1u : 0u);
                 }
                 tc::commit(smem_u32(&bars.s_full[x]));
             };
             auto issue_pv = [&](int x, int j) {
-                const int st = j % STAGES;
+                const uint64_t b0 = dv + (uint64_t)(((j % VST) * kTileBytes) >> 4);
+                const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128;
+                if (j > 0) {
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk) {
-                    const uint64_t bdesc = tc::smem_desc(v_s + st * kTileBytes + kk * 2048, kBox, 1024, 2);
-                    tc::mma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8, bdesc, idesc_o,
-                               (j > 0 || kk > 0) ? 1u : 0u);
+                    for (int kk = 0; kk < kBN / 16; ++kk) tc::mma_ts(d, pa + kk * 8, b0 + kk * 128, idesc_o, 1u);
+                } else {
+#pragma unroll
+                    for (int kk = 0; kk < kBN / 16; ++kk)
+                        tc::mma_ts(d, pa + kk * 8, b0 + kk * 128, idesc_o, kk > 0 ? 1u : 0u);
                 }
             };
             bool ok = true;
@@ -238,23 +278,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (ok && nkv > 0) {
                 tc::fence_after_sync();
                 for (int x = 0; x < ntiles; ++x) issue_s(x, 0);
+                tc::commit(smem_u32(&bars.k_empty[0]));
             }
             for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j % STAGES;
                 const bool more = j + 1 < nkv;
-                ok = wait_bar(&bars, &bars.v_full[st], (j / STAGES) & 1);
-                if (ok && more) ok = wait_bar(&bars, &bars.k_full[(j + 1) % STAGES], ((j + 1) / STAGES) & 1);
+                ok = wait_bar(&bars, &bars.v_full[j % VST], (j / VST) & 1);
                 for (int x = 0; x < ntiles && ok; ++x) {
                     ok = wait_bar(&bars, &bars.p_full[x], j & 1);
                     if (!ok) break;
                     tc::fence_after_sync();
                     issue_pv(x, j);
-                    if (more)
-                        issue_s(x, j + 1);
-                    else
+                    if (!more) {
                         tc::commit(smem_u32(&bars.o_done[x]));
+                        continue;
+                    }
+                    // K_{j+1} is needed only now, after PV_X(j) is queued
+                    if (x == 0) ok = wait_bar(&bars, &bars.k_full[(j + 1) % KST], ((j + 1) / KST) & 1);
+                    if (!ok) break;
+                    tc::fence_after_sync();
+                    issue_s(x, j + 1);
                 }
-                if (ok) tc::commit(smem_u32(&bars.kv_empty[st]));
+                if (!ok) break;
+                if (more) tc::commit(smem_u32(&bars.k_empty[(j + 1) % KST]));
+                tc::commit(smem_u32(&bars.v_empty[j % VST]));
             }
             // all MMAs this thread issued complete before TMEM is released
             tc::commit(smem_u32(&bars.mma_done));
@@ -272,8 +318,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = wait_bar(&bars, &bars.s_full[x], j & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            float s[kBN];
+            const int valid = a.Lk - j * kBN;  // keys of this tile that exist
+            // ---- pass 1: row max of the raw scores (scale > 0 commutes with
+            // max), eight independent 3-input max chains over 16 scores each
+            float mt;
             {
+                float s[kBN];
                 uint32_t r0[32], r1[32], r2[32], r3[32];
                 tc::ld_32col(lane_addr + s_col + 0, r0);
                 tc::ld_32col(lane_addr + s_col + 32, r1);
@@ -287,23 +337,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                     s[64 + i] = __uint_as_float(r2[i]);
                     s[96 + i] = __uint_as_float(r3[i]);
                 }
+                if (valid < kBN) {
+#pragma unroll
+                    for (int i = 0; i < kBN; ++i)
+                        if (i >= valid) s[i] = -INFINITY;
+                }
+                float mx[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    float m = tc::max3f(s[k], s[k + 8], s[k + 16]);
+#pragma unroll
+                    for (int i = k + 24; i < kBN; i += 16) m = tc::max3f(m, s[i], s[i + 8]);
+                    mx[k] = m;
+                }
+                mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
+                               fmaxf(mx[6], mx[7])) * a.scale_log2;
             }
-            const int valid = a.Lk - j * kBN;  // keys of this tile that exist
-            if (valid < kBN) {
-#pragma unroll
-                for (int i = 0; i < kBN; ++i)
-                    if (i >= valid) s[i] = -INFINITY;
-            }
-            // row max of the raw scores (scale > 0 commutes with max): 8-way tree
-            float mx[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) mx[k] = s[k];
-#pragma unroll
-            for (int i = 8; i < kBN; i += 8)
-#pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = fmaxf(mx[k], s[i + k]);
-            const float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                                   fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * a.scale_log2;
             if (j == 0) {
                 m_ref = mt;
             } else {
@@ -325,28 +374,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_ref = m_new;
                 }
             }
-            const float neg_m = -m_ref;
-            float acc[8];
+            // ---- pass 2: S is read again 32 columns at a time (the next chunk's
+            // load overlaps this chunk's math), exponentiated, summed and
+            // written back as bf16 P over the columns already consumed
+            const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
+            const tc::f32x2 negm2 = tc::pack2(-m_ref, -m_ref);
+            tc::f32x2 acc[4];
 #pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = 0.f;
+            for (int k = 0; k < 4; ++k) acc[k] = tc::pack2(0.f, 0.f);
+            uint32_t buf[2][32];
+            tc::ld_32col(lane_addr + s_col, buf[0]);
+            tc::wait_ld();
 #pragma unroll
             for (int c = 0; c < kBN / 32; ++c) {
+                if (c + 1 < kBN / 32) tc::ld_32col(lane_addr + s_col + (c + 1) * 32, buf[(c + 1) & 1]);
                 uint32_t r[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    float p[2];
-#pragma unroll
-                    for (int e = 0; e < 2; ++e) {
-                        const int idx = c * 32 + 2 * i + e;
-                        const float t = fmaf(s[idx], a.scale_log2, neg_m);
-                        p[e] = ((idx & 7) < kPolyOf8) ? exp2_poly(t) : ex2(t);
-                        acc[idx & 7] += p[e];
+                    const int idx = c * 32 + 2 * i;
+                    float s0 = __uint_as_float(buf[c & 1][2 * i]);
+                    float s1 = __uint_as_float(buf[c & 1][2 * i + 1]);
+                    if (valid < kBN) {
+                        if (idx >= valid) s0 = -INFINITY;
+                        if (idx + 1 >= valid) s1 = -INFINITY;
                     }
-                    r[i] = pack_bf16x2(p[0], p[1]);
+                    const tc::f32x2 t = tc::fma2(tc::pack2(s0, s1), scale2, negm2);
+                    float t0, t1, p0, p1;
+                    tc::unpack2(t, t0, t1);
+                    if (((idx >> 1) & 7) < kPolyPairsOf8) {
+                        exp2_poly2(t0, t1, p0, p1);
+                    } else {
+                        p0 = ex2(t0);
+                        p1 = ex2(t1);
+                    }
+                    acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
+                    r[i] = pack_bf16x2(p0, p1);
                 }
+                // P chunk c lands on columns [16c, 16c+16) of S, which chunks
+                // <= c have already delivered; the load in flight reads
+                // columns >= 32(c+1)
                 tc::st_16col(lane_addr + s_col + c * 16, r);
+                if (c + 1 < kBN / 32) tc::wait_ld();
             }
-            l += ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+            {
+                float a0, a1;
+                tc::unpack2(tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3])), a0, a1);
+                l += a0 + a1;
+            }
             tc::wait_st();
             tc::fence_before_sync();
             mbar_arrive(smem_u32(&bars.p_full[x]));
@@ -431,13 +505,14 @@ template <int KSTEPS>
 cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
-    constexpr int STAGES = NB == 1 ? 3 : 2;
-    const size_t smem = (size_t)(2 + 2 * STAGES) * NB * kBox + 1024;
+    constexpr int KST = NB == 1 ? 4 : 3;  // K ring (two tiles of look-ahead + the one in use)
+    constexpr int VST = NB == 1 ? 3 : 2;  // V ring
+    const size_t smem = (size_t)(2 + KST + VST) * NB * kBox + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, STAGES>,
+    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, KST, VST>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
     if (e != cudaSuccess) return e;
-    flash_tc_kernel<KSTEPS, STAGES><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    flash_tc_kernel<KSTEPS, KST, VST><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
 

@@ -139,11 +139,10 @@ cudaError_t launch_layout(int to_temporal, const void* src, void* dst, int T, in
     p.units = (p.rows + R - 1) / R;
     if (p.rows == 0) return cudaSuccess;
     const size_t smem = (size_t)kStages * R * row_bytes;
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(layout_bulk_kernel,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    // the kernel's static shared memory (barriers) comes on top of `smem`
+    cudaError_t e = cudaFuncSetAttribute(layout_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
     const int per_sm = (int)((200 * 1024) / (smem + 1024));
     long long grid = (long long)device_sm_count() * (per_sm < 1 ? 1 : per_sm);
     if (grid > p.units) grid = p.units;

@@ -96,23 +96,24 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
         const int h0 = (int)(unit - (long long)n * hg_count) * G;
         const uint32_t bar = smem_u32(&full_bar[stage]);
         mbar_arrive_expect_tx(bar, unit_bytes);
-        const CUtensorMap* maps[3] = {&tm_q, &tm_k, &tm_v};
-        for (int tsr = 0; tsr < 3; ++tsr)
-            for (int g = 0; g < G; ++g)
-                tc::tma_load_4d(sbase_u32 + 2u * (stage * stage_elems + tsr * tensor_elems + g * head_elems),
-                                maps[tsr], 0, h0 + g, 0, n, bar);
+        for (int g = 0; g < G; ++g) {
+            const uint32_t dst = sbase_u32 + 2u * (stage * stage_elems + g * head_elems);
+            tc::tma_load_4d(dst, &tm_q, 0, h0 + g, 0, n, bar);
+            tc::tma_load_4d(dst + 2u * tensor_elems, &tm_k, 0, h0 + g, 0, n, bar);
+            tc::tma_load_4d(dst + 4u * tensor_elems, &tm_v, 0, h0 + g, 0, n, bar);
+        }
     };
 
     const long long first = blockIdx.x, step = gridDim.x;
-    int issued[2] = {0, 0};
+    // units issued / waited for so far; unit k of this CTA uses stage k & 1
+    long long n_issued = 0, n_waited = 0;
     if (tid == 0 && first < p.units) {
         issue_unit(first, 0);
-        issued[0] = 1;
+        n_issued = 1;
     }
 
     const int mtiles = RT / 16;
     const int tasks = G * mtiles;
-    int waited[2] = {0, 0};
     for (long long i = 0;; ++i) {
         const long long u = first + i * step;
         if (u >= p.units) break;
@@ -123,12 +124,13 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
                 // the other stage held unit i-1: its output store must have read it
                 bulk_wait_read<0>();
                 issue_unit(nu, stage ^ 1);
-                issued[stage ^ 1] += 1;
+                n_issued = i + 2;
             }
         }
-        if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), (uint32_t)(waited[stage] & 1), &g_temporal_err))
+        // unit i is the (i >> 1)-th use of its stage
+        if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), (uint32_t)((i >> 1) & 1), &g_temporal_err))
             abort_flag = 1;
-        waited[stage] += 1;
+        n_waited = i + 1;
         __syncthreads();
         if (abort_flag) break;
 
@@ -247,10 +249,10 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
     }
     if (tid == 0) {
         if (abort_flag) {
-            // let every load this CTA issued land before it exits (bounded)
-            for (int s = 0; s < 2; ++s)
-                if (issued[s] > waited[s])
-                    mbar_wait_bounded(smem_u32(&full_bar[s]), (uint32_t)((issued[s] - 1) & 1), &g_temporal_err);
+            // let every load this CTA issued land before it exits (bounded):
+            // units n_waited-1 (timed out) .. n_issued-1 may still be in flight
+            for (long long k = (n_waited > 0 ? n_waited - 1 : 0); k < n_issued; ++k)
+                mbar_wait_bounded(smem_u32(&full_bar[k & 1]), (uint32_t)((k >> 1) & 1), &g_temporal_err);
         }
         bulk_wait<0>();
     }

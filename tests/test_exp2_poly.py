@@ -1,4 +1,4 @@
-"""The flash kernel's software exp2 (exp2_poly in flash_tc.cu), emulated bit
+"""The flash kernel's software exp2 (exp2_poly2 in flash_tc.cu), emulated bit
 for bit in numpy float32 with the coefficients read from the kernel source,
 against numpy's exp2 in float64 over the whole input range the softmax
 produces (x <= 8; x < -120 clamped).  The kernel moves part of the softmax
@@ -15,12 +15,8 @@ SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
 
 def kernel_coefficients():
     text = open(SRC).read()
-    body = text[text.index("PAB_DEV float exp2_poly"):]
-    body = body[:body.index("\n}\n")]
-    c3, c2 = re.search(r"fmaf\(([-0-9.e]+)f, f, ([-0-9.e]+)f\)", body).groups()
-    c1 = re.search(r"fmaf\(p, f, ([-0-9.e]+)f\);\s*p = fmaf\(p, f", body).group(1)
-    c0 = re.findall(r"fmaf\(p, f, ([-0-9.e]+)f\)", body)[-1]
-    return [np.float32(c) for c in (c0, c1, c2, c3)]
+    vals = dict(re.findall(r"\b(kP[0-3]) = ([-0-9.e]+)f", text))
+    return [np.float32(vals[f"kP{i}"]) for i in range(4)]
 
 
 def exp2_poly_emulated(x):
