@@ -6,15 +6,17 @@
 //
 // A CTA owns 256 query rows of one (batch, head) as two 128-row tiles A and B
 // that share every K/V tile, and runs four roles:
-//   warp 8 (one thread)   TMA producer: Q_A, Q_B once, then K_j / V_j tiles of
-//                          128 keys into separate shared-memory rings, K two
-//                          tiles ahead of V (K is consumed one step earlier);
-//   warp 9 (one thread)   MMA issuer: S_X = Q_X K_j^T (SS form, fp32 in TMEM)
-//                          and O_X += P_X V_j (TS form: P from TMEM, V from
-//                          shared memory), ping-ponging between the tiles:
-//                          PV_A(j), S_A(j+1), PV_B(j), S_B(j+1), ... so the
-//                          tensor cores work on one tile while the other
-//                          tile's softmax runs; warp 9 also owns TMEM;
+//   warp 8 (one thread)   TMA producer: Q_A, Q_B, K_0, K_1 once, then per
+//                          step j one ring slot with V_j and K_{j+2} (tiles of
+//                          64 keys; K is consumed two steps before V);
+//   warps 9, 10 (one thread each)  MMA issuers, one per query tile X:
+//                          S_X(j) = Q_X K_j^T (SS form, fp32 in TMEM) and
+//                          O_X += P_X(j) V_j (TS form: P from TMEM, V from
+//                          shared memory).  S is double-buffered per tile, so
+//                          S_X(j+2) is issued right behind PV_X(j) and is
+//                          ready before the softmax needs it: the softmax
+//                          never waits for a round trip through the tensor
+//                          cores.  Warp 9 also owns TMEM;
 //   warps 0-3 / 4-7       softmax of tile A / B: thread i owns query row i =
 //                          TMEM lane i.  It reads its row of S with tcgen05.ld,
 //                          keeps the running max and sum in registers (tree
@@ -25,16 +27,18 @@
 //                          unit, 3/8 on the FMA pipes (exp2_poly2).
 //                          At the end it normalises O and writes it through
 //                          shared memory with a TMA tensor store.
-// When S_X(j) completes, every earlier MMA of the issuing thread -- PV_X(j-1)
-// in particular -- has completed too, so the softmax may rescale O_X then.
+// Rescaling O_X at step j needs PV_X(j-1) retired: the softmax then waits for
+// step j-1's slot to be done.
 //
-// TMEM columns: S_A [0,128), S_B [128,256), O_A [256,256+NO), O_B [384,384+NO).
+// TMEM columns: S_A0 [0,64), S_A1 [64,128), S_B0 [128,192), S_B1 [192,256),
+//               O_A [256,256+NO), O_B [384,384+NO).
 // Operand layouts (128-byte swizzle, TMA-written):
-//   Q, K: [128 rows][64 cols] boxes, K-major (d contiguous); a 16-wide K step
-//         advances the descriptor start by 32 bytes inside the box.
-//   V:    the same boxes read MN-major (B of the PV product has N = d
-//         contiguous); a 16-key K step advances by 16 rows = 2048 bytes, the
-//         next 64 columns of d are one box (16 KB) further (LBO).
+//   Q, K: [rows][64 cols] boxes (128 rows for Q, 64 for K), K-major (d
+//         contiguous); a 16-wide K step advances the descriptor start by 32
+//         bytes inside the box.
+//   V:    [64 rows][64 cols] boxes read MN-major (B of the PV product has
+//         N = d contiguous); a 16-key K step advances by 16 rows = 2048 bytes,
+//         the next 64 columns of d are one box (8 KB) further (LBO).
 // Head dims that are not a multiple of 64 read zero-filled columns past d
 // (the tensor map's innermost extent is d); keys past Lk are masked to -inf;
 // query rows past Lq are zero-filled on load and clipped by the TMA store; a
@@ -50,9 +54,10 @@ namespace pab {
 namespace {
 
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
-constexpr int kBN = 128;          // keys per K/V tile
-constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
-constexpr int kThreads = 320;     // 2 softmax warpgroups + producer warp + MMA warp
+constexpr int kBN = 64;           // keys per K/V tile
+constexpr int kQBox = 128 * 128;  // bytes of one [128 rows][64 cols] bf16 box (Q, O)
+constexpr int kKVBox = 64 * 128;  // bytes of one [64 rows][64 cols] bf16 box (K, V)
+constexpr int kThreads = 352;     // 2 softmax warpgroups + producer warp + 2 MMA warps
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 // Exponentials: of every 8 consecutive pairs of a row's scores, this many go
@@ -74,16 +79,23 @@ struct FlashTcArgs {
     float scale_log2;  // log2(e) / sqrt(d)
 };
 
+constexpr int kMaxStages = 8;
+
+// A tcgen05.commit costs the tensor pipe about as much as two small MMAs, so
+// the pipeline is built around ONE commit per tile and K/V step: slot s of the
+// ring holds V_j and K_{j+2} (j = s mod NST); after issuing PV_X(j) and
+// S_X(j+2) each tile's issuer commits slot_done[s] once.  Its completion frees
+// the slot for the producer, tells the softmax that S_X(j+2) is in TMEM and
+// proves PV_X(j) retired (in-order completion).
 struct Bars {
     unsigned long long q_full[2];
-    unsigned long long k_full[4];
-    unsigned long long v_full[4];
-    unsigned long long k_empty[4];
-    unsigned long long v_empty[4];
-    unsigned long long s_full[2];
-    unsigned long long p_full[2];
-    unsigned long long o_done[2];
-    unsigned long long mma_done;
+    unsigned long long k01_full;               // K_0, K_1 (own buffer)
+    unsigned long long s01_done;               // S_X(0), S_X(1) of every tile retired
+    unsigned long long slot_full[kMaxStages];  // V_j (+ K_{j+2}) landed
+    unsigned long long slot_done[kMaxStages];  // one arrival per tile issuer
+    unsigned long long p_full[2][2];           // [tile][S buffer]
+    unsigned long long o_done[2];              // the last PV_X retired
+    unsigned long long mma_done[2];
     uint32_t tmem_base;
     int abort;
 };
@@ -129,21 +141,23 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
     return true;
 }
 
-template <int KSTEPS, int KST, int VST>
+template <int KSTEPS, int NST>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     FlashTcArgs a) {
     constexpr int NB = (KSTEPS + 3) / 4;  // 64-column boxes covering d
     constexpr int NO = KSTEPS * 16;       // N of the PV product (d rounded up to 16)
-    constexpr uint32_t kTileBytes = NB * kBox;
+    constexpr uint32_t kQTile = NB * kQBox;
+    constexpr uint32_t kKVTile = NB * kKVBox;
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ Bars bars;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t q_s = sbase;                   // [2 tiles][NB boxes]
-    const uint32_t k_s = q_s + 2 * kTileBytes;    // [KST][NB boxes]
-    const uint32_t v_s = k_s + KST * kTileBytes;  // [VST][NB boxes]
+    const uint32_t q_s = sbase;                  // [2 tiles][NB boxes]
+    const uint32_t k01_s = q_s + 2 * kQTile;     // [2][NB boxes]: K_0, K_1
+    const uint32_t v_s = k01_s + 2 * kKVTile;    // [NST][NB boxes]: V_j
+    const uint32_t k_s = v_s + NST * kKVTile;    // [NST][NB boxes]: K_{j+2}
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -155,19 +169,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 256) {
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&bars.q_full[x]), 1);
-            mbar_init(smem_u32(&bars.s_full[x]), 1);
-            mbar_init(smem_u32(&bars.p_full[x]), 128);
+            for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&bars.p_full[x][u]), 128);
             mbar_init(smem_u32(&bars.o_done[x]), 1);
+            mbar_init(smem_u32(&bars.mma_done[x]), 1);
         }
-        for (int s = 0; s < KST; ++s) {
-            mbar_init(smem_u32(&bars.k_full[s]), 1);
-            mbar_init(smem_u32(&bars.k_empty[s]), 1);
+        mbar_init(smem_u32(&bars.k01_full), 1);
+        mbar_init(smem_u32(&bars.s01_done), ntiles);
+        for (int st = 0; st < NST; ++st) {
+            mbar_init(smem_u32(&bars.slot_full[st]), 1);
+            mbar_init(smem_u32(&bars.slot_done[st]), ntiles);
         }
-        for (int s = 0; s < VST; ++s) {
-            mbar_init(smem_u32(&bars.v_full[s]), 1);
-            mbar_init(smem_u32(&bars.v_empty[s]), 1);
-        }
-        mbar_init(smem_u32(&bars.mma_done), 1);
         bars.abort = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&tm_q);
@@ -189,153 +200,132 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             for (int x = 0; x < ntiles; ++x) {
-                mbar_arrive_expect_tx(smem_u32(&bars.q_full[x]), kTileBytes);
+                mbar_arrive_expect_tx(smem_u32(&bars.q_full[x]), kQTile);
                 for (int bx = 0; bx < NB; ++bx)
-                    tc::tma_load_4d(q_s + x * kTileBytes + bx * kBox, &tm_q, bx * 64, h,
-                                    (qblk * 2 + x) * kBM, b, smem_u32(&bars.q_full[x]));
+                    tc::tma_load_4d(q_s + x * kQTile + bx * kQBox, &tm_q, bx * 64, h, (qblk * 2 + x) * kBM, b,
+                                    smem_u32(&bars.q_full[x]));
             }
-            // K runs two tiles ahead of V: K_{j+2} is requested as soon as
-            // V_j's slot is granted, so every K tile lands an iteration early
-            int nk = 0, nv = 0;  // K / V tiles whose loads were issued
-            auto load_k = [&](int j) -> bool {
-                const int st = j % KST;
-                if (j >= KST && !wait_bar(&bars, &bars.k_empty[st], ((j / KST) - 1) & 1)) return false;
-                mbar_arrive_expect_tx(smem_u32(&bars.k_full[st]), kTileBytes);
-                for (int bx = 0; bx < NB; ++bx)
-                    tc::tma_load_4d(k_s + st * kTileBytes + bx * kBox, &tm_k, bx * 64, h, j * kBN, kvb,
-                                    smem_u32(&bars.k_full[st]));
-                nk = j + 1;
-                return true;
-            };
-            auto load_v = [&](int j) -> bool {
-                const int st = j % VST;
-                if (j >= VST && !wait_bar(&bars, &bars.v_empty[st], ((j / VST) - 1) & 1)) return false;
-                mbar_arrive_expect_tx(smem_u32(&bars.v_full[st]), kTileBytes);
-                for (int bx = 0; bx < NB; ++bx)
-                    tc::tma_load_4d(v_s + st * kTileBytes + bx * kBox, &tm_v, bx * 64, h, j * kBN, kvb,
-                                    smem_u32(&bars.v_full[st]));
-                nv = j + 1;
-                return true;
-            };
+            const int n01 = nkv < 2 ? nkv : 2;
+            if (n01 > 0) {
+                mbar_arrive_expect_tx(smem_u32(&bars.k01_full), n01 * kKVTile);
+                for (int j = 0; j < n01; ++j)
+                    for (int bx = 0; bx < NB; ++bx)
+                        tc::tma_load_4d(k01_s + j * kKVTile + bx * kKVBox, &tm_k, bx * 64, h, j * kBN, kvb,
+                                        smem_u32(&bars.k01_full));
+            }
+            int nslot = 0;  // slot loads issued
             bool ok = true;
-            for (int j = 0; j < 2 && j < nkv && ok; ++j) ok = load_k(j);
             for (int j = 0; j < nkv && ok; ++j) {
-                ok = load_v(j);
-                if (ok && j + 2 < nkv) ok = load_k(j + 2);
+                const int st = j % NST;
+                if (j >= NST) ok = wait_bar(&bars, &bars.slot_done[st], ((j / NST) - 1) & 1);
+                if (!ok) break;
+                const bool with_k = j + 2 < nkv;
+                const uint32_t bar = smem_u32(&bars.slot_full[st]);
+                mbar_arrive_expect_tx(bar, with_k ? 2 * kKVTile : kKVTile);
+                for (int bx = 0; bx < NB; ++bx)
+                    tc::tma_load_4d(v_s + st * kKVTile + bx * kKVBox, &tm_v, bx * 64, h, j * kBN, kvb, bar);
+                if (with_k)
+                    for (int bx = 0; bx < NB; ++bx)
+                        tc::tma_load_4d(k_s + st * kKVTile + bx * kKVBox, &tm_k, bx * 64, h, (j + 2) * kBN, kvb,
+                                        bar);
+                nslot = j + 1;
             }
             if (!ok || *(volatile int*)&bars.abort) {
                 // drain: let this CTA's loads land before it exits (bounded)
-                for (int st = 0; st < KST; ++st) {
-                    const int uses = (nk - st + KST - 1) / KST;  // loads issued into K slot st
-                    if (uses > 0) mbar_wait_bounded(smem_u32(&bars.k_full[st]), (uses - 1) & 1, &g_flash_err);
+                for (int st = 0; st < NST; ++st) {
+                    const int uses = (nslot - st + NST - 1) / NST;  // loads issued into slot st
+                    if (uses > 0)
+                        mbar_wait_bounded(smem_u32(&bars.slot_full[st]), (uses - 1) & 1, &g_flash_err);
                 }
-                for (int st = 0; st < VST; ++st) {
-                    const int uses = (nv - st + VST - 1) / VST;
-                    if (uses > 0) mbar_wait_bounded(smem_u32(&bars.v_full[st]), (uses - 1) & 1, &g_flash_err);
-                }
+                if (n01 > 0) mbar_wait_bounded(smem_u32(&bars.k01_full), 0, &g_flash_err);
                 for (int x = 0; x < ntiles; ++x)
                     mbar_wait_bounded(smem_u32(&bars.q_full[x]), 0, &g_flash_err);
             }
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------ MMA issuer
-        if (lane == 0) {
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------ MMA issuers
+        // One thread per query tile: a wait of one issuer overlaps the other's
+        // MMA issue, so the tensor core queue stays fed.
+        const int x = warp - 9;
+        if (lane == 0 && x < ntiles) {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
-            // Descriptors are built once; a K step or stage only moves the start
-            // address (bits 0..13, in 16-byte units), which stays below 2^14
-            // because shared memory is smaller than 256 KB.
-            const uint64_t dq = tc::smem_desc(q_s, 16, 1024, 2);
+            // Descriptors are built once; a K step, tile or slot only moves the
+            // start address (bits 0..13, in 16-byte units), which stays below
+            // 2^14 because shared memory is smaller than 256 KB.
+            const uint64_t dq = tc::smem_desc(q_s + x * kQTile, 16, 1024, 2);
+            const uint64_t dk01 = tc::smem_desc(k01_s, 16, 1024, 2);
             const uint64_t dk = tc::smem_desc(k_s, 16, 1024, 2);
-            const uint64_t dv = tc::smem_desc(v_s, kBox, 1024, 2);
-            auto issue_s = [&](int x, int j) {
-                const uint64_t a0 = dq + (uint64_t)((x * kTileBytes) >> 4);
-                const uint64_t b0 = dk + (uint64_t)(((j % KST) * kTileBytes) >> 4);
-                const uint32_t d = tmem + x * 128;
+            const uint64_t dv = tc::smem_desc(v_s, kKVBox, 1024, 2);
+            auto issue_s = [&](uint64_t kdesc, int j) {  // S_X(j) into buffer j & 1
+                const uint32_t d = tmem + x * 128 + (j & 1) * 64;
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
-                    constexpr uint32_t kBox16 = kBox >> 4;
-                    const uint32_t off = (ks >> 2) * kBox16 + (ks & 3) * 2;
-                    tc::mma_ss(d, a0 + off, b0 + off, idesc_s, ks > 0 ? 1u : 0u);
-                }
-                tc::commit(smem_u32(&bars.s_full[x]));
-            };
-            auto issue_pv = [&](int x, int j) {
-                const uint64_t b0 = dv + (uint64_t)(((j % VST) * kTileBytes) >> 4);
-                const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128;
-                if (j > 0) {
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk) tc::mma_ts(d, pa + kk * 8, b0 + kk * 128, idesc_o, 1u);
-                } else {
-#pragma unroll
-                    for (int kk = 0; kk < kBN / 16; ++kk)
-                        tc::mma_ts(d, pa + kk * 8, b0 + kk * 128, idesc_o, kk > 0 ? 1u : 0u);
+                    const uint32_t offa = (ks >> 2) * (kQBox >> 4) + (ks & 3) * 2;
+                    const uint32_t offb = (ks >> 2) * (kKVBox >> 4) + (ks & 3) * 2;
+                    tc::mma_ss(d, dq + offa, kdesc + offb, idesc_s, ks > 0 ? 1u : 0u);
                 }
             };
-            bool ok = true;
-            for (int x = 0; x < ntiles && ok; ++x) ok = wait_bar(&bars, &bars.q_full[x], 0);
-            if (ok && nkv > 0) ok = wait_bar(&bars, &bars.k_full[0], 0);
+            bool ok = wait_bar(&bars, &bars.q_full[x], 0);
+            if (ok && nkv > 0) ok = wait_bar(&bars, &bars.k01_full, 0);
             if (ok && nkv > 0) {
                 tc::fence_after_sync();
-                for (int x = 0; x < ntiles; ++x) issue_s(x, 0);
-                tc::commit(smem_u32(&bars.k_empty[0]));
+                issue_s(dk01, 0);
+                if (nkv > 1) issue_s(dk01 + (kKVTile >> 4), 1);
+                tc::commit(smem_u32(&bars.s01_done));
             }
             for (int j = 0; j < nkv && ok; ++j) {
-                const bool more = j + 1 < nkv;
-                ok = wait_bar(&bars, &bars.v_full[j % VST], (j / VST) & 1);
-                for (int x = 0; x < ntiles && ok; ++x) {
-                    ok = wait_bar(&bars, &bars.p_full[x], j & 1);
-                    if (!ok) break;
-                    tc::fence_after_sync();
-                    issue_pv(x, j);
-                    if (!more) {
-                        tc::commit(smem_u32(&bars.o_done[x]));
-                        continue;
-                    }
-                    // K_{j+1} is needed only now, after PV_X(j) is queued
-                    if (x == 0) ok = wait_bar(&bars, &bars.k_full[(j + 1) % KST], ((j + 1) / KST) & 1);
-                    if (!ok) break;
-                    tc::fence_after_sync();
-                    issue_s(x, j + 1);
-                }
+                const int st = j % NST;
+                ok = wait_bar(&bars, &bars.slot_full[st], (j / NST) & 1);
+                if (ok) ok = wait_bar(&bars, &bars.p_full[x][j & 1], (j >> 1) & 1);
                 if (!ok) break;
-                if (more) tc::commit(smem_u32(&bars.k_empty[(j + 1) % KST]));
-                tc::commit(smem_u32(&bars.v_empty[j % VST]));
+                tc::fence_after_sync();
+                // O_X += P_X(j) V_j
+                const uint64_t vdesc = dv + (uint64_t)((st * kKVTile) >> 4);
+                const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128 + (j & 1) * 64;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    tc::mma_ts(d, pa + kk * 8, vdesc + kk * 128, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
+                // S_X(j+2) reuses the buffer PV_X(j) has just been queued on
+                if (j + 2 < nkv) issue_s(dk + (uint64_t)((st * kKVTile) >> 4), j + 2);
+                tc::commit(smem_u32(&bars.slot_done[st]));
+                if (j + 1 == nkv) tc::commit(smem_u32(&bars.o_done[x]));
             }
             // all MMAs this thread issued complete before TMEM is released
-            tc::commit(smem_u32(&bars.mma_done));
-            mbar_wait_bounded(smem_u32(&bars.mma_done), 0, &g_flash_err);
+            tc::commit(smem_u32(&bars.mma_done[x]));
+            mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_flash_err);
         }
     } else {
         // ------------------------------------------------ softmax warpgroups
         const int x = warp >> 2;  // tile
         const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t s_col = x * 128, o_col = 256 + x * 128;
+        const uint32_t o_col = 256 + x * 128;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = x < ntiles;
         for (int j = 0; j < nkv && ok; ++j) {
-            ok = wait_bar(&bars, &bars.s_full[x], j & 1);
+            const uint32_t s_col = x * 128 + (j & 1) * 64;
+            // S_X(j) was issued with step j-2's slot (or in the prologue)
+            if (j < 2)
+                ok = wait_bar(&bars, &bars.s01_done, 0);
+            else
+                ok = wait_bar(&bars, &bars.slot_done[(j - 2) % NST], ((j - 2) / NST) & 1);
             if (!ok) break;
             tc::fence_after_sync();
             const int valid = a.Lk - j * kBN;  // keys of this tile that exist
             // ---- pass 1: row max of the raw scores (scale > 0 commutes with
-            // max), eight independent 3-input max chains over 16 scores each
+            // max), eight independent 3-input max chains over 8 scores each
             float mt;
             {
                 float s[kBN];
-                uint32_t r0[32], r1[32], r2[32], r3[32];
+                uint32_t r0[32], r1[32];
                 tc::ld_32col(lane_addr + s_col + 0, r0);
                 tc::ld_32col(lane_addr + s_col + 32, r1);
-                tc::ld_32col(lane_addr + s_col + 64, r2);
-                tc::ld_32col(lane_addr + s_col + 96, r3);
                 tc::wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     s[i] = __uint_as_float(r0[i]);
                     s[32 + i] = __uint_as_float(r1[i]);
-                    s[64 + i] = __uint_as_float(r2[i]);
-                    s[96 + i] = __uint_as_float(r3[i]);
                 }
                 if (valid < kBN) {
 #pragma unroll
@@ -346,9 +336,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
                     float m = tc::max3f(s[k], s[k + 8], s[k + 16]);
-#pragma unroll
-                    for (int i = k + 24; i < kBN; i += 16) m = tc::max3f(m, s[i], s[i + 8]);
-                    mx[k] = m;
+                    m = tc::max3f(m, s[k + 24], s[k + 32]);
+                    m = tc::max3f(m, s[k + 40], s[k + 48]);
+                    mx[k] = fmaxf(m, s[k + 56]);
                 }
                 mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
                                fmaxf(mx[6], mx[7])) * a.scale_log2;
@@ -358,7 +348,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else {
                 const bool need = mt > m_ref + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
-                    // PV_X(j-1) completed before S_X(j) did: O_X is stable here
+                    // O_X must hold exactly PV_X(0..j-1): PV_X(j-1) retired
+                    // once step j-1's slot is done
+                    ok = wait_bar(&bars, &bars.slot_done[(j - 1) % NST], ((j - 1) / NST) & 1);
+                    if (!ok) break;
+                    tc::fence_after_sync();
                     const float m_new = need ? mt : m_ref;
                     const float f = ex2(m_ref - m_new);
 #pragma unroll
@@ -423,14 +417,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc::wait_st();
             tc::fence_before_sync();
-            mbar_arrive(smem_u32(&bars.p_full[x]));
+            mbar_arrive(smem_u32(&bars.p_full[x][j & 1]));
         }
         // ---------------- epilogue: O / l -> bf16 -> swizzled smem -> TMA store
         if (ok && nkv > 0) ok = wait_bar(&bars, &bars.o_done[x], 0);
         if (ok) {
             tc::fence_after_sync();
             const float inv = 1.f / l;
-            unsigned char* stage = gen_base + x * kTileBytes;  // this tile's Q buffer (all S MMAs done)
+            unsigned char* stage = gen_base + x * kQTile;  // this tile's Q buffer (all S MMAs done)
 #pragma unroll
             for (int c = 0; c < NO / 16; ++c) {
                 uint32_t r[16];
@@ -443,7 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int col = c * 16;
                 const int bx = col >> 6;
                 const int ch = (col & 63) >> 3;
-                unsigned char* rowp = stage + bx * kBox + row * 128;
+                unsigned char* rowp = stage + bx * kQBox + row * 128;
                 *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
                 *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
                     make_uint4(w[4], w[5], w[6], w[7]);
@@ -453,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::named_bar_sync(1 + x, 128);
         if (ok && row == 0) {
             for (int bx = 0; bx < NB; ++bx)
-                tc::tma_store_4d(&tm_o, q_s + x * kTileBytes + bx * kBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
+                tc::tma_store_4d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
             bulk_commit();
             bulk_wait<0>();
         }
@@ -485,15 +479,15 @@ EncodeTiledFn encode_fn() {
 }
 
 // 4-D map over a [batches][rows][heads][d] bf16 view (row stride C elements):
-// dims (d, heads, rows, batches), box (64, 1, 128, 1), 128-byte swizzle.
+// dims (d, heads, rows, batches), box (64, 1, box_rows, 1), 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows, long long batches,
-              long long row_stride_elems, long long batch_stride_elems) {
+              long long row_stride_elems, long long batch_stride_elems, int box_rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows, (cuuint64_t)batches};
     cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)row_stride_elems * 2,
                              (cuuint64_t)(batch_stride_elems > 0 ? batch_stride_elems : rows * row_stride_elems) * 2};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -505,14 +499,13 @@ template <int KSTEPS>
 cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
-    constexpr int KST = NB == 1 ? 4 : 3;  // K ring (two tiles of look-ahead + the one in use)
-    constexpr int VST = NB == 1 ? 3 : 2;  // V ring
-    const size_t smem = (size_t)(2 + KST + VST) * NB * kBox + 1024;
+    constexpr int NST = NB == 1 ? 6 : 4;  // ring slots of (V_j, K_{j+2})
+    const size_t smem = (size_t)NB * (2 * kQBox + (2 + 2 * NST) * kKVBox) + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, KST, VST>,
+    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
     if (e != cudaSuccess) return e;
-    flash_tc_kernel<KSTEPS, KST, VST><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    flash_tc_kernel<KSTEPS, NST><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
 
@@ -527,10 +520,10 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
         return cudaErrorInvalidValue;
     CUtensorMap mq, mk, mv, mo;
     const long long kv_batches = kv_bstride > 0 ? batches : 1;
-    if (!make_map(&mq, q, d, heads, Lq, batches, C, q_bstride) ||
-        !make_map(&mk, k, d, heads, Lk, kv_batches, C, kv_bstride) ||
-        !make_map(&mv, v, d, heads, Lk, kv_batches, C, kv_bstride) ||
-        !make_map(&mo, out, d, heads, Lq, batches, C, q_bstride))
+    if (!make_map(&mq, q, d, heads, Lq, batches, C, q_bstride, kBM) ||
+        !make_map(&mk, k, d, heads, Lk, kv_batches, C, kv_bstride, kBN) ||
+        !make_map(&mv, v, d, heads, Lk, kv_batches, C, kv_bstride, kBN) ||
+        !make_map(&mo, out, d, heads, Lq, batches, C, q_bstride, kBM))
         return cudaErrorInvalidValue;
     FlashTcArgs a;
     a.Lq = (int)Lq;
