@@ -97,9 +97,21 @@ PAB_DEV bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
     return ok != 0;
 }
+// Non-blocking test of the phase with the given parity.
+PAB_DEV bool mbar_test_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n .reg .pred p;\n"
+        " mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}"
+        : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    return ok != 0;
+}
 // Wait for the phase with the given parity to complete, giving up after
-// kWaitLimitNs.  Returns false (and sets `err_word` bits) on time-out.
+// kWaitLimitNs.  Returns false (and sets `err_word` bits) on time-out.  A
+// phase that has already completed is detected by a non-blocking test.
 PAB_DEV bool mbar_wait_bounded(uint32_t bar, uint32_t parity, unsigned int* err_word) {
+    if (mbar_test_wait(bar, parity)) return true;
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer_ns();
     for (;;) {

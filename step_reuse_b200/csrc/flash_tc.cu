@@ -313,32 +313,35 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!ok) break;
             tc::fence_after_sync();
             const int valid = a.Lk - j * kBN;  // keys of this tile that exist
-            // ---- pass 1: row max of the raw scores (scale > 0 commutes with
-            // max), eight independent 3-input max chains over 8 scores each
-            float mt;
+            // the row's 64 scores fit in registers: one TMEM read
+            float sv[kBN];
             {
-                float s[kBN];
                 uint32_t r0[32], r1[32];
                 tc::ld_32col(lane_addr + s_col + 0, r0);
                 tc::ld_32col(lane_addr + s_col + 32, r1);
                 tc::wait_ld();
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    s[i] = __uint_as_float(r0[i]);
-                    s[32 + i] = __uint_as_float(r1[i]);
+                    sv[i] = __uint_as_float(r0[i]);
+                    sv[32 + i] = __uint_as_float(r1[i]);
                 }
-                if (valid < kBN) {
+            }
+            if (valid < kBN) {
 #pragma unroll
-                    for (int i = 0; i < kBN; ++i)
-                        if (i >= valid) s[i] = -INFINITY;
-                }
+                for (int i = 0; i < kBN; ++i)
+                    if (i >= valid) sv[i] = -INFINITY;
+            }
+            // row max of the raw scores (scale > 0 commutes with max): eight
+            // independent 3-input max chains over 8 scores each
+            float mt;
+            {
                 float mx[8];
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
-                    float m = tc::max3f(s[k], s[k + 8], s[k + 16]);
-                    m = tc::max3f(m, s[k + 24], s[k + 32]);
-                    m = tc::max3f(m, s[k + 40], s[k + 48]);
-                    mx[k] = fmaxf(m, s[k + 56]);
+                    float m = tc::max3f(sv[k], sv[k + 8], sv[k + 16]);
+                    m = tc::max3f(m, sv[k + 24], sv[k + 32]);
+                    m = tc::max3f(m, sv[k + 40], sv[k + 48]);
+                    mx[k] = fmaxf(m, sv[k + 56]);
                 }
                 mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
                                fmaxf(mx[6], mx[7])) * a.scale_log2;
@@ -368,31 +371,19 @@ __global__ void __launch_bounds__(kThreads, 1)
                     m_ref = m_new;
                 }
             }
-            // ---- pass 2: S is read again 32 columns at a time (the next chunk's
-            // load overlaps this chunk's math), exponentiated, summed and
-            // written back as bf16 P over the columns already consumed
+            // exponentiate, sum and write P back as bf16 over S's columns
             const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
             const tc::f32x2 negm2 = tc::pack2(-m_ref, -m_ref);
             tc::f32x2 acc[4];
 #pragma unroll
             for (int k = 0; k < 4; ++k) acc[k] = tc::pack2(0.f, 0.f);
-            uint32_t buf[2][32];
-            tc::ld_32col(lane_addr + s_col, buf[0]);
-            tc::wait_ld();
 #pragma unroll
             for (int c = 0; c < kBN / 32; ++c) {
-                if (c + 1 < kBN / 32) tc::ld_32col(lane_addr + s_col + (c + 1) * 32, buf[(c + 1) & 1]);
                 uint32_t r[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int idx = c * 32 + 2 * i;
-                    float s0 = __uint_as_float(buf[c & 1][2 * i]);
-                    float s1 = __uint_as_float(buf[c & 1][2 * i + 1]);
-                    if (valid < kBN) {
-                        if (idx >= valid) s0 = -INFINITY;
-                        if (idx + 1 >= valid) s1 = -INFINITY;
-                    }
-                    const tc::f32x2 t = tc::fma2(tc::pack2(s0, s1), scale2, negm2);
+                    const tc::f32x2 t = tc::fma2(tc::pack2(sv[idx], sv[idx + 1]), scale2, negm2);
                     float t0, t1, p0, p1;
                     tc::unpack2(t, t0, t1);
                     if (((idx >> 1) & 7) < kPolyPairsOf8) {
@@ -404,11 +395,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
                     r[i] = pack_bf16x2(p0, p1);
                 }
-                // P chunk c lands on columns [16c, 16c+16) of S, which chunks
-                // <= c have already delivered; the load in flight reads
-                // columns >= 32(c+1)
                 tc::st_16col(lane_addr + s_col + c * 16, r);
-                if (c + 1 < kBN / 32) tc::wait_ld();
             }
             {
                 float a0, a1;
