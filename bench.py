@@ -193,12 +193,19 @@ class ClockSampler:
 
 # ----------------------------------------------------------------- the stack
 class AttentionStack:
-    """One PAB sampling run of the three attention kinds through libpab."""
+    """One PAB sampling run of the three attention kinds through libpab.
 
-    def __init__(self, pab, w, device):
-        self.pab, self.w, self.dev = pab, w, device
+    fused=False: temporal attention as the three layouts + temporal-view
+    kernel + layout back (every step of the hot path runs);
+    fused=True: the temporal kernel reads and writes the spatial view itself
+    (pab_plan_set_temporal_view), no layout launches."""
+
+    def __init__(self, pab, w, device, fused=False):
+        self.pab, self.w, self.dev, self.fused = pab, w, device, fused
         self.plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges,
                              dtype=torch.bfloat16)
+        if fused:
+            self.plan.set_temporal_view(True)
         self.plan.prepare()
         T, N, C = w.T, w.N, w.C
         # temporal-view scratch and the spatial-view copy of the temporal output
@@ -218,7 +225,7 @@ class AttentionStack:
         for i in range(self.w.steps):
             for k in synth.KINDS:
                 if self.sched[k][i]:
-                    n += 1 if k != "temporal" else 5  # 3 layouts + attention + layout back
+                    n += 1 if (k != "temporal" or self.fused) else 5  # 3 layouts + attention + layout back
                     if not first[k]:
                         n += 2  # MSE: partials + final
                     first[k] = False
@@ -252,7 +259,12 @@ class AttentionStack:
                 if not self.sched[k][i]:
                     self.last_ptr[k] = plan.attention_ptr(k, i, None, None, None, stream)
                     continue
-                if k == "temporal":
+                if k == "temporal" and self.fused:
+                    ptr = timed("temporal", lambda: plan.attention_ptr(k, i, x[k]["q"], x[k]["k"], x[k]["v"],
+                                                                       stream))
+                    self.last_ptr[k] = ptr
+                    cur = pab._wrap(ptr, (T, N, C), torch.bfloat16, self.dev)
+                elif k == "temporal":
                     for src, dst in ((x[k]["q"], self.tq), (x[k]["k"], self.tk), (x[k]["v"], self.tv)):
                         timed("layout", lambda: pab.layout(src, True, out=dst, stream=stream))
                     ptr = timed("temporal", lambda: plan.attention_ptr(k, i, self.tq, self.tk, self.tv, stream))
@@ -476,6 +488,29 @@ def run_ours(args):
         "kernels": kernels,
         "clocks": clk,
     }
+
+    # the same stack with the temporal kernel reading / writing the spatial
+    # view itself (no layout launches): reported beside the main figure
+    fstack = AttentionStack(pab, w, device, fused=True)
+    for _ in range(args.warmup):
+        fstack.run(inputs, stream)
+    fsteps = max(3, args.steps // 4)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    f0 = torch.cuda.Event(enable_timing=True)
+    f1 = torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(fsteps):
+        fstack.run(inputs, stream)
+    f1.record(stream)
+    torch.cuda.synchronize(device)
+    fms = max_over_ranks(f0.elapsed_time(f1) / fsteps, device)
+    line["fused_temporal_view"] = {
+        "value": world * dense_flops / (fms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": fms, "steps": fsteps,
+        "denoising_steps_per_s": world * w.steps / (fms * 1e-3),
+        "gpu_launches": fstack.launches_per_run * fsteps,
+        "note": "temporal attention reads/writes the spatial view via TMA; no layout launches"}
+    fstack.close()
 
     if not args.no_e2e:
         line["e2e"] = run_e2e(pab, w, stack, device, stream, args)

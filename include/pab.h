@@ -89,6 +89,14 @@ int pab_spatial_attention(const void* q, const void* k, const void* v, void* out
 int pab_temporal_attention(const void* q, const void* k, const void* v, void* out,
                            int N, int T, int heads, int d, void* cuda_stream);
 
+/* Temporal attention taking and returning the SPATIAL view: q, k, v, out are
+ * [T, N, C]; out[t, n, h] is the same value pab_temporal_attention gives for
+ * the permuted tensors.  The kernel gathers each position's T frames at
+ * stride N*C itself, so a caller holding the spatial view needs no
+ * pab_layout calls around it.  T <= 128.  PAB_BF16 only. */
+int pab_temporal_attention_sv(const void* q, const void* k, const void* v, void* out,
+                              int T, int N, int heads, int d, void* cuda_stream);
+
 /* Cross attention (same section: video tokens to text tokens).
  * q, out: [R, C] (R video tokens in any order; out keeps it);
  * kt, vt: [text_len, C].  Every text token is attended (no text mask).
@@ -173,6 +181,11 @@ int pab_plan_destroy(pab_plan* plan);
  * Device memory is kept. */
 int pab_plan_reset(pab_plan* plan);
 
+/* Choose the layout of TEMPORAL q, k, v and of its output for this plan:
+ * spatial_view = 0 (default) -> [N, T, C]; 1 -> [T, N, C] (the spatial view,
+ * no layout change needed around the call).  Call before the run starts. */
+int pab_plan_set_temporal_view(pab_plan* plan, int spatial_view);
+
 /* Allocate the cache (2 output slots per kind, plus bf16 staging for
  * PAB_FP32 plans) on the current device now instead of at each kind's first
  * compute.  Idempotent. */
@@ -192,7 +205,8 @@ int pab_schedule_count(const pab_plan* plan, int kind, int* computes);
 /* Run attention `kind` for diffusion step `step` under the schedule.
  *  Compute step: runs the kind's kernel on cuda_stream into one of the
  *    plan's two output slots of that kind and sets *out to it.
- *    Shapes: SPATIAL q,k,v [T, N, C]; TEMPORAL q,k,v [N, T, C];
+ *    Shapes: SPATIAL q,k,v [T, N, C]; TEMPORAL q,k,v [N, T, C] (or
+ *    [T, N, C] after pab_plan_set_temporal_view(plan, 1));
  *    CROSS q [T*N, C], k,v [text_len, C].  *out has q's layout.
  *  Broadcast hit: launches nothing, copies nothing, ignores q, k, v (which
  *    may be NULL) and sets *out to the slot that holds the output of the

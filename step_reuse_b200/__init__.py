@@ -33,6 +33,7 @@ BF16, FP32 = 0, 1
 # every symbol include/pab.h declares
 EXPORTS = (
     "pab_version", "pab_last_error_string", "pab_spatial_attention", "pab_temporal_attention",
+    "pab_temporal_attention_sv", "pab_plan_set_temporal_view",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
     "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
@@ -61,6 +62,8 @@ def _load() -> ctypes.CDLL:
         "pab_last_error_string": ([], ctypes.c_char_p),
         "pab_spatial_attention": ([vp, vp, vp, vp, i, i, i, i, vp], i),
         "pab_temporal_attention": ([vp, vp, vp, vp, i, i, i, i, vp], i),
+        "pab_temporal_attention_sv": ([vp, vp, vp, vp, i, i, i, i, vp], i),
+        "pab_plan_set_temporal_view": ([vp, i], i),
         "pab_cross_attention": ([vp, vp, vp, vp, ll, i, i, i, vp], i),
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
         "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
@@ -134,6 +137,15 @@ def temporal_attention(q, k, v, heads: int, out=None, stream=None):
     out = torch.empty_like(q) if out is None else out
     _check(lib.pab_temporal_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), N, T, heads, C // heads,
                                       _stream(stream)))
+    return out
+
+
+def temporal_attention_sv(q, k, v, heads: int, out=None, stream=None):
+    """Temporal attention on the spatial view: q, k, v [T, N, C] -> [T, N, C]."""
+    T, N, C = q.shape
+    out = torch.empty_like(q) if out is None else out
+    _check(lib.pab_temporal_attention_sv(_ptr(q), _ptr(k), _ptr(v), _ptr(out), T, N, heads, C // heads,
+                                         _stream(stream)))
     return out
 
 
@@ -227,6 +239,11 @@ class Plan:
     def reset(self):
         _check(lib.pab_plan_reset(self._h))
 
+    def set_temporal_view(self, spatial_view: bool):
+        """True: TEMPORAL takes and returns [T, N, C] instead of [N, T, C]."""
+        _check(lib.pab_plan_set_temporal_view(self._h, 1 if spatial_view else 0))
+        self.temporal_sv = bool(spatial_view)
+
     def prepare(self):
         _check(lib.pab_plan_prepare(self._h))
 
@@ -259,7 +276,8 @@ class Plan:
     def attention(self, kind, step: int, q=None, k=None, v=None, stream=None) -> torch.Tensor:
         kind = KIND.get(kind, kind)
         ptr = self.attention_ptr(kind, step, q, k, v, stream)
-        shape = {SPATIAL: (self.T, self.N, self.C), TEMPORAL: (self.N, self.T, self.C),
+        tshape = (self.T, self.N, self.C) if getattr(self, "temporal_sv", False) else (self.N, self.T, self.C)
+        shape = {SPATIAL: (self.T, self.N, self.C), TEMPORAL: tshape,
                  CROSS: (self.T * self.N, self.C)}[kind]
         dev = q.device if q is not None else torch.device("cuda", torch.cuda.current_device())
         return _wrap(ptr, shape, self.dtype, dev)

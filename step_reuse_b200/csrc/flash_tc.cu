@@ -68,7 +68,7 @@ constexpr float kRescaleLog2 = 8.0f;
 #endif
 constexpr int kPolyPairsOf8 = PAB_POLY_PAIRS_OF_8;
 // 2^f ~ kP0 + kP1 f + kP2 f^2 + kP3 f^3 on [-0.5, 0.5] (see exp2_poly2)
-constexpr float kP0 = 0.999928057f, kP1 = 0.693260968f, kP2 = 0.242611125f, kP3 = 0.0551716685f;
+constexpr float kP0 = 1.0f, kP1 = 0.693282962f, kP2 = 0.242210999f, kP3 = 0.0550089180f;
 
 __device__ unsigned int g_flash_err = 0;
 
@@ -110,9 +110,10 @@ PAB_DEV float ex2(float x) {
 // rescaled softmax never exceeds 2^8).  Cody-Waite style range reduction:
 // x = n + f with n = rint(x) (the 1.5*2^23 rounding trick) and f in
 // [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted here by minimising the
-// maximum relative error on [-0.5, 0.5] (linear-programming minimax fit; max
-// relative error 7.5e-5, far below the bf16 rounding of P); 2^n is added to
-// the exponent field.  x below -120 is clamped (the result, ~1e-36, is
+// maximum relative error on [-0.5, 0.5] with p(0) = 1 fixed, so integer x
+// give exact powers of two (linear-programming minimax fit; max relative
+// error 1.0e-4, far below the bf16 rounding of P); 2^n is added to the
+// exponent field.  x below -120 is clamped (the result, ~1e-36, is
 // negligible next to the row maximum's weight 1).
 PAB_DEV void exp2_poly2(float x0, float x1, float& p0, float& p1) {
     const tc::f32x2 x = tc::pack2(fmaxf(x0, -120.0f), fmaxf(x1, -120.0f));

@@ -26,8 +26,9 @@ cudaError_t launch_layout(int to_temporal, const void* src, void* dst, int T, in
 unsigned int layout_device_errors(bool clear);
 
 // --- temporal short-sequence attention ([N,T,C], L = T) -------------------
+// spatial_view = 1: q, k, v, out are [T, N, C] instead of [N, T, C]
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
-                            int heads, int d, cudaStream_t s);
+                            int heads, int d, int spatial_view, cudaStream_t s);
 unsigned int temporal_device_errors(bool clear);
 
 // --- flash attention for spatial (per frame) and cross (shared text K/V) --
@@ -38,6 +39,11 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
                          long long kv_bstride, cudaStream_t s);
 
 unsigned int flash_device_errors(bool clear);
+
+// --- cross attention (text_len <= 128: persistent cross_tc; longer: flash) --
+cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,
+                         int d, cudaStream_t s);
+unsigned int cross_device_errors(bool clear);
 
 // --- dtype conversion for fp32 plans --------------------------------------
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t s);

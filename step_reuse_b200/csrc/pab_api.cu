@@ -105,14 +105,14 @@ int run_spatial(const void* q, const void* k, const void* v, void* out, int T, i
 }
 
 int run_temporal(const void* q, const void* k, const void* v, void* out, int N, int T, int heads,
-                 int d, cudaStream_t s) {
-    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, s);
+                 int d, int spatial_view, cudaStream_t s) {
+    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "temporal attention launch");
 }
 
 int run_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lt,
               int heads, int d, cudaStream_t s) {
-    cudaError_t e = pab::launch_flash(q, kt, vt, out, 1, R, Lt, heads, d, 0, 0, s);
+    cudaError_t e = pab::launch_cross(q, kt, vt, out, R, Lt, heads, d, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "cross attention launch");
 }
 
@@ -149,6 +149,7 @@ struct pab_plan {
     long long C;
     int range[3];
     int edge_pct, lo, hi;
+    int temporal_sv;  // temporal attention takes / returns the spatial view
     // cache
     int device;
     void* slot[3][2];
@@ -237,7 +238,7 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
     if (kind == PAB_SPATIAL)
         rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s);
     else if (kind == PAB_TEMPORAL)
-        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, s);
+        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, p->temporal_sv, s);
     else
         rc = run_cross(qq, kk, vv, oo, (long long)p->T * p->N, p->text_len, p->heads, p->d, s);
     if (rc) return rc;
@@ -290,7 +291,21 @@ int pab_temporal_attention(const void* q, const void* k, const void* v, void* ou
     if ((long long)T * N == 0) return PAB_OK;
     rc = check_ptrs("q, k, v, out", q, k, v, out);
     if (rc) return rc;
-    return run_temporal(q, k, v, out, N, T, heads, d, static_cast<cudaStream_t>(cuda_stream));
+    return run_temporal(q, k, v, out, N, T, heads, d, 0, static_cast<cudaStream_t>(cuda_stream));
+    PAB_GUARD_END
+}
+
+int pab_temporal_attention_sv(const void* q, const void* k, const void* v, void* out, int T, int N,
+                              int heads, int d, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || N < 0) return fail(PAB_ERR_ARG, "T (%d) and N (%d) must be >= 0", T, N);
+    if (T > 128) return fail(PAB_ERR_UNSUPPORTED, "temporal length T=%d exceeds 128", T);
+    if ((long long)T * N == 0) return PAB_OK;
+    rc = check_ptrs("q, k, v, out", q, k, v, out);
+    if (rc) return rc;
+    return run_temporal(q, k, v, out, N, T, heads, d, 1, static_cast<cudaStream_t>(cuda_stream));
     PAB_GUARD_END
 }
 
@@ -378,8 +393,8 @@ int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype, doub
 int pab_device_errors(int clear, unsigned int* flags) {
     PAB_GUARD_BEGIN
     if (!flags) return fail(PAB_ERR_ARG, "null flags pointer");
-    const unsigned int words[3] = {pab::layout_device_errors(clear != 0), pab::flash_device_errors(clear != 0),
-                                   pab::temporal_device_errors(clear != 0)};
+    const unsigned int words[4] = {pab::layout_device_errors(clear != 0), pab::flash_device_errors(clear != 0),
+                                   pab::temporal_device_errors(clear != 0), pab::cross_device_errors(clear != 0)};
     unsigned int v = 0;
     for (unsigned int w : words) {
         if (w == 0xffffffffu) return fail(PAB_ERR_CUDA, "could not read the device status words");
@@ -458,6 +473,13 @@ int pab_plan_reset(pab_plan* plan) {
         plan->cached_step[k] = -1;
         plan->last_step[k] = -1;
     }
+    return PAB_OK;
+}
+
+int pab_plan_set_temporal_view(pab_plan* plan, int spatial_view) {
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    if (spatial_view != 0 && spatial_view != 1) return fail(PAB_ERR_ARG, "spatial_view must be 0 or 1");
+    plan->temporal_sv = spatial_view;
     return PAB_OK;
 }
 

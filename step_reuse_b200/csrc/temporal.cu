@@ -1,7 +1,8 @@
 // temporal.cu -- temporal attention: at every spatial position n and head h
 // the T frames attend to each other (PAB report, "Implementation": temporal
 // attention, the mid-frequency kind).  q, k, v, out: [N, T, C] (temporal
-// view), bf16.  L = T is short (16..64 in the workloads), the batch
+// view) or, with no separate layout change, [T, N, C] (spatial view: the TMA
+// tensor maps gather a position's frames at stride N*C), bf16.  L = T is short (16..64 in the workloads), the batch
 // (N * heads) is in the tens of thousands, so the kernel is HBM-bound
 // (2 * T * d * 2 flop per loaded byte ~ 8-32 flop/B).
 //
@@ -37,6 +38,7 @@ __device__ unsigned int g_temporal_err = 0;
 
 struct TemporalArgs {
     int N, T, heads, d;
+    int spatial_view;  // 1: tensors are [T, N, C] (tensor map dims (d, heads, N, T))
     int G;       // heads per unit
     int P;       // smem row pitch (elements) = TMA box width
     int RT;      // rows per head block in smem (T rounded up to 16)
@@ -96,11 +98,13 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
         const int h0 = (int)(unit - (long long)n * hg_count) * G;
         const uint32_t bar = smem_u32(&full_bar[stage]);
         mbar_arrive_expect_tx(bar, unit_bytes);
+        // position n is coordinate 3 of the temporal-view map, 2 of the spatial-view one
+        const int c2 = p.spatial_view ? n : 0, c3 = p.spatial_view ? 0 : n;
         for (int g = 0; g < G; ++g) {
             const uint32_t dst = sbase_u32 + 2u * (stage * stage_elems + g * head_elems);
-            tc::tma_load_4d(dst, &tm_q, 0, h0 + g, 0, n, bar);
-            tc::tma_load_4d(dst + 2u * tensor_elems, &tm_k, 0, h0 + g, 0, n, bar);
-            tc::tma_load_4d(dst + 4u * tensor_elems, &tm_v, 0, h0 + g, 0, n, bar);
+            tc::tma_load_4d(dst, &tm_q, 0, h0 + g, c2, c3, bar);
+            tc::tma_load_4d(dst + 2u * tensor_elems, &tm_k, 0, h0 + g, c2, c3, bar);
+            tc::tma_load_4d(dst + 4u * tensor_elems, &tm_v, 0, h0 + g, c2, c3, bar);
         }
     };
 
@@ -242,8 +246,10 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
         if (tid == 0) {
             const int n = (int)(u / hg_count);
             const int h0 = (int)(u - (long long)n * hg_count) * G;
+            const int c2 = p.spatial_view ? n : 0, c3 = p.spatial_view ? 0 : n;
             for (int g = 0; g < G; ++g)
-                tc::tma_store_4d(&tm_o, sbase_u32 + 2u * (stage * stage_elems + g * head_elems), 0, h0 + g, 0, n);
+                tc::tma_store_4d(&tm_o, sbase_u32 + 2u * (stage * stage_elems + g * head_elems), 0, h0 + g, c2,
+                                 c3);
             bulk_commit();
         }
     }
@@ -258,9 +264,12 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
     }
 }
 
-// 4-D map over [N][T][heads][d] (row stride C): dims (d, heads, T, N),
-// box (P, 1, T, 1), no swizzle; columns d..P-1 of the box read as zero.
-bool make_map(CUtensorMap* m, const void* base, int d, int heads, int T, int N, int P) {
+// 4-D map over the temporal view [N][T][heads][d]: dims (d, heads, T, N),
+// box (P, 1, T, 1); or over the spatial view [T][N][heads][d]: dims
+// (d, heads, N, T), box (P, 1, 1, T).  Either way one box is a position's T
+// frames of one head, landing as [T][P] in shared memory.  No swizzle;
+// columns d..P-1 of the box read as zero.
+bool make_map(CUtensorMap* m, const void* base, int d, int heads, int T, int N, int P, int spatial_view) {
     typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                       const cuuint64_t*, const cuuint32_t*, const cuuint32_t*,
                                       CUtensorMapInterleave, CUtensorMapSwizzle, CUtensorMapL2promotion,
@@ -278,6 +287,13 @@ bool make_map(CUtensorMap* m, const void* base, int d, int heads, int T, int N, 
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)T, (cuuint64_t)N};
     cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)C * 2, (cuuint64_t)T * C * 2};
     cuuint32_t box[4] = {(cuuint32_t)P, 1, (cuuint32_t)T, 1};
+    if (spatial_view) {
+        dims[2] = (cuuint64_t)N;
+        dims[3] = (cuuint64_t)T;
+        strides[2] = (cuuint64_t)N * C * 2;
+        box[2] = 1;
+        box[3] = (cuuint32_t)T;
+    }
     cuuint32_t estr[4] = {1, 1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -302,8 +318,9 @@ cudaError_t launch_dn(const CUtensorMap* maps, const TemporalArgs& p, size_t sme
 }  // namespace
 
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
-                            int heads, int d, cudaStream_t s) {
+                            int heads, int d, int spatial_view, cudaStream_t s) {
     TemporalArgs p;
+    p.spatial_view = spatial_view;
     p.N = N;
     p.T = T;
     p.heads = heads;
@@ -324,7 +341,7 @@ cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* o
     CUtensorMap maps[4];
     const void* bases[4] = {q, k, v, out};
     for (int i = 0; i < 4; ++i)
-        if (!make_map(&maps[i], bases[i], d, heads, T, N, p.P)) return cudaErrorInvalidValue;
+        if (!make_map(&maps[i], bases[i], d, heads, T, N, p.P, spatial_view)) return cudaErrorInvalidValue;
     const size_t smem = (size_t)2 * 3 * G * p.RT * p.P * 2 + 256;
     switch (d / 8) {
 #define PAB_T_CASE(DNV) \

@@ -95,6 +95,9 @@ def test_temporal_parity(pab, oracle_mod, N, T, heads, d):
     (129, 1, 2, 64),      # a single text token: output = v row
     (77, 512, 2, 64),     # documented maximum text_len
     (64, 300, 3, 24),
+    (5000, 120, 16, 72),  # 640 query tiles: several per CTA, heads change inside a CTA's run
+    (100, 64, 300, 8),    # one query tile per head: the head changes at every tile
+    (25440, 120, 4, 72),  # a 480p frame stack's rows, 4 heads
 ])
 def test_cross_parity(pab, oracle_mod, R, Lt, heads, d):
     C = heads * d
@@ -106,7 +109,10 @@ def test_cross_parity(pab, oracle_mod, R, Lt, heads, d):
     assert_attn_close(out, want, f"cross R={R} Lt={Lt} h={heads} d={d}")
     check_guards(base)
     if Lt == 1:
-        assert torch.equal(out.view(torch.int16), vt.expand(R, C).contiguous().view(torch.int16))
+        want1 = vt.expand(R, C).contiguous()
+        bad = (out.view(torch.int16) != want1.view(torch.int16)).nonzero()
+        assert bad.numel() == 0, (f"{bad.shape[0]} elements differ; first {bad[:8].tolist()}; "
+                                  f"got {out[bad[:4, 0], bad[:4, 1]].tolist()} want {want1[bad[:4, 0], bad[:4, 1]].tolist()}")
 
 
 def test_cross_row_order_is_kept(pab):
@@ -171,3 +177,22 @@ def test_mse_special_cases(pab):
     x = (ints.float() / 8).to(torch.bfloat16).cuda()
     y = (x.float() + 0.25).to(torch.bfloat16)
     assert pab.attn_diff_mse(y, x) == 0.0625
+
+
+# ------------------------------------------------------------------ temporal on the spatial view
+@pytest.mark.parametrize("T,N,heads,d", [(16, 37, 16, 72), (24, 50, 4, 128), (64, 20, 16, 64), (4, 33, 2, 32),
+                                         (1, 9, 2, 64), (17, 11, 3, 40)])
+def test_temporal_spatial_view(pab, oracle_mod, T, N, heads, d):
+    """[T, N, C] in and out, no layout change: bit-identical to permuting,
+    running the temporal-view kernel and permuting back; and oracle parity."""
+    C = heads * d
+    q, k, v = (randn((T, N, C), s) for s in (71, 72, 73))
+    base, out = guarded_empty((T, N, C), torch.bfloat16)
+    pab.temporal_attention_sv(q, k, v, heads, out=out)
+    check_guards(base)
+    tv = [x.permute(1, 0, 2).contiguous() for x in (q, k, v)]
+    ref = pab.temporal_attention(*tv, heads).permute(1, 0, 2).contiguous()
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
+    want = oracle_mod.temporal_attention(*(np.transpose(to_f64(x), (1, 0, 2)) for x in (q, k, v)), heads)
+    assert_attn_close(out, np.transpose(want, (1, 0, 2)), f"temporal_sv T={T} N={N} h={heads} d={d}")
+    no_device_errors(pab)

@@ -139,6 +139,29 @@ def test_large_runs_sampled(pab, oracle_mod, name):
             mse_steps={1, w.steps - 1})
 
 
+def test_plan_temporal_spatial_view(pab, oracle_mod):
+    """A plan set to the spatial view takes [T, N, C] temporal inputs and
+    returns [T, N, C]; hits still serve the cached slot bit-identically."""
+    w = synth.WORKLOADS["480p"]
+    plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges, dtype=w.torch_dtype)
+    plan.set_temporal_view(True)
+    x = synth.initial_inputs(w, device="cuda")
+    q, k, v = (x["temporal"][n].reshape(w.N, w.T, w.C).permute(1, 0, 2).contiguous() for n in ("q", "k", "v"))
+    out = plan.attention("temporal", 0, q, k, v)
+    assert out.shape == (w.T, w.N, w.C)
+    rng = np.random.default_rng(5)
+    pos = np.sort(rng.choice(w.N, size=256, replace=False))
+    want = oracle_mod.temporal_attention(*(np.transpose(to_f64(t[:, pos]), (1, 0, 2)) for t in (q, k, v)), w.heads)
+    assert_attn_close(out[:, pos], np.transpose(want, (1, 0, 2)), "plan temporal spatial view")
+    saved = out.clone()
+    e = oracle_mod.edge_steps(w.steps)
+    for i in range(1, e + 1):
+        plan.attention("temporal", i, q, k, v)
+    hit = plan.attention("temporal", e + 1)
+    assert not plan.is_compute("temporal", e + 1) and hit.shape == (w.T, w.N, w.C)
+    plan.close()
+
+
 def test_sweep_u_shape_and_counts(pab, oracle_mod):
     """Sweep workload (480p shapes, 50 steps, drift 0.2 on edge steps, 0.02 in
     the middle): the compute counts follow the ranges, and with no broadcast
