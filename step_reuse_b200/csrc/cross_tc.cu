@@ -12,8 +12,9 @@
 //                            issuers' MMAs on the old ones have retired --
 //                            a barrier each issuer commits once per change,
 //                            so no wait is ever two phases behind) and the query
-//                            tiles, up to three ahead, through four Q
-//                            buffers;
+//                            tiles through a ring of three Q buffers; a
+//                            buffer is refilled as soon as its S product has
+//                            retired, so loads run two to three tiles ahead;
 //   warps 9, 10 (one thread) tcgen05.mma issuers, one per slot: S = Q Kt^T
 //                            (SS form, fp32 in TMEM) and O = P Vt (TS form,
 //                            P from TMEM);
@@ -22,7 +23,7 @@
 //                            text_len, exponentiates (MUFU ex2 with a share
 //                            on the FMA pipes), writes P as bf16 over S, then
 //                            normalises O, stages it (128-byte swizzle) in the
-//                            tile's Q buffer and stores it with TMA.
+//                            slot's output buffer and stores it with TMA.
 // TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+NO), O_1 [384,384+NO).
 // Every wait is bounded; on time-out the CTA raises the error word, drains
 // its copies and MMAs, frees TMEM and exits.
@@ -51,11 +52,13 @@ struct CrossArgs {
     float scale_log2;  // log2(e) / sqrt(d)
 };
 
+constexpr int kQBufs = 3;
+
 struct Bars {
     unsigned long long kv_full;
     unsigned long long kv_free;  // both issuers are done with the previous head's Kt / Vt
-    unsigned long long q_full[4];
-    unsigned long long q_free[4];
+    unsigned long long q_full[kQBufs];
+    unsigned long long q_free[kQBufs];  // the S product reading the buffer retired
     unsigned long long s_done[2];
     unsigned long long p_full[2];
     unsigned long long o_full[2];
@@ -113,22 +116,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ Bars bars;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t q_s = sbase;              // [4 buffers][NB boxes]
-    const uint32_t k_s = q_s + 4 * kTile;    // [NB boxes]
-    const uint32_t v_s = k_s + kTile;        // [NB boxes]
+    const uint32_t q_s = sbase;                 // [kQBufs][NB boxes]
+    const uint32_t o_s = q_s + kQBufs * kTile;  // [2 slots][NB boxes]: output staging
+    const uint32_t k_s = o_s + 2 * kTile;       // [NB boxes]
+    const uint32_t v_s = k_s + kTile;           // [NB boxes]
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // this CTA's contiguous run of work items
-    const long long per = (a.tiles + gridDim.x - 1) / gridDim.x;
-    const long long t_begin = (long long)blockIdx.x * per;
-    const long long t_end = t_begin + per < a.tiles ? t_begin + per : a.tiles;
-    const int n = t_begin < t_end ? (int)(t_end - t_begin) : 0;
+    // (work-item indices fit 32 bits: heads * query tiles < 2^31, checked on the host)
+    const int tiles = (int)a.tiles;
+    const int per = (tiles + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int t_begin = (int)blockIdx.x * per;
+    const int t_end = t_begin + per < tiles ? t_begin + per : tiles;
+    const int n = t_begin < t_end ? t_end - t_begin : 0;
 
     if (threadIdx.x == 256) {
         mbar_init(smem_u32(&bars.kv_full), 1);
         mbar_init(smem_u32(&bars.kv_free), 2);
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < kQBufs; ++b) {
             mbar_init(smem_u32(&bars.q_full[b]), 1);
             mbar_init(smem_u32(&bars.q_free[b]), 1);
         }
@@ -161,8 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             int cur_h = -1, heads_loaded = 0, nq = 0;
             bool ok = true;
             for (int i = 0; i < n && ok; ++i) {
-                const long long t = t_begin + i;
-                const int h = (int)(t / a.nqt), qt = (int)(t - (long long)h * a.nqt);
+                const int t = t_begin + i;
+                const int h = t / a.nqt, qt = t - h * a.nqt;
                 if (h != cur_h) {
                     // every MMA of the earlier tiles has retired before Kt / Vt change:
                     // each issuer commits kv_free once per head change
@@ -176,8 +182,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     cur_h = h;
                     ++heads_loaded;
                 }
-                const int b = i & 3;
-                if (i >= 4) ok = wait_bar(&bars, &bars.q_free[b], ((i - 4) >> 2) & 1);
+                const int b = i % kQBufs;
+                if (i >= kQBufs) ok = wait_bar(&bars, &bars.q_free[b], ((i / kQBufs) - 1) & 1);
                 if (!ok) break;
                 mbar_arrive_expect_tx(smem_u32(&bars.q_full[b]), kTile);
                 for (int bx = 0; bx < NB; ++bx)
@@ -187,8 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (!ok || *(volatile int*)&bars.abort) {
                 // drain: every load issued lands before the CTA exits (bounded)
-                for (int i = (nq > 4 ? nq - 4 : 0); i < nq; ++i)
-                    mbar_wait_bounded(smem_u32(&bars.q_full[i & 3]), (i >> 2) & 1, &g_cross_err);
+                for (int i = (nq > kQBufs ? nq - kQBufs : 0); i < nq; ++i)
+                    mbar_wait_bounded(smem_u32(&bars.q_full[i % kQBufs]), (i / kQBufs) & 1, &g_cross_err);
                 if (heads_loaded > 0)
                     mbar_wait_bounded(smem_u32(&bars.kv_full), (heads_loaded - 1) & 1, &g_cross_err);
             }
@@ -204,12 +210,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t dv = tc::smem_desc(v_s, kBox, 1024, 2);
             const uint32_t s_t = tmem + x * 128, o_t = tmem + 256 + x * 128;
             int heads_seen = 0;
-            long long hcur = -1;
+            int hcur = -1;
             bool ok = true;
             for (int i = 0; i < n && ok; ++i) {
                 // follow every Kt / Vt reload in order (also those at the other
                 // slot's tiles), so a wait is never two phases behind
-                const long long h = (t_begin + i) / a.nqt;
+                const int h = (t_begin + i) / a.nqt;
                 if (h != hcur) {
                     // release the old head's Kt / Vt once this issuer's MMAs on them
                     // retire, then wait for the new ones
@@ -220,16 +226,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (!ok) break;
                 }
                 if ((i & 1) != x) continue;
-                if (ok) ok = wait_bar(&bars, &bars.q_full[i & 3], (i >> 2) & 1);
+                const int qb = i % kQBufs;
+                if (ok) ok = wait_bar(&bars, &bars.q_full[qb], (i / kQBufs) & 1);
                 if (!ok) break;
                 tc::fence_after_sync();
-                const uint64_t a0 = dq + (uint64_t)(((i & 3) * kTile) >> 4);
+                const uint64_t a0 = dq + (uint64_t)((qb * kTile) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const uint32_t off = (ks >> 2) * (kBox >> 4) + (ks & 3) * 2;
                     tc::mma_ss(s_t, a0 + off, dk + off, idesc_s, ks > 0 ? 1u : 0u);
                 }
                 tc::commit(smem_u32(&bars.s_done[x]));
+                tc::commit(smem_u32(&bars.q_free[qb]));  // the Q buffer may be refilled
                 // O_X is free once the previous tile of this slot was read out
                 if (i >= 2) ok = wait_bar(&bars, &bars.o_free[x], ((i - 2) >> 1) & 1);
                 if (ok) ok = wait_bar(&bars, &bars.p_full[x], (i >> 1) & 1);
@@ -258,31 +266,33 @@ __global__ void __launch_bounds__(kThreads, 1)
             // pass 1: row max over the text keys (scale > 0 commutes with max)
             float mrow;
             {
-                float sv[kBN];
-                uint32_t r0[32], r1[32], r2[32], r3[32];
-                tc::ld_32col(lane_addr + s_col + 0, r0);
-                tc::ld_32col(lane_addr + s_col + 32, r1);
-                tc::ld_32col(lane_addr + s_col + 64, r2);
-                tc::ld_32col(lane_addr + s_col + 96, r3);
-                tc::wait_ld();
-#pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    sv[c] = __uint_as_float(r0[c]);
-                    sv[32 + c] = __uint_as_float(r1[c]);
-                    sv[64 + c] = __uint_as_float(r2[c]);
-                    sv[96 + c] = __uint_as_float(r3[c]);
-                }
-#pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (c >= a.Lk) sv[c] = -INFINITY;
-                // eight independent chains; chain k covers scores k, k+8, ..., k+120
+                // two halves of 64 scores keep the register footprint low;
+                // eight independent 3-input max chains per half
                 float mx[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    float m = tc::max3f(sv[k], sv[k + 8], sv[k + 16]);
+                for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
 #pragma unroll
-                    for (int mm = 3; mm + 1 < kBN / 8; mm += 2) m = tc::max3f(m, sv[k + 8 * mm], sv[k + 8 * mm + 8]);
-                    mx[k] = fmaxf(m, sv[k + kBN - 8]);
+                for (int half = 0; half < 2; ++half) {
+                    uint32_t r0[32], r1[32];
+                    tc::ld_32col(lane_addr + s_col + half * 64, r0);
+                    tc::ld_32col(lane_addr + s_col + half * 64 + 32, r1);
+                    tc::wait_ld();
+                    float sv[64];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) {
+                        sv[c] = __uint_as_float(r0[c]);
+                        sv[32 + c] = __uint_as_float(r1[c]);
+                    }
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (half * 64 + c >= a.Lk) sv[c] = -INFINITY;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        float m = tc::max3f(mx[k], sv[k], sv[k + 8]);
+                        m = tc::max3f(m, sv[k + 16], sv[k + 24]);
+                        m = tc::max3f(m, sv[k + 32], sv[k + 40]);
+                        mx[k] = tc::max3f(m, sv[k + 48], sv[k + 56]);
+                    }
                 }
                 mrow = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
                                  fmaxf(mx[6], mx[7])) * a.scale_log2;
@@ -337,13 +347,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = wait_bar(&bars, &bars.o_full[x], (i >> 1) & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            if (row == 0 && i >= 2) {
-                // tile i-2's store has read its buffer: hand it back to the producer
-                bulk_wait_read<0>();
-                mbar_arrive(smem_u32(&bars.q_free[(i - 2) & 3]));
-            }
+            // the slot's output buffer: tile i-2's store must have read it
+            if (row == 0) bulk_wait_read<0>();
+            tc::named_bar_sync(1 + x, 128);
             const float inv = 1.f / l;
-            unsigned char* stage = gen_base + (i & 3) * kTile;
+            unsigned char* stage = gen_base + (o_s - sbase) + x * kTile;
 #pragma unroll
             for (int c = 0; c < NO / 16; ++c) {
                 uint32_t r[16];
@@ -366,10 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             fence_proxy_async_smem();
             tc::named_bar_sync(1 + x, 128);
             if (row == 0) {
-                const long long t = t_begin + i;
-                const int h = (int)(t / a.nqt), qt = (int)(t - (long long)h * a.nqt);
+                const int t = t_begin + i;
+                const int h = t / a.nqt, qt = t - h * a.nqt;
                 for (int bx = 0; bx < NB; ++bx)
-                    tc::tma_store_4d(&tm_o, q_s + (i & 3) * kTile + bx * kBox, bx * 64, h, qt * kBM, 0);
+                    tc::tma_store_4d(&tm_o, o_s + x * kTile + bx * kBox, bx * 64, h, qt * kBM, 0);
                 bulk_commit();
             }
         }
@@ -414,7 +422,7 @@ bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows
 template <int KSTEPS>
 cudaError_t launch_ks(const CUtensorMap* m, const CrossArgs& a, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
-    const size_t smem = (size_t)6 * NB * kBox + 1024;
+    const size_t smem = (size_t)(kQBufs + 4) * NB * kBox + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
     cudaError_t e = cudaFuncSetAttribute(cross_tc_kernel<KSTEPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_req);
@@ -433,7 +441,9 @@ cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* ou
     if (Lk > kBN) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s);
     CrossArgs a;
     a.Lk = Lk;
-    a.nqt = (int)((R + kBM - 1) / kBM);
+    const long long nqt = (R + kBM - 1) / kBM;
+    if (nqt * heads >= (1LL << 31)) return cudaErrorInvalidValue;
+    a.nqt = (int)nqt;
     a.tiles = (long long)heads * a.nqt;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
     CUtensorMap m[4];
