@@ -132,8 +132,10 @@ PAB_DEV void exp2_poly2(float x0, float x1, float& p0, float& p1) {
     p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(y1) << 23));
 }
 
-// bounded wait that gives up at once when the CTA has already aborted
+// bounded wait that gives up at once when the CTA has already aborted (a
+// phase that has completed is taken without reading the abort flag)
 PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
+    if (mbar_test_wait(smem_u32(bar), parity)) return true;
     if (*(volatile int*)&b->abort) return false;
     if (!mbar_wait_bounded(smem_u32(bar), parity, &g_flash_err)) {
         *(volatile int*)&b->abort = 1;
