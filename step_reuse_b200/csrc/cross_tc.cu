@@ -286,9 +286,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         sv[c] = __uint_as_float(r0[c]);
                         sv[32 + c] = __uint_as_float(r1[c]);
                     }
+                    if ((half + 1) * 64 > a.Lk) {  // uniform: only the half holding the end of the keys
 #pragma unroll
-                    for (int c = 0; c < 64; ++c)
-                        if (half * 64 + c >= a.Lk) sv[c] = -INFINITY;
+                        for (int c = 0; c < 64; ++c)
+                            if (half * 64 + c >= a.Lk) sv[c] = -INFINITY;
+                    }
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
                         float m = tc::max3f(mx[k], sv[k], sv[k + 8]);
@@ -314,13 +316,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int c = 0; c < kBN / 32; ++c) {
                 if (c + 1 < kBN / 32) tc::ld_32col(lane_addr + s_col + (c + 1) * 32, buf[(c + 1) & 1]);
                 uint32_t r[16];
+                if (c * 32 >= a.Lk) {
+                    // no key of this chunk exists: P = 0 (uniform branch)
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) r[e] = 0u;
+                    tc::st_16col(lane_addr + s_col + c * 16, r);
+                    if (c + 1 < kBN / 32) tc::wait_ld();
+                    continue;
+                }
+                const bool tail = (c + 1) * 32 > a.Lk;  // uniform: the chunk holding the end of the keys
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int idx = c * 32 + 2 * e;
                     float s0 = __uint_as_float(buf[c & 1][2 * e]);
                     float s1 = __uint_as_float(buf[c & 1][2 * e + 1]);
-                    if (idx >= a.Lk) s0 = -INFINITY;
-                    if (idx + 1 >= a.Lk) s1 = -INFINITY;
+                    if (tail) {
+                        if (idx >= a.Lk) s0 = -INFINITY;
+                        if (idx + 1 >= a.Lk) s1 = -INFINITY;
+                    }
                     const tc::f32x2 t = tc::fma2(tc::pack2(s0, s1), scale2, negm2);
                     float t0, t1, p0, p1;
                     tc::unpack2(t, t0, t1);
@@ -355,15 +368,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc::named_bar_sync(1 + x, 128);
             const float inv = 1.f / l;
             unsigned char* stage = gen_base + (o_s - sbase) + x * kTile;
+            uint32_t ov[NO / 16][16];
+#pragma unroll
+            for (int c = 0; c < NO / 16; ++c) tc::ld_16col(lane_addr + o_col + c * 16, ov[c]);
+            tc::wait_ld();
 #pragma unroll
             for (int c = 0; c < NO / 16; ++c) {
-                uint32_t r[16];
-                tc::ld_16col(lane_addr + o_col + c * 16, r);
-                tc::wait_ld();
                 uint32_t w[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(r[2 * e]) * inv, __uint_as_float(r[2 * e + 1]) * inv);
+                    w[e] = pack_bf16x2(__uint_as_float(ov[c][2 * e]) * inv, __uint_as_float(ov[c][2 * e + 1]) * inv);
                 const int col = c * 16;
                 const int bx = col >> 6;
                 const int ch = (col & 63) >> 3;
