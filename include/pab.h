@@ -124,8 +124,9 @@ int pab_layout(int to_temporal, const void* src, void* dst, int T, int N, int C,
 /* *result (HOST pointer) = mean over n elements of (a - b)^2, accumulated in
  * fp64 in a fixed order (bitwise reproducible for a given n).  a and b hold n
  * elements of dtype (PAB_BF16 or PAB_FP32).  n == 0 gives 0.  Uses a
- * per-device scratch buffer of fp64 partial sums that the library allocates
- * on first use.  SYNCHRONISES cuda_stream before returning. */
+ * per-device scratch buffer (fp64 partial sums and a completion ticket) that
+ * the library allocates on first use.  SYNCHRONISES cuda_stream before
+ * returning. */
 int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype,
                       double* result, void* cuda_stream);
 
@@ -144,12 +145,12 @@ int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype
  * DEVICE pointer; no synchronisation), but the fp64 partial sums live in a
  * static device array of 4096 doubles (32 KiB) that every GPU loading the
  * library holds until exit; the call allocates nothing.  A call that would
- * need more than 4096 partial sums (only on devices with more than 1024 SMs)
+ * need more than 4095 partial sums (only on devices with more than 1023 SMs)
  * returns PAB_ERR_UNSUPPORTED.  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress) and caches it; make that
- * first call before any stream capture.  All calls share the array: calls
- * whose kernels overlap on the GPU race and must be serialised by the
- * caller. */
+ * array's device address (cudaGetSymbolAddress), caches it and clears the
+ * array's completion ticket on cuda_stream; make that first call before any
+ * stream capture.  All calls share the array: calls whose kernels overlap on
+ * the GPU race and must be serialised by the caller. */
 int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long n, int dtype,
                               double* result_dev, void* cuda_stream);
 

@@ -14,10 +14,12 @@ int device_sm_count();
 // Record `code` and a message as the calling thread's last error; returns code.
 int report_error(int code, const char* fmt, ...);
 
-// --- attention-difference MSE (two passes, fp64, deterministic) ----------
-// Number of first-pass partial sums used for n elements on this device.
+// --- attention-difference MSE (one launch, fp64, deterministic) ----------
+// Number of per-block partial sums used for n elements on this device.
 int mse_num_partials(long long n, int elem_size);
-cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, double* partials,
+// scratch: num_partials + 1 doubles; scratch[0] is the completion ticket
+// (zero before the call, zero again after it), the rest the partials.
+cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, double* scratch,
                        int num_partials, double* result_dev, cudaStream_t s);
 
 // --- layout change [T,N,C] <-> [N,T,C] (bulk-copy engine) ----------------

@@ -4,12 +4,15 @@
 // quantified by MSE).
 //
 // HBM-bound: each element is read once from each tensor (2 x size bytes).
-// Pass 1: a grid of (SM count x 4) blocks streams 16-byte vectors with a
+// One launch: a grid of (SM count x 4) blocks streams 16-byte vectors with a
 // grid-stride loop, accumulates (a - b)^2 in fp64 per thread, reduces each
 // warp with shuffles and each block through shared memory, and writes one
-// fp64 partial per block.  Pass 2: one block sums the partials in a fixed
-// order and divides by n.  The split depends only on n and the SM count, so
-// the result is bitwise reproducible on a given device.
+// fp64 partial per block.  The block that finishes last (a completion
+// ticket counted with an atomic add) sums the partials in a fixed order,
+// divides by n and returns the ticket to zero for the next call.  The split
+// depends only on n and the SM count, and the final sum's order does not
+// depend on which block finishes last, so the result is bitwise reproducible
+// on a given device.
 #include <mutex>
 
 #include "../../include/pab.h"
@@ -92,11 +95,12 @@ PAB_DEV double block_sum(double x, double* red) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) mse_partials_kernel(const T* __restrict__ a,
-                                                                const T* __restrict__ b,
-                                                                long long n,
-                                                                double* __restrict__ partials) {
+__global__ void __launch_bounds__(kThreads) mse_kernel(const T* __restrict__ a, const T* __restrict__ b,
+                                                       long long n, unsigned long long* __restrict__ ticket,
+                                                       double* __restrict__ partials,
+                                                       double* __restrict__ result) {
     __shared__ double red[kThreads / 32];
+    __shared__ bool last;
     constexpr int E = Vec<T>::kElems;
     const long long nvec = n / E;
     const uint4* va = reinterpret_cast<const uint4*>(a);
@@ -122,17 +126,22 @@ __global__ void __launch_bounds__(kThreads) mse_partials_kernel(const T* __restr
         if (t < n) acc += Vec<T>::sq_one(a, b, t);
     }
     const double s = block_sum(acc, red);
-    if (threadIdx.x == 0) partials[blockIdx.x] = s;
-}
-
-__global__ void __launch_bounds__(kThreads) mse_final_kernel(const double* __restrict__ partials,
-                                                             int count, long long n,
-                                                             double* __restrict__ result) {
-    __shared__ double red[kThreads / 32];
-    double acc = 0.0;
-    for (int i = threadIdx.x; i < count; i += blockDim.x) acc += partials[i];
-    const double s = block_sum(acc, red);
-    if (threadIdx.x == 0) *result = (n > 0) ? s / (double)n : 0.0;
+    if (threadIdx.x == 0) {
+        partials[blockIdx.x] = s;
+        __threadfence();  // the partial is visible before the ticket is taken
+        last = atomicAdd(ticket, 1ull) == (unsigned long long)gridDim.x - 1;
+    }
+    __syncthreads();
+    if (!last) return;
+    // the last block: every partial has been published
+    __threadfence();
+    double acc2 = 0.0;
+    for (int k = threadIdx.x; k < (int)gridDim.x; k += blockDim.x) acc2 += __ldcg(partials + k);
+    const double tot = block_sum(acc2, red);
+    if (threadIdx.x == 0) {
+        *result = (n > 0) ? tot / (double)n : 0.0;
+        *ticket = 0ull;  // ready for the next call on this scratch
+    }
 }
 
 }  // namespace
@@ -147,17 +156,18 @@ int mse_num_partials(long long n, int elem_size) {
     return (int)blocks;
 }
 
-cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, double* partials,
+cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, double* scratch,
                        int num_partials, double* result_dev, cudaStream_t s) {
+    unsigned long long* ticket = reinterpret_cast<unsigned long long*>(scratch);
+    double* partials = scratch + 1;
     if (dtype == 1)
-        mse_partials_kernel<float><<<num_partials, kThreads, 0, s>>>(
-            static_cast<const float*>(a), static_cast<const float*>(b), n, partials);
+        mse_kernel<float><<<num_partials, kThreads, 0, s>>>(static_cast<const float*>(a),
+                                                          static_cast<const float*>(b), n, ticket, partials,
+                                                          result_dev);
     else
-        mse_partials_kernel<__nv_bfloat16><<<num_partials, kThreads, 0, s>>>(
-            static_cast<const __nv_bfloat16*>(a), static_cast<const __nv_bfloat16*>(b), n, partials);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    mse_final_kernel<<<1, kThreads, 0, s>>>(partials, num_partials, n, result_dev);
+        mse_kernel<__nv_bfloat16><<<num_partials, kThreads, 0, s>>>(
+            static_cast<const __nv_bfloat16*>(a), static_cast<const __nv_bfloat16*>(b), n, ticket, partials,
+            result_dev);
     return cudaGetLastError();
 }
 
@@ -174,18 +184,22 @@ cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, dou
 // file-scope device array instead of the lazily allocated per-device buffer
 // that pab_attn_diff_mse / pab_attn_diff_mse_async use.
 //
-// The array holds kNoAllocMaxPartials doubles (32 KiB).  Every GPU that loads
-// this library keeps it until the process exits.  Every call shares it and
-// it keeps the last call's contents; nothing in it has to start at zero,
-// because each first-pass block overwrites its own slot and the second pass
-// reads only the slots this call wrote.  Calls whose kernels overlap on the
-// GPU (different streams, or different host threads on one device) race on
-// the array and must be serialised by the caller.
+// The array holds kNoAllocScratch doubles (32 KiB): slot 0 is the kernel's
+// completion ticket, the rest are partial sums (at most kNoAllocMaxPartials).
+// Every GPU that loads this library keeps it until the process exits.  Every
+// call shares it and it keeps the last call's contents.  Only the ticket must
+// start at zero: the first call on a device clears it (stream-ordered before
+// its kernel), and every call's last block returns it to zero.  The partial
+// slots need no clearing: each block overwrites its own slot and the final
+// sum reads only the slots this call wrote.  Calls whose kernels overlap on
+// the GPU (different streams, or different host threads on one device) race
+// on the array and must be serialised by the caller.
 // ===========================================================================
 namespace {
 
-constexpr int kNoAllocMaxPartials = 4096;
-static __device__ __align__(256) double g_mse_noalloc_scratch[kNoAllocMaxPartials];
+constexpr int kNoAllocScratch = 4096;
+constexpr int kNoAllocMaxPartials = kNoAllocScratch - 1;
+static __device__ __align__(256) double g_mse_noalloc_scratch[kNoAllocScratch];
 
 constexpr int kNoAllocMaxDevices = 64;
 std::mutex g_noalloc_mu;
@@ -194,8 +208,9 @@ double* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
 // Device address of the array on the current device.  Host code cannot use
 // the array's name as a device pointer (it names a host-side stand-in), so
 // the address is looked up once per device with cudaGetSymbolAddress while
-// that device is current, and cached.
-int noalloc_scratch(double** out) {
+// that device is current, and cached; that first call also clears the
+// completion ticket on `stream`.
+int noalloc_scratch(double** out, cudaStream_t stream) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
@@ -208,6 +223,10 @@ int noalloc_scratch(double** out) {
         e = cudaGetSymbolAddress(&p, g_mse_noalloc_scratch);
         if (e != cudaSuccess || !p)
             return pab::report_error(PAB_ERR_CUDA, "cudaGetSymbolAddress of the MSE scratch array: %s",
+                                     cudaGetErrorString(e));
+        e = cudaMemsetAsync(p, 0, sizeof(unsigned long long), stream);
+        if (e != cudaSuccess)
+            return pab::report_error(PAB_ERR_CUDA, "clearing the MSE completion ticket: %s",
                                      cudaGetErrorString(e));
         g_noalloc_ptr[dev] = static_cast<double*>(p);
     }
@@ -234,7 +253,7 @@ extern "C" int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long
                                  "this call needs %d partial sums; the static scratch array holds %d",
                                  parts, kNoAllocMaxPartials);
     double* scratch = nullptr;
-    const int rc = noalloc_scratch(&scratch);
+    const int rc = noalloc_scratch(&scratch, static_cast<cudaStream_t>(cuda_stream));
     if (rc != PAB_OK) return rc;
     const cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, result_dev,
                                           static_cast<cudaStream_t>(cuda_stream));

@@ -47,7 +47,9 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 constexpr int kMaxDevices = 64;
 
-// Per-device scratch for the MSE first pass: fp64 partials + one result slot.
+// Per-device scratch of the MSE kernel: a completion ticket, the fp64
+// partials and (for the synchronous call) one result slot.  The ticket is
+// cleared when the buffer is allocated and returned to zero by every call.
 struct MseScratch {
     double* buf = nullptr;
     int capacity = 0;  // doubles
@@ -62,7 +64,7 @@ int current_device(int* dev) {
     return PAB_OK;
 }
 
-int mse_scratch(int need, double** out) {
+int mse_scratch(int need, double** out, cudaStream_t stream) {
     int dev;
     int rc = current_device(&dev);
     if (rc) return rc;
@@ -74,6 +76,8 @@ int mse_scratch(int need, double** out) {
         s.capacity = 0;
         cudaError_t e = cudaMalloc(&s.buf, sizeof(double) * (size_t)need);
         if (e != cudaSuccess) return cuda_fail(e, "MSE scratch allocation");
+        e = cudaMemsetAsync(s.buf, 0, sizeof(unsigned long long), stream);  // the completion ticket
+        if (e != cudaSuccess) return cuda_fail(e, "MSE scratch clear");
         s.capacity = need;
     }
     *out = s.buf;
@@ -358,7 +362,7 @@ int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype
     const int elem = dtype == PAB_FP32 ? 4 : 2;
     const int parts = pab::mse_num_partials(n, elem);
     double* scratch = nullptr;
-    int rc = mse_scratch(parts + 1, &scratch);
+    int rc = mse_scratch(parts + 1, &scratch, static_cast<cudaStream_t>(cuda_stream));
     if (rc) return rc;
     cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, result_dev,
                                     static_cast<cudaStream_t>(cuda_stream));
@@ -377,12 +381,13 @@ int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype, doub
     const int elem = dtype == PAB_FP32 ? 4 : 2;
     const int parts = pab::mse_num_partials(n, elem);
     double* scratch = nullptr;
-    int rc = mse_scratch(parts + 1, &scratch);
-    if (rc) return rc;
     cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
-    cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, scratch + parts, s);
+    int rc = mse_scratch(parts + 2, &scratch, s);
+    if (rc) return rc;
+    double* result_dev = scratch + 1 + parts;
+    cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, result_dev, s);
     if (e != cudaSuccess) return cuda_fail(e, "MSE launch");
-    e = cudaMemcpyAsync(result, scratch + parts, sizeof(double), cudaMemcpyDeviceToHost, s);
+    e = cudaMemcpyAsync(result, result_dev, sizeof(double), cudaMemcpyDeviceToHost, s);
     if (e != cudaSuccess) return cuda_fail(e, "MSE result copy");
     e = cudaStreamSynchronize(s);
     if (e != cudaSuccess) return cuda_fail(e, "MSE stream synchronise");
