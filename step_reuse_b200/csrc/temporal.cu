@@ -7,7 +7,10 @@
 // (2 * T * d * 2 flop per loaded byte ~ 8-32 flop/B).
 //
 // Design:
-//  - persistent grid; a unit of work is (position n, group of G heads); one
+//  - persistent grid; a unit of work is (position n, group of G heads), G
+//    the smallest head count that gives each of the 8 warps a task when two
+//    such stages fit one CTA per SM (d = 128, T = 24: G = 4), else the largest
+//    that keeps two CTAs per SM (more warps hide the warp-MMA latency); one
 //    thread streams the unit's q, k, v into shared memory with TMA tensor
 //    loads (one [T rows][P cols] box per tensor and head), double-buffered
 //    across units so the next unit's loads overlap this unit's math, and
@@ -31,7 +34,8 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
-constexpr int kMaxStageBytes = 56 * 1024;
+constexpr int kMaxStageBytes = 56 * 1024;        // two CTAs per SM
+constexpr int kMaxStageBytesLarge = 110 * 1024;  // one CTA per SM
 constexpr float kLog2e = 1.4426950408889634f;
 
 __device__ unsigned int g_temporal_err = 0;
@@ -327,13 +331,25 @@ cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* o
     p.d = d;
     p.P = ((d / 8) & 1) ? d : d + 8;
     p.RT = (T + 15) / 16 * 16;
-    // largest divisor of heads whose stage fits the budget
-    int G = 1;
-    for (int g = heads; g >= 1; --g)
-        if (heads % g == 0 && 3 * g * p.RT * p.P * 2 <= kMaxStageBytes) {
+    // heads per unit: the smallest divisor of heads that gives every warp a
+    // (head, 16-row tile) task, if its stage fits the large budget (two
+    // stages per CTA, one CTA per SM); otherwise the largest divisor whose
+    // stage fits the small budget (two CTAs per SM)
+    int G = 0;
+    const int mt = p.RT / 16;
+    for (int g = 1; g <= heads; ++g)
+        if (heads % g == 0 && g * mt >= kWarps && 3 * g * p.RT * p.P * 2 <= kMaxStageBytesLarge) {
             G = g;
             break;
         }
+    if (G == 0) {
+        G = 1;
+        for (int g = heads; g >= 1; --g)
+            if (heads % g == 0 && 3 * g * p.RT * p.P * 2 <= kMaxStageBytes) {
+                G = g;
+                break;
+            }
+    }
     p.G = G;
     p.units = (long long)N * (heads / G);
     p.scale_log2 = kLog2e / sqrtf((float)d);
