@@ -7,24 +7,31 @@
 //
 // Persistent CTAs (one per SM) each own a contiguous run of (head, 128-row
 // query tile) work items and alternate them between two slots:
-//   warp 8 (one thread)      TMA producer: the current head's Kt / Vt
+//   warp 12 (one thread)     TMA producer: the current head's Kt / Vt
 //                            (reloaded when the head changes, once both
 //                            issuers' MMAs on the old ones have retired --
 //                            a barrier each issuer commits once per change,
-//                            so no wait is ever two phases behind) and the query
-//                            tiles through a ring of three Q buffers; a
-//                            buffer is refilled as soon as its S product has
-//                            retired, so loads run two to three tiles ahead;
-//   warps 9, 10 (one thread) tcgen05.mma issuers, one per slot: S = Q Kt^T
-//                            (SS form, fp32 in TMEM) and O = P Vt (TS form,
-//                            P from TMEM);
-//   warps 0-3 / 4-7          softmax and epilogue of slot 0 / 1: thread i
-//                            owns row i (TMEM lane i), masks keys past
-//                            text_len, exponentiates (MUFU ex2 with a share
-//                            on the FMA pipes), writes P as bf16 over S, then
-//                            normalises O, stages it (128-byte swizzle) in the
-//                            slot's output buffer and stores it with TMA.
+//                            so no wait is ever two phases behind), after
+//                            which it writes 1.0 into Vt's column d for every
+//                            key; and the query tiles through a ring of three
+//                            Q buffers, each refilled as soon as its S
+//                            product has retired;
+//   warps 13, 14             tcgen05.mma issuers, one warp per slot (one
+//                            elected lane issues): S = Q Kt^T (SS form, fp32
+//                            in TMEM) and O = P Vt (TS form, P from TMEM, N =
+//                            d plus the ones column); the slot's next S is
+//                            queued right behind each P Vt product;
+//   warps 0-3 / 4-7          softmax of slot 0 / 1: thread i owns row i (TMEM
+//                            lane i), masks keys past text_len, exponentiates
+//                            (MUFU ex2 with a share on the FMA pipes) and
+//                            writes P as bf16 over S;
+//   warps 8-11               epilogue of both slots, tiles in order: O's
+//                            column d is the row sum of P (the ones column),
+//                            so O / O[:, d] is normalised, staged (128-byte
+//                            swizzle) in the slot's output buffer and stored
+//                            with TMA while the softmax warps go on.
 // TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+NO), O_1 [384,384+NO).
+// Head dims up to 112 (column d must exist in O's 128 columns).
 // Every wait is bounded; on time-out the CTA raises the error word, drains
 // its copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -38,7 +45,7 @@ namespace {
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // text keys (one tile; text_len <= 128)
 constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
-constexpr int kThreads = 352;     // 2 softmax warpgroups + producer + 2 MMA warps
+constexpr int kThreads = 480;     // 2 softmax warpgroups + epilogue warpgroup + producer + 2 MMA warps
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPolyPairsOf8 = 3;  // share of exponentials on the FMA pipes
 constexpr float kC0 = 1.0f, kC1 = 0.693282962f, kC2 = 0.242210999f, kC3 = 0.0550089180f;
@@ -47,6 +54,7 @@ __device__ unsigned int g_cross_err = 0;
 
 struct CrossArgs {
     int Lk;            // text_len (<= 128)
+    int d;             // head dim (<= 112: column d of the PV product carries the row sums)
     int nqt;           // query tiles per head
     long long tiles;   // heads * nqt
     float scale_log2;  // log2(e) / sqrt(d)
@@ -55,8 +63,9 @@ struct CrossArgs {
 constexpr int kQBufs = 3;
 
 struct Bars {
-    unsigned long long kv_full;
-    unsigned long long kv_free;  // both issuers are done with the previous head's Kt / Vt
+    unsigned long long kv_full;   // Kt / Vt landed
+    unsigned long long kv_ready;  // ... and Vt's ones column written
+    unsigned long long kv_free;   // both issuers are done with the previous head's Kt / Vt
     unsigned long long q_full[kQBufs];
     unsigned long long q_free[kQBufs];  // the S product reading the buffer retired
     unsigned long long s_done[2];
@@ -107,13 +116,18 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
     return true;
 }
 
-template <int KSTEPS>
+PAB_DEV bool wait_bar_warp(Bars* b, unsigned long long* bar, uint32_t parity) {
+    return __all_sync(0xffffffffu, wait_bar(b, bar, parity));
+}
+
+template <int KSTEPS, int NO>
 __global__ void __launch_bounds__(kThreads, 1)
     cross_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                     CrossArgs a) {
-    constexpr int NB = (KSTEPS + 3) / 4;
-    constexpr int NO = KSTEPS * 16;
+    constexpr int NB = (KSTEPS + 3) / 4;  // 64-column boxes of Q, Kt and the output (d columns)
+    constexpr int NBV = (NO + 63) / 64;   // boxes of Vt: d columns + the ones column
+    static_assert(NO <= 128, "O of a slot lives in 128 TMEM columns");
     constexpr uint32_t kTile = NB * kBox;
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -122,7 +136,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t q_s = sbase;                 // [kQBufs][NB boxes]
     const uint32_t o_s = q_s + kQBufs * kTile;  // [2 slots][NB boxes]: output staging
     const uint32_t k_s = o_s + 2 * kTile;       // [NB boxes]
-    const uint32_t v_s = k_s + kTile;           // [NB boxes]
+    const uint32_t v_s = k_s + kTile;           // [NBV boxes]
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -134,8 +148,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t_end = t_begin + per < tiles ? t_begin + per : tiles;
     const int n = t_begin < t_end ? t_end - t_begin : 0;
 
-    if (threadIdx.x == 256) {
+    if (threadIdx.x == 384) {
         mbar_init(smem_u32(&bars.kv_full), 1);
+        mbar_init(smem_u32(&bars.kv_ready), 1);
         mbar_init(smem_u32(&bars.kv_free), 2);
         for (int b = 0; b < kQBufs; ++b) {
             mbar_init(smem_u32(&bars.q_full[b]), 1);
@@ -155,7 +170,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::prefetch_tmap(&tm_v);
         tc::prefetch_tmap(&tm_o);
     }
-    if (warp == 9) {
+    if (warp == 13) {
         tc::tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -164,29 +179,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     const uint32_t tmem = bars.tmem_base;
 
-    if (warp == 8) {
+    if (warp == 12) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             int cur_h = -1, heads_loaded = 0, nq = 0;
             bool ok = true;
+            // Kt / Vt of the latest head are in flight and Vt's ones column is
+            // not written yet; finished before the producer blocks on anything
+            // the issuers release (they need kv_ready first)
+            bool pending = false;
+            auto finish_kv = [&]() -> bool {
+                if (!pending) return true;
+                if (!wait_bar(&bars, &bars.kv_full, (heads_loaded - 1) & 1)) return false;
+                // column d of Vt (zero-filled past the head) becomes all ones, so the
+                // P Vt product also delivers the row sums of P in O's column d
+                const uint32_t col = (uint32_t)a.d;
+                unsigned char* vbox = gen_base + (v_s - sbase) + (col >> 6) * kBox;
+                const uint32_t ch = (col & 63) >> 3, e = col & 7;
+                for (int r = 0; r < kBN; ++r)
+                    *reinterpret_cast<uint16_t*>(vbox + r * 128 + ((ch ^ (r & 7)) << 4) + e * 2) = 0x3F80u;
+                fence_proxy_async_smem();
+                mbar_arrive(smem_u32(&bars.kv_ready));
+                pending = false;
+                return true;
+            };
             for (int i = 0; i < n && ok; ++i) {
                 const int t = t_begin + i;
                 const int h = t / a.nqt, qt = t - h * a.nqt;
                 if (h != cur_h) {
                     // every MMA of the earlier tiles has retired before Kt / Vt change:
                     // each issuer commits kv_free once per head change
-                    if (heads_loaded > 0) ok = wait_bar(&bars, &bars.kv_free, (heads_loaded - 1) & 1);
+                    ok = finish_kv();
+                    if (ok && heads_loaded > 0) ok = wait_bar(&bars, &bars.kv_free, (heads_loaded - 1) & 1);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(smem_u32(&bars.kv_full), 2 * kTile);
-                    for (int bx = 0; bx < NB; ++bx) {
+                    mbar_arrive_expect_tx(smem_u32(&bars.kv_full), (NB + NBV) * kBox);
+                    for (int bx = 0; bx < NB; ++bx)
                         tc::tma_load_4d(k_s + bx * kBox, &tm_k, bx * 64, h, 0, 0, smem_u32(&bars.kv_full));
+                    for (int bx = 0; bx < NBV; ++bx)
                         tc::tma_load_4d(v_s + bx * kBox, &tm_v, bx * 64, h, 0, 0, smem_u32(&bars.kv_full));
-                    }
-                    cur_h = h;
                     ++heads_loaded;
+                    pending = true;
+                    cur_h = h;
                 }
                 const int b = i % kQBufs;
-                if (i >= kQBufs) ok = wait_bar(&bars, &bars.q_free[b], ((i / kQBufs) - 1) & 1);
+                if (i >= kQBufs) {
+                    ok = finish_kv();
+                    if (ok) ok = wait_bar(&bars, &bars.q_free[b], ((i / kQBufs) - 1) & 1);
+                }
                 if (!ok) break;
                 mbar_arrive_expect_tx(smem_u32(&bars.q_full[b]), kTile);
                 for (int bx = 0; bx < NB; ++bx)
@@ -194,6 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                     smem_u32(&bars.q_full[b]));
                 nq = i + 1;
             }
+            if (ok) ok = finish_kv();
             if (!ok || *(volatile int*)&bars.abort) {
                 // drain: every load issued lands before the CTA exits (bounded)
                 for (int i = (nq > kQBufs ? nq - kQBufs : 0); i < nq; ++i)
@@ -202,64 +242,81 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait_bounded(smem_u32(&bars.kv_full), (heads_loaded - 1) & 1, &g_cross_err);
             }
         }
-    } else if (warp == 9 || warp == 10) {
+    } else if (warp == 13 || warp == 14) {
         // ------------------------------------------------ MMA issuers (slot x: tiles i = x, x+2, ...)
-        const int x = warp - 9;
-        if (lane == 0) {
+        const int x = warp - 13;
+        {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
             const uint64_t dq = tc::smem_desc(q_s, 16, 1024, 2);
             const uint64_t dk = tc::smem_desc(k_s, 16, 1024, 2);
             const uint64_t dv = tc::smem_desc(v_s, kBox, 1024, 2);
             const uint32_t s_t = tmem + x * 128, o_t = tmem + 256 + x * 128;
-            int heads_seen = 0;
-            int hcur = -1;
-            bool ok = true;
-            for (int i = 0; i < n && ok; ++i) {
-                // follow every Kt / Vt reload in order (also those at the other
-                // slot's tiles), so a wait is never two phases behind
-                const int h = (t_begin + i) / a.nqt;
-                if (h != hcur) {
-                    // release the old head's Kt / Vt once this issuer's MMAs on them
-                    // retire, then wait for the new ones
-                    if (heads_seen > 0) tc::commit(smem_u32(&bars.kv_free));
-                    hcur = h;
-                    ++heads_seen;
-                    ok = wait_bar(&bars, &bars.kv_full, (heads_seen - 1) & 1);
-                    if (!ok) break;
+            // Kt / Vt reloads are followed in tile order (the other slot's tiles
+            // included), so a wait on kv_ready is never two phases behind
+            int heads_seen = 0, hcur = -1, next_t = 0;
+            auto advance_heads = [&](int upto) -> bool {
+                for (; next_t <= upto; ++next_t) {
+                    const int h = (t_begin + next_t) / a.nqt;
+                    if (h != hcur) {
+                        // release the old head's Kt / Vt once this issuer's MMAs on
+                        // them retire, then wait for the new ones (ones column written)
+                        if (heads_seen > 0) tc::commit_warp(smem_u32(&bars.kv_free));
+                        hcur = h;
+                        ++heads_seen;
+                        if (!wait_bar_warp(&bars, &bars.kv_ready, (heads_seen - 1) & 1)) return false;
+                    }
                 }
-                if ((i & 1) != x) continue;
+                return true;
+            };
+            // S(i) = Q(i) Kt^T into this slot's S columns
+            auto issue_s = [&](int i) -> bool {
                 const int qb = i % kQBufs;
-                if (ok) ok = wait_bar(&bars, &bars.q_full[qb], (i / kQBufs) & 1);
-                if (!ok) break;
+                if (!wait_bar_warp(&bars, &bars.q_full[qb], (i / kQBufs) & 1)) return false;
                 tc::fence_after_sync();
                 const uint64_t a0 = dq + (uint64_t)((qb * kTile) >> 4);
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const uint32_t off = (ks >> 2) * (kBox >> 4) + (ks & 3) * 2;
-                    tc::mma_ss(s_t, a0 + off, dk + off, idesc_s, ks > 0 ? 1u : 0u);
+                    tc::mma_ss_warp(s_t, a0 + off, dk + off, idesc_s, ks > 0 ? 1u : 0u);
                 }
-                tc::commit(smem_u32(&bars.s_done[x]));
-                tc::commit(smem_u32(&bars.q_free[qb]));  // the Q buffer may be refilled
-                // O_X is free once the previous tile of this slot was read out
-                if (i >= 2) ok = wait_bar(&bars, &bars.o_free[x], ((i - 2) >> 1) & 1);
-                if (ok) ok = wait_bar(&bars, &bars.p_full[x], (i >> 1) & 1);
+                tc::commit_warp(smem_u32(&bars.s_done[x]));
+                tc::commit_warp(smem_u32(&bars.q_free[qb]));  // the Q buffer may be refilled
+                return true;
+            };
+            bool ok = true;
+            if (x < n) {
+                ok = advance_heads(x);
+                if (ok) ok = issue_s(x);
+            }
+            for (int i = x; i < n && ok; i += 2) {
+                // O_X is free once the epilogue has read out the previous tile of this slot
+                if (i >= 2) ok = wait_bar_warp(&bars, &bars.o_free[x], ((i - 2) >> 1) & 1);
+                if (ok) ok = wait_bar_warp(&bars, &bars.p_full[x], (i >> 1) & 1);
                 if (!ok) break;
                 tc::fence_after_sync();
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    tc::mma_ts(o_t, s_t + kk * 8, dv + kk * 128, idesc_o, kk > 0 ? 1u : 0u);
-                tc::commit(smem_u32(&bars.o_full[x]));
+                    tc::mma_ts_warp(o_t, s_t + kk * 8, dv + kk * 128, idesc_o, kk > 0 ? 1u : 0u);
+                tc::commit_warp(smem_u32(&bars.o_full[x]));
+                // the slot's next S, queued right behind this P Vt product (which
+                // reads P from the columns S overwrites: in-order execution)
+                if (i + 2 < n) {
+                    ok = advance_heads(i + 2);
+                    if (ok) ok = issue_s(i + 2);
+                }
             }
-            tc::commit(smem_u32(&bars.mma_done[x]));
+            // the head changes past this slot's last tile: the producer counts on
+            // both issuers' releases at every change
+            if (ok && n > 0) ok = advance_heads(n - 1);
+            tc::commit_warp(smem_u32(&bars.mma_done[x]));
             mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_cross_err);
         }
-    } else {
-        // ------------------------------------------------ softmax + epilogue (slot x)
+    } else if (warp < 8) {
+        // ------------------------------------------------ softmax (slot x)
         const int x = warp >> 2;
-        const int row = (warp & 3) * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t s_col = x * 128, o_col = 256 + x * 128;
+        const uint32_t s_col = x * 128;
         const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
         bool ok = true;
         for (int i = x; i < n && ok; i += 2) {
@@ -303,12 +360,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                  fmaxf(mx[6], mx[7])) * a.scale_log2;
             }
             // pass 2: S again, 32 columns at a time (next chunk's load in
-            // flight), exponentiated, summed, written back as bf16 P over the
-            // columns already consumed
+            // flight), exponentiated and written back as bf16 P over the
+            // columns already consumed (the row sums come out of the P Vt product)
             const tc::f32x2 negm2 = tc::pack2(-mrow, -mrow);
-            tc::f32x2 acc[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = tc::pack2(0.f, 0.f);
             uint32_t buf[2][32];
             tc::ld_32col(lane_addr + s_col, buf[0]);
             tc::wait_ld();
@@ -343,54 +397,65 @@ __global__ void __launch_bounds__(kThreads, 1)
                         p0 = ex2(t0);
                         p1 = ex2(t1);
                     }
-                    acc[e & 3] = tc::add2(acc[e & 3], tc::pack2(p0, p1));
                     r[e] = pack_bf16x2(p0, p1);
                 }
                 tc::st_16col(lane_addr + s_col + c * 16, r);
                 if (c + 1 < kBN / 32) tc::wait_ld();
             }
-            float l;
-            {
-                float a0, a1;
-                tc::unpack2(tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3])), a0, a1);
-                l = a0 + a1;
-            }
             tc::wait_st();
             tc::fence_before_sync();
             mbar_arrive(smem_u32(&bars.p_full[x]));
-
-            // ---------------- epilogue: O / l -> bf16 -> tile's Q buffer -> TMA store
-            ok = wait_bar(&bars, &bars.o_full[x], (i >> 1) & 1);
-            if (!ok) break;
-            tc::fence_after_sync();
-            // the slot's output buffer: tile i-2's store must have read it
-            if (row == 0) bulk_wait_read<0>();
-            tc::named_bar_sync(1 + x, 128);
-            const float inv = 1.f / l;
-            unsigned char* stage = gen_base + (o_s - sbase) + x * kTile;
-            uint32_t ov[NO / 16][16];
+        }
+    } else if (warp < 12) {
+        // ------------------------------------------------ epilogue (both slots, tiles in order)
+        // Every thread runs all n iterations and both named barriers of each,
+        // also after a wait gave up (then the work is skipped), so the barrier
+        // counts always match.
+        const int row = (warp & 3) * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+        constexpr int NC = NO / 16 < NB * 4 ? NO / 16 : NB * 4;  // 16-column chunks staged
+        bool ok = true;
+        for (int i = 0; i < n; ++i) {
+            const int x = i & 1;
+            const uint32_t o_col = 256 + x * 128;
+            if (ok) ok = wait_bar(&bars, &bars.o_full[x], (i >> 1) & 1);
+            uint32_t ov[NC][16];
+            float inv = 0.f;
+            if (ok) {
+                tc::fence_after_sync();
 #pragma unroll
-            for (int c = 0; c < NO / 16; ++c) tc::ld_16col(lane_addr + o_col + c * 16, ov[c]);
-            tc::wait_ld();
-#pragma unroll
-            for (int c = 0; c < NO / 16; ++c) {
-                uint32_t w[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    w[e] = pack_bf16x2(__uint_as_float(ov[c][2 * e]) * inv, __uint_as_float(ov[c][2 * e + 1]) * inv);
-                const int col = c * 16;
-                const int bx = col >> 6;
-                const int ch = (col & 63) >> 3;
-                unsigned char* rowp = stage + bx * kBox + row * 128;
-                *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
-                    make_uint4(w[4], w[5], w[6], w[7]);
+                for (int c = 0; c < NC; ++c) tc::ld_16col(lane_addr + o_col + c * 16, ov[c]);
+                uint32_t lbits;  // O's column d: the row sum of P (ones column of Vt)
+                tc::ld_1col(lane_addr + o_col + (uint32_t)a.d, lbits);
+                tc::wait_ld();
+                tc::fence_before_sync();
+                mbar_arrive(smem_u32(&bars.o_free[x]));  // O_X has been read out
+                inv = 1.f / __uint_as_float(lbits);
             }
-            tc::fence_before_sync();
-            mbar_arrive(smem_u32(&bars.o_free[x]));  // O_X has been read out
-            fence_proxy_async_smem();
-            tc::named_bar_sync(1 + x, 128);
-            if (row == 0) {
+            // the slot's staging buffer: the store of tile i-2 must have read it
+            if (row == 0) bulk_wait_read<1>();
+            tc::named_bar_sync(1, 128);
+            if (ok) {
+                unsigned char* stage = gen_base + (o_s - sbase) + x * kTile;
+#pragma unroll
+                for (int c = 0; c < NC; ++c) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        w[e] = pack_bf16x2(__uint_as_float(ov[c][2 * e]) * inv,
+                                           __uint_as_float(ov[c][2 * e + 1]) * inv);
+                    const int col = c * 16;
+                    const int bx = col >> 6;
+                    const int ch = (col & 63) >> 3;
+                    unsigned char* rowp = stage + bx * kBox + row * 128;
+                    *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
+                        make_uint4(w[4], w[5], w[6], w[7]);
+                }
+                fence_proxy_async_smem();
+            }
+            tc::named_bar_sync(1, 128);
+            if (ok && row == 0) {
                 const int t = t_begin + i;
                 const int h = t / a.nqt, qt = t - h * a.nqt;
                 for (int bx = 0; bx < NB; ++bx)
@@ -402,7 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == 13) {
         __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
@@ -436,17 +501,20 @@ bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KSTEPS>
+// NO = N of the P Vt product: d rounded up to 16, plus 16 when d is a
+// multiple of 16, so that column d (the ones column) exists
+template <int KSTEPS, int NO>
 cudaError_t launch_ks(const CUtensorMap* m, const CrossArgs& a, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
-    const size_t smem = (size_t)(kQBufs + 4) * NB * kBox + 1024;
+    constexpr int NBV = (NO + 63) / 64;
+    const size_t smem = (size_t)((kQBufs + 3) * NB + NBV) * kBox + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(cross_tc_kernel<KSTEPS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(cross_tc_kernel<KSTEPS, NO>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_req);
     if (e != cudaSuccess) return e;
     long long grid = device_sm_count();
     if (grid > a.tiles) grid = a.tiles;
-    cross_tc_kernel<KSTEPS><<<(unsigned)grid, kThreads, smem_req, s>>>(m[0], m[1], m[2], m[3], a);
+    cross_tc_kernel<KSTEPS, NO><<<(unsigned)grid, kThreads, smem_req, s>>>(m[0], m[1], m[2], m[3], a);
     return cudaGetLastError();
 }
 
@@ -455,9 +523,12 @@ cudaError_t launch_ks(const CUtensorMap* m, const CrossArgs& a, cudaStream_t s) 
 cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,
                          int d, cudaStream_t s) {
     if (R == 0) return cudaSuccess;
-    if (Lk > kBN) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s);
+    // longer texts, and head dims whose P Vt product has no column to spare
+    // for the row sums, take the general flash kernel
+    if (Lk > kBN || d > 112) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s);
     CrossArgs a;
     a.Lk = Lk;
+    a.d = d;
     const long long nqt = (R + kBM - 1) / kBM;
     if (nqt * heads >= (1LL << 31)) return cudaErrorInvalidValue;
     a.nqt = (int)nqt;
@@ -467,15 +538,15 @@ cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* ou
     if (!make_map(&m[0], q, d, heads, R) || !make_map(&m[1], kt, d, heads, Lk) ||
         !make_map(&m[2], vt, d, heads, Lk) || !make_map(&m[3], out, d, heads, R))
         return cudaErrorInvalidValue;
+    const bool extra = d % 16 == 0;  // no padding column inside ceil16(d): one more 16-column chunk
     switch ((d + 15) / 16) {
-        case 1: return launch_ks<1>(m, a, s);
-        case 2: return launch_ks<2>(m, a, s);
-        case 3: return launch_ks<3>(m, a, s);
-        case 4: return launch_ks<4>(m, a, s);
-        case 5: return launch_ks<5>(m, a, s);
-        case 6: return launch_ks<6>(m, a, s);
-        case 7: return launch_ks<7>(m, a, s);
-        case 8: return launch_ks<8>(m, a, s);
+        case 1: return extra ? launch_ks<1, 32>(m, a, s) : launch_ks<1, 16>(m, a, s);
+        case 2: return extra ? launch_ks<2, 48>(m, a, s) : launch_ks<2, 32>(m, a, s);
+        case 3: return extra ? launch_ks<3, 64>(m, a, s) : launch_ks<3, 48>(m, a, s);
+        case 4: return extra ? launch_ks<4, 80>(m, a, s) : launch_ks<4, 64>(m, a, s);
+        case 5: return extra ? launch_ks<5, 96>(m, a, s) : launch_ks<5, 80>(m, a, s);
+        case 6: return extra ? launch_ks<6, 112>(m, a, s) : launch_ks<6, 96>(m, a, s);
+        case 7: return extra ? launch_ks<7, 128>(m, a, s) : launch_ks<7, 112>(m, a, s);
         default: return cudaErrorInvalidValue;
     }
 }
