@@ -41,12 +41,12 @@ import synth  # noqa: E402
 METRIC = "attention TFLOP/s & steps/s per DiT attn stack; % of bf16 TC / HBM roofline"
 UNIT = "TFLOP/s (dense-equivalent attention)"
 
-# Per-launch DRAM bytes (read + write) measured by ncu for the dominant kernel
-# on the 480p-like workload, keyed by the sha256 of the kernel's source; a
-# different source hash means the counters are stale and traffic is null.
+# Per-launch DRAM bytes (read + write) measured by ncu for the dominant kernel,
+# keyed by (sha256 of the kernel's source, workload); a different source hash
+# or a workload without a capture means traffic is null.
 MEASURED_TRAFFIC = {
     # flash_tc spatial, 480p-like, 1 launch: dram read 175.91 MB + write 42.61 MB
-    "ddc0e33765e69db2": 218520064,
+    ("ddc0e33765e69db2", "480p"): 218520064,
 }
 
 
@@ -462,7 +462,7 @@ def run_ours(args):
     sp_ms = kms["spatial"]
     achieved = flops["spatial"] / (sp_ms * 1e-3) / 1e12
     src_hash = kernel_source_hash("flash_tc.cu")
-    traffic = MEASURED_TRAFFIC.get(src_hash)
+    traffic = MEASURED_TRAFFIC.get((src_hash, args.workload))
     roofline = {"kernel": "spatial flash attention (flash_tc)", "bound": "tensor", "achieved": achieved,
                 "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak, "traffic": traffic,
                 "peak_source": f"{peak_src} bf16_tflops_sustained",
