@@ -57,7 +57,7 @@ constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
 constexpr int kBN = 64;           // keys per K/V tile
 constexpr int kQBox = 128 * 128;  // bytes of one [128 rows][64 cols] bf16 box (Q, O)
 constexpr int kKVBox = 64 * 128;  // bytes of one [64 rows][64 cols] bf16 box (K, V)
-constexpr int kThreads = 352;     // 2 softmax warpgroups + producer warp + 2 MMA warps
+constexpr int kThreads = 384;     // 2 softmax warpgroups + producer warp + 2 MMA warps + V-ones warp
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 // Exponentials: of every 8 consecutive pairs of a row's scores, this many go
@@ -67,6 +67,9 @@ constexpr float kRescaleLog2 = 8.0f;
 #define PAB_POLY_PAIRS_OF_8 3
 #endif
 constexpr int kPolyPairsOf8 = PAB_POLY_PAIRS_OF_8;
+#ifndef PAB_FLASH_ONES
+#define PAB_FLASH_ONES 1
+#endif
 // 2^f ~ kP0 + kP1 f + kP2 f^2 + kP3 f^3 on [-0.5, 0.5] (see exp2_poly2)
 constexpr float kP0 = 1.0f, kP1 = 0.693282962f, kP2 = 0.242210999f, kP3 = 0.0550089180f;
 
@@ -76,6 +79,7 @@ struct FlashTcArgs {
     int Lq;            // query rows per batch
     int Lk;            // keys per batch
     int kv_batched;    // 1: K/V have a batch coordinate (spatial); 0: shared (cross)
+    int d;             // head dim
     float scale_log2;  // log2(e) / sqrt(d)
 };
 
@@ -92,6 +96,7 @@ struct Bars {
     unsigned long long k01_full;               // K_0, K_1 (own buffer)
     unsigned long long s01_done;               // S_X(0), S_X(1) of every tile retired
     unsigned long long slot_full[kMaxStages];  // V_j (+ K_{j+2}) landed
+    unsigned long long slot_ready[kMaxStages]; // ... and (ONES) V_j's column d set to 1
     unsigned long long slot_done[kMaxStages];  // one arrival per tile issuer
     unsigned long long p_full[2][2];           // [tile][S buffer]
     unsigned long long o_done[2];              // the last PV_X retired
@@ -144,7 +149,11 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
     return true;
 }
 
-template <int KSTEPS, int NST>
+// ONES (head dims with d % 16 != 0): column d of every V tile -- a padding
+// column inside the PV product's N = 16 * KSTEPS -- is set to 1 once the tile
+// lands (warp 11), so O's column d accumulates the row sum of P with the same
+// bf16 P as the numerator; the softmax then keeps no running sum.
+template <int KSTEPS, int NST, bool ONES>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -180,6 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(smem_u32(&bars.s01_done), ntiles);
         for (int st = 0; st < NST; ++st) {
             mbar_init(smem_u32(&bars.slot_full[st]), 1);
+            mbar_init(smem_u32(&bars.slot_ready[st]), 1);
             mbar_init(smem_u32(&bars.slot_done[st]), ntiles);
         }
         bars.abort = 0;
@@ -279,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             for (int j = 0; j < nkv && ok; ++j) {
                 const int st = j % NST;
-                ok = wait_bar(&bars, &bars.slot_full[st], (j / NST) & 1);
+                ok = wait_bar(&bars, ONES ? &bars.slot_ready[st] : &bars.slot_full[st], (j / NST) & 1);
                 if (ok) ok = wait_bar(&bars, &bars.p_full[x][j & 1], (j >> 1) & 1);
                 if (!ok) break;
                 tc::fence_after_sync();
@@ -297,6 +307,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             // all MMAs this thread issued complete before TMEM is released
             tc::commit(smem_u32(&bars.mma_done[x]));
             mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_flash_err);
+        }
+    } else if (warp == 11) {
+        // ------------------------------------------------ V-ones warp
+        if constexpr (ONES) {
+            const uint32_t col = (uint32_t)a.d;
+            const uint32_t ch = (col & 63) >> 3, e = col & 7;
+            bool ok = true;
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int st = j % NST;
+                ok = __all_sync(0xffffffffu, wait_bar(&bars, &bars.slot_full[st], (j / NST) & 1));
+                if (!ok) break;
+                unsigned char* vbox = gen_base + (v_s - sbase) + st * kKVTile + (col >> 6) * kKVBox;
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int r = lane + 32 * h2;
+                    *reinterpret_cast<uint16_t*>(vbox + r * 128 + ((ch ^ (r & 7)) << 4) + e * 2) = 0x3F80u;
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars.slot_ready[st]));
+            }
         }
     } else {
         // ------------------------------------------------ softmax warpgroups
@@ -370,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
                         tc::st_16col(lane_addr + o_col + c * 16, r);
                     }
-                    l *= f;
+                    if constexpr (!ONES) l *= f;
                     m_ref = m_new;
                 }
             }
@@ -395,12 +426,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         p0 = ex2(t0);
                         p1 = ex2(t1);
                     }
-                    acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
+                    if constexpr (!ONES) acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
                     r[i] = pack_bf16x2(p0, p1);
                 }
                 tc::st_16col(lane_addr + s_col + c * 16, r);
             }
-            {
+            if constexpr (!ONES) {
                 float a0, a1;
                 tc::unpack2(tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3])), a0, a1);
                 l += a0 + a1;
@@ -413,6 +444,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ok && nkv > 0) ok = wait_bar(&bars, &bars.o_done[x], 0);
         if (ok) {
             tc::fence_after_sync();
+            if constexpr (ONES) {  // O's column d: the row sum of P
+                uint32_t lbits;
+                tc::ld_1col(lane_addr + o_col + (uint32_t)a.d, lbits);
+                tc::wait_ld();
+                l = __uint_as_float(lbits);
+            }
             const float inv = 1.f / l;
             unsigned char* stage = gen_base + x * kQTile;  // this tile's Q buffer (all S MMAs done)
 #pragma unroll
@@ -485,18 +522,25 @@ bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows
     return r == CUDA_SUCCESS;
 }
 
-template <int KSTEPS>
-cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
-                      const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
+template <int KSTEPS, bool ONES>
+cudaError_t launch_ks1(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
     constexpr int NST = NB == 1 ? 6 : 4;  // ring slots of (V_j, K_{j+2})
     const size_t smem = (size_t)NB * (2 * kQBox + (2 + 2 * NST) * kKVBox) + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST>,
+    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST, ONES>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
     if (e != cudaSuccess) return e;
-    flash_tc_kernel<KSTEPS, NST><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    flash_tc_kernel<KSTEPS, NST, ONES><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
+}
+template <int KSTEPS>
+cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                      const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
+    // a padding column inside the PV product carries the row sums when d % 16 != 0
+    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true>(mq, mk, mv, mo, a, grid, s);
+    return launch_ks1<KSTEPS, false>(mq, mk, mv, mo, a, grid, s);
 }
 
 }  // namespace
@@ -519,6 +563,7 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
     a.Lq = (int)Lq;
     a.Lk = Lk;
     a.kv_batched = kv_bstride > 0 ? 1 : 0;
+    a.d = d;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
     dim3 grid((unsigned)qblocks, (unsigned)heads, (unsigned)batches);
     switch ((d + 15) / 16) {
