@@ -85,19 +85,24 @@ struct FlashTcArgs {
 
 constexpr int kMaxStages = 8;
 
-// A tcgen05.commit costs the tensor pipe about as much as two small MMAs, so
-// the pipeline is built around ONE commit per tile and K/V step: slot s of the
-// ring holds V_j and K_{j+2} (j = s mod NST); after issuing PV_X(j) and
-// S_X(j+2) each tile's issuer commits slot_done[s] once.  Its completion frees
-// the slot for the producer, tells the softmax that S_X(j+2) is in TMEM and
-// proves PV_X(j) retired (in-order completion).
+// The pipeline is built around ONE commit per tile and K/V step: slot s of
+// the ring holds V_j and K_{j+2} (j = s mod NST); after issuing PV_X(j) and
+// S_X(j+2) tile X's issuer commits slot_done[s][X] once.  Its completion
+// tells tile X's softmax that S_X(j+2) is in TMEM and proves PV_X(j) retired
+// (in-order completion); the producer refills the slot once both tiles'
+// barriers of the slot completed.  The tiles never wait on each other's
+// MMAs, and tile B's softmax starts only once tile A's first row maximum is
+// done: the two tiles' score reads and maxima then fall into each other's
+// exponential phases instead of coinciding (measured 5-10% faster at
+// d = 64-72; the offset fades over a long key loop).
 struct Bars {
     unsigned long long q_full[2];
     unsigned long long k01_full;               // K_0, K_1 (own buffer)
-    unsigned long long s01_done;               // S_X(0), S_X(1) of every tile retired
+    unsigned long long s01_done[2];            // [tile]: S_X(0), S_X(1) retired
+    unsigned long long b_go;                   // tile A's step-0 maximum is done
     unsigned long long slot_full[kMaxStages];  // V_j (+ K_{j+2}) landed
     unsigned long long slot_ready[kMaxStages]; // ... and (ONES) V_j's column d set to 1
-    unsigned long long slot_done[kMaxStages];  // one arrival per tile issuer
+    unsigned long long slot_done[kMaxStages][2];  // [slot][tile]: PV_X(j), S_X(j+2) retired
     unsigned long long p_full[2][2];           // [tile][S buffer]
     unsigned long long o_done[2];              // the last PV_X retired
     unsigned long long mma_done[2];
@@ -186,11 +191,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&bars.mma_done[x]), 1);
         }
         mbar_init(smem_u32(&bars.k01_full), 1);
-        mbar_init(smem_u32(&bars.s01_done), ntiles);
+        for (int x = 0; x < 2; ++x) mbar_init(smem_u32(&bars.s01_done[x]), 1);
+        mbar_init(smem_u32(&bars.b_go), 128);
         for (int st = 0; st < NST; ++st) {
             mbar_init(smem_u32(&bars.slot_full[st]), 1);
             mbar_init(smem_u32(&bars.slot_ready[st]), 1);
-            mbar_init(smem_u32(&bars.slot_done[st]), ntiles);
+            for (int x = 0; x < 2; ++x) mbar_init(smem_u32(&bars.slot_done[st][x]), 1);
         }
         bars.abort = 0;
         fence_mbar_init();
@@ -230,7 +236,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             bool ok = true;
             for (int j = 0; j < nkv && ok; ++j) {
                 const int st = j % NST;
-                if (j >= NST) ok = wait_bar(&bars, &bars.slot_done[st], ((j / NST) - 1) & 1);
+                for (int x = 0; x < ntiles && ok && j >= NST; ++x)
+                    ok = wait_bar(&bars, &bars.slot_done[st][x], ((j / NST) - 1) & 1);
                 if (!ok) break;
                 const bool with_k = j + 2 < nkv;
                 const uint32_t bar = smem_u32(&bars.slot_full[st]);
@@ -285,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc::fence_after_sync();
                 issue_s(dk01, 0);
                 if (nkv > 1) issue_s(dk01 + (kKVTile >> 4), 1);
-                tc::commit(smem_u32(&bars.s01_done));
+                tc::commit(smem_u32(&bars.s01_done[x]));
             }
             for (int j = 0; j < nkv && ok; ++j) {
                 const int st = j % NST;
@@ -301,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc::mma_ts(d, pa + kk * 8, vdesc + kk * 128, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
                 // S_X(j+2) reuses the buffer PV_X(j) has just been queued on
                 if (j + 2 < nkv) issue_s(dk + (uint64_t)((st * kKVTile) >> 4), j + 2);
-                tc::commit(smem_u32(&bars.slot_done[st]));
+                tc::commit(smem_u32(&bars.slot_done[st][x]));
                 if (j + 1 == nkv) tc::commit(smem_u32(&bars.o_done[x]));
             }
             // all MMAs this thread issued complete before TMEM is released
@@ -337,13 +344,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t o_col = 256 + x * 128;
         float m_ref = -INFINITY, l = 0.f;
         bool ok = x < ntiles;
+        if (ok && x == 1 && nkv > 0) ok = wait_bar(&bars, &bars.b_go, 0);
         for (int j = 0; j < nkv && ok; ++j) {
             const uint32_t s_col = x * 128 + (j & 1) * 64;
             // S_X(j) was issued with step j-2's slot (or in the prologue)
             if (j < 2)
-                ok = wait_bar(&bars, &bars.s01_done, 0);
+                ok = wait_bar(&bars, &bars.s01_done[x], 0);
             else
-                ok = wait_bar(&bars, &bars.slot_done[(j - 2) % NST], ((j - 2) / NST) & 1);
+                ok = wait_bar(&bars, &bars.slot_done[(j - 2) % NST][x], ((j - 2) / NST) & 1);
             if (!ok) break;
             tc::fence_after_sync();
             const int valid = a.Lk - j * kBN;  // keys of this tile that exist
@@ -382,12 +390,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (j == 0) {
                 m_ref = mt;
+                if (x == 0) mbar_arrive(smem_u32(&bars.b_go));
             } else {
                 const bool need = mt > m_ref + kRescaleLog2;
                 if (__any_sync(0xffffffffu, need)) {
                     // O_X must hold exactly PV_X(0..j-1): PV_X(j-1) retired
                     // once step j-1's slot is done
-                    ok = wait_bar(&bars, &bars.slot_done[(j - 1) % NST], ((j - 1) / NST) & 1);
+                    ok = wait_bar(&bars, &bars.slot_done[(j - 1) % NST][x], ((j - 1) / NST) & 1);
                     if (!ok) break;
                     tc::fence_after_sync();
                     const float m_new = need ? mt : m_ref;
