@@ -7,14 +7,17 @@
 // (2 * T * d * 2 flop per loaded byte ~ 8-32 flop/B).
 //
 // Design:
+//  - warp specialisation: a producer warp (one thread) issues each unit's
+//    TMA loads into a stage and, once every compute warp has arrived on the
+//    stage's done barrier, the TMA store of its output; the 8 compute warps
+//    wait only on the stage's full barrier (no block-wide barriers);
 //  - persistent grid; a unit of work is (position n, group of G heads), G
 //    the smallest head count that gives each of the 8 warps a task when two
 //    such stages fit one CTA per SM (d = 128, T = 24: G = 4), else the largest
-//    that keeps two CTAs per SM (more warps hide the warp-MMA latency); one
-//    thread streams the unit's q, k, v into shared memory with TMA tensor
-//    loads (one [T rows][P cols] box per tensor and head), double-buffered
-//    across units so the next unit's loads overlap this unit's math, and
-//    writes the unit's output back with TMA tensor stores;
+//    that keeps two CTAs per SM (more warps hide the warp-MMA latency); the
+//    unit's q, k, v arrive with TMA tensor loads (one [T rows][P cols] box
+//    per tensor and head), double-buffered across units so the next unit's
+//    loads overlap this unit's math, and the output leaves with TMA stores;
 //  - one warp per (head, 16-query tile): QK^T and PV run on warp-level bf16
 //    MMA (m16n8k16, fp32 accumulate) from ldmatrix fragments; the softmax is
 //    an online (streaming) softmax over 16-key blocks with quad shuffles;
@@ -33,7 +36,7 @@ namespace pab {
 namespace {
 
 constexpr int kWarps = 8;
-constexpr int kThreads = kWarps * 32;
+constexpr int kThreads = (kWarps + 1) * 32;  // 8 compute warps + a TMA producer warp
 constexpr int kMaxStageBytes = 56 * 1024;        // two CTAs per SM
 constexpr int kMaxStageBytesLarge = 110 * 1024;  // one CTA per SM
 constexpr float kLog2e = 1.4426950408889634f;
@@ -65,6 +68,7 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
                                                             TemporalArgs p) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) unsigned long long full_bar[2];
+    __shared__ __align__(8) unsigned long long done_bar[2];  // every compute warp finished the stage's unit
     __shared__ int abort_flag;
     constexpr int DK = (DN + 1) / 2;  // 16-wide k chunks covering d
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -82,8 +86,10 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
         for (int i = tid; i < n16; i += kThreads) z[i] = make_uint4(0, 0, 0, 0);
     }
     if (tid == 0) {
-        mbar_init(smem_u32(&full_bar[0]), 1);
-        mbar_init(smem_u32(&full_bar[1]), 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(smem_u32(&full_bar[s]), 1);
+            mbar_init(smem_u32(&done_bar[s]), kWarps);
+        }
         abort_flag = 0;
         fence_mbar_init();
         tc::prefetch_tmap(&tm_q);
@@ -113,35 +119,60 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
     };
 
     const long long first = blockIdx.x, step = gridDim.x;
-    // units issued / waited for so far; unit k of this CTA uses stage k & 1
-    long long n_issued = 0, n_waited = 0;
-    if (tid == 0 && first < p.units) {
-        issue_unit(first, 0);
-        n_issued = 1;
-    }
-
     const int mtiles = RT / 16;
     const int tasks = G * mtiles;
-    for (long long i = 0;; ++i) {
-        const long long u = first + i * step;
-        if (u >= p.units) break;
-        const int stage = (int)(i & 1);
-        if (tid == 0) {
-            const long long nu = u + step;
-            if (nu < p.units) {
-                // the other stage held unit i-1: its output store must have read it
-                bulk_wait_read<0>();
-                issue_unit(nu, stage ^ 1);
-                n_issued = i + 2;
-            }
-        }
-        // unit i is the (i >> 1)-th use of its stage
-        if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), (uint32_t)((i >> 1) & 1), &g_temporal_err))
-            abort_flag = 1;
-        n_waited = i + 1;
-        __syncthreads();
-        if (abort_flag) break;
+    auto store_unit = [&](long long unit, int stage) {
+        const int n = (int)(unit / hg_count);
+        const int h0 = (int)(unit - (long long)n * hg_count) * G;
+        const int c2 = p.spatial_view ? n : 0, c3 = p.spatial_view ? 0 : n;
+        for (int g = 0; g < G; ++g)
+            tc::tma_store_4d(&tm_o, sbase_u32 + 2u * (stage * stage_elems + g * head_elems), 0, h0 + g, c2, c3);
+        bulk_commit();
+    };
 
+    if (warp == kWarps) {
+        // ------------------------------------------------ producer warp (one thread)
+        if (lane == 0) {
+            // unit k of this CTA uses stage k & 1; before stage s takes unit k, the
+            // output of unit k-2 (computed in it) is stored and the store has read it
+            long long k = 0, n_issued = 0;
+            bool ok = true;
+            for (long long u = first; u < p.units; u += step, ++k) {
+                const int s = (int)(k & 1);
+                if (k >= 2) {
+                    ok = mbar_wait_bounded(smem_u32(&done_bar[s]), (uint32_t)(((k - 2) >> 1) & 1), &g_temporal_err);
+                    if (!ok) break;
+                    store_unit(u - 2 * step, s);
+                    bulk_wait_read<0>();
+                }
+                issue_unit(u, s);
+                n_issued = k + 1;
+            }
+            // the last (up to) two units' outputs
+            for (long long kk = (k >= 2 ? k - 2 : 0); ok && kk < k; ++kk) {
+                const int s = (int)(kk & 1);
+                ok = mbar_wait_bounded(smem_u32(&done_bar[s]), (uint32_t)((kk >> 1) & 1), &g_temporal_err);
+                if (ok) store_unit(first + kk * step, s);
+            }
+            if (!ok) {
+                abort_flag = 1;
+                // let every load this CTA issued land before it exits (bounded)
+                for (long long kk = (n_issued > 2 ? n_issued - 2 : 0); kk < n_issued; ++kk)
+                    mbar_wait_bounded(smem_u32(&full_bar[kk & 1]), (uint32_t)((kk >> 1) & 1), &g_temporal_err);
+            }
+            bulk_wait<0>();
+        }
+    } else {
+        // ------------------------------------------------ compute warps
+        long long i = 0;
+        for (long long u = first; u < p.units; u += step, ++i) {
+            const int stage = (int)(i & 1);
+            // unit i is the (i >> 1)-th use of its stage
+            if (!mbar_wait_bounded(smem_u32(&full_bar[stage]), (uint32_t)((i >> 1) & 1), &g_temporal_err)) {
+                abort_flag = 1;
+                break;
+            }
+            if (*(volatile int*)&abort_flag) break;
         __nv_bfloat16* st = sbase + stage * stage_elems;
         for (int task = warp; task < tasks; task += kWarps) {
             const int g = task / mtiles, mt = task - (task / mtiles) * mtiles;
@@ -245,26 +276,12 @@ __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constan
                     pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
             }
         }
-        fence_proxy_async_smem();
-        __syncthreads();
-        if (tid == 0) {
-            const int n = (int)(u / hg_count);
-            const int h0 = (int)(u - (long long)n * hg_count) * G;
-            const int c2 = p.spatial_view ? n : 0, c3 = p.spatial_view ? 0 : n;
-            for (int g = 0; g < G; ++g)
-                tc::tma_store_4d(&tm_o, sbase_u32 + 2u * (stage * stage_elems + g * head_elems), 0, h0 + g, c2,
-                                 c3);
-            bulk_commit();
+            // the outputs are written over this warp's own q rows: visible to the
+            // TMA store (async proxy) once the producer sees every warp's arrival
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&done_bar[stage]));
         }
-    }
-    if (tid == 0) {
-        if (abort_flag) {
-            // let every load this CTA issued land before it exits (bounded):
-            // units n_waited-1 (timed out) .. n_issued-1 may still be in flight
-            for (long long k = (n_waited > 0 ? n_waited - 1 : 0); k < n_issued; ++k)
-                mbar_wait_bounded(smem_u32(&full_bar[k & 1]), (uint32_t)((k >> 1) & 1), &g_temporal_err);
-        }
-        bulk_wait<0>();
     }
 }
 
