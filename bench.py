@@ -45,8 +45,8 @@ UNIT = "TFLOP/s (dense-equivalent attention)"
 # keyed by (sha256 of the kernel's source, workload); a different source hash
 # or a workload without a capture means traffic is null.
 MEASURED_TRAFFIC = {
-    # flash_tc spatial, 480p-like, 1 launch: dram read 175.91 MB + write 42.61 MB
-    ("ddc0e33765e69db2", "480p"): 218520064,
+    # flash_tc spatial, 480p-like, 1 launch: dram read 176.15 MB + write 42.39 MB
+    ("ca2dcfe83a42d92b", "480p"): 218539520,
 }
 
 
