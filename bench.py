@@ -112,6 +112,13 @@ def algorithmic_bytes(w):
             "layout": 2 * v, "mse": 2 * v}
 
 
+def workload_config(w) -> dict:
+    """The workload part of the JSON line's config, shared by both arms."""
+    return {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d,
+            "text_len": w.text_len, "diffusion_steps": w.steps, "ranges": list(w.ranges),
+            "step": "one PAB sampling run of the spatial+temporal+cross attention stack"}
+
+
 def kernel_source_hash(name: str) -> str:
     path = os.path.join(ROOT, "step_reuse_b200", "csrc", name)
     try:
@@ -381,7 +388,7 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": run_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name, "steps": w.steps, "ranges": list(w.ranges)},
+        "data": "synthetic", "config": workload_config(w),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": info["cores"], "kind": "oracle",
                          "sample": info["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -474,12 +481,10 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "T": w.T, "H": w.H, "W": w.W, "heads": w.heads, "d": w.d,
-                   "text_len": w.text_len, "diffusion_steps": w.steps, "ranges": list(w.ranges),
-                   "step": "one PAB sampling run of the spatial+temporal+cross attention stack",
-                   "l2": f"inputs larger than L2 ({n_sets} drifted input sets of "
-                         f"{7 * w.T * w.N * w.C * 2 / 1e6:.0f} MB each, cycled)",
-                   "parallelism": f"replicas x{world} (one video per GPU)"},
+        "config": dict(workload_config(w),
+                       l2=f"inputs larger than L2 ({n_sets} drifted input sets of "
+                          f"{7 * w.T * w.N * w.C * 2 / 1e6:.0f} MB each, cycled)",
+                       parallelism=f"replicas x{world} (one video per GPU)"),
         "denoising_steps_per_s": world * w.steps / (ms * 1e-3),
         "executed_tflops": world * exec_flops / (ms * 1e-3) / 1e12,
         "computes": counts,
