@@ -234,7 +234,7 @@ class AttentionStack:
                 if self.sched[k][i]:
                     n += 1 if (k != "temporal" or self.fused) else 5  # 3 layouts + attention + layout back
                     if not first[k]:
-                        n += 2  # MSE: partials + final
+                        n += 1  # MSE: one launch
                     first[k] = False
         return n
 
