@@ -98,6 +98,9 @@ def test_temporal_parity(pab, oracle_mod, N, T, heads, d):
     (5000, 120, 16, 72),  # 640 query tiles: several per CTA, heads change inside a CTA's run
     (100, 64, 300, 8),    # one query tile per head: the head changes at every tile
     (25440, 120, 4, 72),  # a 480p frame stack's rows, 4 heads
+    (257, 100, 2, 112),   # d % 16 == 0 at the largest head dim whose ones column fits O (N = 128)
+    (130, 128, 3, 96),    # d % 16 == 0: the row-sum column in an extra 16-column chunk; full 128 keys
+    (300, 90, 2, 128),    # d = 128 with a short text: the general flash kernel
 ])
 def test_cross_parity(pab, oracle_mod, R, Lt, heads, d):
     C = heads * d
