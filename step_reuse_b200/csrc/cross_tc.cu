@@ -6,32 +6,35 @@
 // kernel is bound by streaming Q in and O out of HBM.
 //
 // Persistent CTAs (one per SM) each own a contiguous run of (head, 128-row
-// query tile) work items and alternate them between two slots:
+// query tile) work items; tile i uses S buffer i & 1 and O buffer i & 1, so
+// the next tile's S is computed while the softmax works on this one:
 //   warp 12 (one thread)     TMA producer: the current head's Kt / Vt
-//                            (reloaded when the head changes, once both
-//                            issuers' MMAs on the old ones have retired --
-//                            a barrier each issuer commits once per change,
-//                            so no wait is ever two phases behind), after
-//                            which it writes 1.0 into Vt's column d for every
-//                            key; and the query tiles through a ring of three
-//                            Q buffers, each refilled as soon as its S
-//                            product has retired;
-//   warps 13, 14             tcgen05.mma issuers, one warp per slot (one
-//                            elected lane issues): S = Q Kt^T (SS form, fp32
-//                            in TMEM) and O = P Vt (TS form, P from TMEM, N =
-//                            d plus the ones column); the slot's next S is
-//                            queued right behind each P Vt product;
-//   warps 0-3 / 4-7          softmax of slot 0 / 1: thread i owns row i (TMEM
-//                            lane i), masks keys past text_len, exponentiates
-//                            (MUFU ex2 with a share on the FMA pipes) and
-//                            writes P as bf16 over S;
-//   warps 8-11               epilogue of both slots, tiles in order: O's
-//                            column d is the row sum of P (the ones column),
-//                            so O / O[:, d] is normalised, staged (128-byte
-//                            swizzle) in the slot's output buffer and stored
-//                            with TMA while the softmax warps go on.
-// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+NO), O_1 [384,384+NO).
-// Head dims up to 112 (column d must exist in O's 128 columns).
+//                            (reloaded when the head changes, once the MMAs
+//                            on the old ones have retired), after which it
+//                            writes 1.0 into Vt's column d for every key; and
+//                            the query tiles through a ring of three Q
+//                            buffers, each refilled as soon as its S product
+//                            has retired;
+//   warp 13                  tcgen05.mma issuer (one elected lane): S(i) =
+//                            Q(i) Kt^T (SS form, fp32 in TMEM) and O(i) =
+//                            P(i) Vt (TS form, P from TMEM, N = d plus the
+//                            ones column); S(i+2) is queued right behind
+//                            P(i) Vt, whose P it overwrites (in-order
+//                            execution); a tile that starts a new head also
+//                            waits for every earlier P Vt to be queued;
+//   warps 0-3 / 4-7          softmax of every tile, warpgroup hf taking keys
+//                            [64 hf, 64 hf + 64): thread i owns row i (TMEM
+//                            lane i); the two half-row maxima meet through
+//                            spare TMEM columns past O_0's N (named barrier
+//                            2); each half exponentiates its 64 scores (MUFU
+//                            ex2 with a share on the FMA pipes) and writes
+//                            its half of P as bf16 over S;
+//   warps 8-11               epilogue, tiles in order: O's column d is the
+//                            row sum of P (the ones column), so O / O[:, d]
+//                            is normalised, staged (128-byte swizzle) in the
+//                            tile's output buffer and stored with TMA.
+// TMEM: S_0 [0,128), S_1 [128,256), O_0 [256,256+NO), O_1 [384,384+NO),
+// exchange columns [368, 372).  Head dims up to 96 (NO <= 112).
 // Every wait is bounded; on time-out the CTA raises the error word, drains
 // its copies and MMAs, frees TMEM and exits.
 #include <cuda.h>
@@ -45,7 +48,7 @@ namespace {
 constexpr int kBM = 128;          // query rows per tile
 constexpr int kBN = 128;          // text keys (one tile; text_len <= 128)
 constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
-constexpr int kThreads = 480;     // 2 softmax warpgroups + epilogue warpgroup + producer + 2 MMA warps
+constexpr int kThreads = 448;     // 2 softmax warpgroups (key halves) + epilogue warpgroup + producer + MMA warp
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPolyPairsOf8 = 3;  // share of exponentials on the FMA pipes
 constexpr float kC0 = 1.0f, kC1 = 0.693282962f, kC2 = 0.242210999f, kC3 = 0.0550089180f;
@@ -54,7 +57,7 @@ __device__ unsigned int g_cross_err = 0;
 
 struct CrossArgs {
     int Lk;            // text_len (<= 128)
-    int d;             // head dim (<= 112: column d of the PV product carries the row sums)
+    int d;             // head dim (<= 96: column d of the PV product carries the row sums)
     int nqt;           // query tiles per head
     long long tiles;   // heads * nqt
     float scale_log2;  // log2(e) / sqrt(d)
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     CrossArgs a) {
     constexpr int NB = (KSTEPS + 3) / 4;  // 64-column boxes of Q, Kt and the output (d columns)
     constexpr int NBV = (NO + 63) / 64;   // boxes of Vt: d columns + the ones column
-    static_assert(NO <= 128, "O of a slot lives in 128 TMEM columns");
+    static_assert(NO <= 112, "O's columns 112..115 carry the softmax halves' maxima");
     constexpr uint32_t kTile = NB * kBox;
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -151,14 +154,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (threadIdx.x == 384) {
         mbar_init(smem_u32(&bars.kv_full), 1);
         mbar_init(smem_u32(&bars.kv_ready), 1);
-        mbar_init(smem_u32(&bars.kv_free), 2);
+        mbar_init(smem_u32(&bars.kv_free), 1);
         for (int b = 0; b < kQBufs; ++b) {
             mbar_init(smem_u32(&bars.q_full[b]), 1);
             mbar_init(smem_u32(&bars.q_free[b]), 1);
         }
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&bars.s_done[x]), 1);
-            mbar_init(smem_u32(&bars.p_full[x]), 128);
+            mbar_init(smem_u32(&bars.p_full[x]), 256);
             mbar_init(smem_u32(&bars.o_full[x]), 1);
             mbar_init(smem_u32(&bars.o_free[x]), 128);
             mbar_init(smem_u32(&bars.mma_done[x]), 1);
@@ -242,156 +245,137 @@ __global__ void __launch_bounds__(kThreads, 1)
                     mbar_wait_bounded(smem_u32(&bars.kv_full), (heads_loaded - 1) & 1, &g_cross_err);
             }
         }
-    } else if (warp == 13 || warp == 14) {
-        // ------------------------------------------------ MMA issuers (slot x: tiles i = x, x+2, ...)
-        const int x = warp - 13;
+    } else if (warp == 13) {
+        // ------------------------------------------------ MMA issuer (tile i: S and O buffers i & 1)
         {
             constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
             constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
             const uint64_t dq = tc::smem_desc(q_s, 16, 1024, 2);
             const uint64_t dk = tc::smem_desc(k_s, 16, 1024, 2);
             const uint64_t dv = tc::smem_desc(v_s, kBox, 1024, 2);
-            const uint32_t s_t = tmem + x * 128, o_t = tmem + 256 + x * 128;
-            // Kt / Vt reloads are followed in tile order (the other slot's tiles
-            // included), so a wait on kv_ready is never two phases behind
-            int heads_seen = 0, hcur = -1, next_t = 0;
-            auto advance_heads = [&](int upto) -> bool {
-                for (; next_t <= upto; ++next_t) {
-                    const int h = (t_begin + next_t) / a.nqt;
-                    if (h != hcur) {
-                        // release the old head's Kt / Vt once this issuer's MMAs on
-                        // them retire, then wait for the new ones (ones column written)
-                        if (heads_seen > 0) tc::commit_warp(smem_u32(&bars.kv_free));
-                        hcur = h;
-                        ++heads_seen;
-                        if (!wait_bar_warp(&bars, &bars.kv_ready, (heads_seen - 1) & 1)) return false;
-                    }
-                }
-                return true;
-            };
-            // S(i) = Q(i) Kt^T into this slot's S columns
+            int heads_seen = 0, hcur = -1;
+            // S(i) = Q(i) Kt^T into buffer i & 1
             auto issue_s = [&](int i) -> bool {
                 const int qb = i % kQBufs;
                 if (!wait_bar_warp(&bars, &bars.q_full[qb], (i / kQBufs) & 1)) return false;
                 tc::fence_after_sync();
                 const uint64_t a0 = dq + (uint64_t)((qb * kTile) >> 4);
+                const uint32_t s_t = tmem + (i & 1) * 128;
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const uint32_t off = (ks >> 2) * (kBox >> 4) + (ks & 3) * 2;
                     tc::mma_ss_warp(s_t, a0 + off, dk + off, idesc_s, ks > 0 ? 1u : 0u);
                 }
-                tc::commit_warp(smem_u32(&bars.s_done[x]));
+                tc::commit_warp(smem_u32(&bars.s_done[i & 1]));
                 tc::commit_warp(smem_u32(&bars.q_free[qb]));  // the Q buffer may be refilled
                 return true;
             };
-            bool ok = true;
-            if (x < n) {
-                ok = advance_heads(x);
-                if (ok) ok = issue_s(x);
-            }
-            for (int i = x; i < n && ok; i += 2) {
-                // O_X is free once the epilogue has read out the previous tile of this slot
-                if (i >= 2) ok = wait_bar_warp(&bars, &bars.o_free[x], ((i - 2) >> 1) & 1);
-                if (ok) ok = wait_bar_warp(&bars, &bars.p_full[x], (i >> 1) & 1);
+            // S(i) goes into the buffer whose P the P Vt product of tile i-2 reads, so
+            // it is queued once that product is (in-order execution); a tile that
+            // starts a new head also waits for every earlier P Vt product to be
+            // queued, then releases the old Kt / Vt and waits for the new ones
+            int s_next = 0;
+            auto issue_pending = [&](int pv_queued) -> bool {  // P Vt of tiles 0..pv_queued queued
+                while (s_next < n && s_next <= pv_queued + 2) {
+                    const int h = (t_begin + s_next) / a.nqt;
+                    if (h != hcur) {
+                        if (s_next > pv_queued + 1) break;
+                        if (heads_seen > 0) tc::commit_warp(smem_u32(&bars.kv_free));
+                        hcur = h;
+                        ++heads_seen;
+                        if (!wait_bar_warp(&bars, &bars.kv_ready, (heads_seen - 1) & 1)) return false;
+                    }
+                    if (!issue_s(s_next)) return false;
+                    ++s_next;
+                }
+                return true;
+            };
+            bool ok = issue_pending(-1);
+            for (int i = 0; i < n && ok; ++i) {
+                const int b = i & 1;
+                // O buffer b is free once the epilogue has read out tile i-2
+                if (i >= 2) ok = wait_bar_warp(&bars, &bars.o_free[b], ((i - 2) >> 1) & 1);
+                if (ok) ok = wait_bar_warp(&bars, &bars.p_full[b], (i >> 1) & 1);
                 if (!ok) break;
                 tc::fence_after_sync();
+                const uint32_t s_t = tmem + b * 128, o_t = tmem + 256 + b * 128;
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
                     tc::mma_ts_warp(o_t, s_t + kk * 8, dv + kk * 128, idesc_o, kk > 0 ? 1u : 0u);
-                tc::commit_warp(smem_u32(&bars.o_full[x]));
-                // the slot's next S, queued right behind this P Vt product (which
-                // reads P from the columns S overwrites: in-order execution)
-                if (i + 2 < n) {
-                    ok = advance_heads(i + 2);
-                    if (ok) ok = issue_s(i + 2);
-                }
+                tc::commit_warp(smem_u32(&bars.o_full[b]));
+                ok = issue_pending(i);
             }
-            // the head changes past this slot's last tile: the producer counts on
-            // both issuers' releases at every change
-            if (ok && n > 0) ok = advance_heads(n - 1);
-            tc::commit_warp(smem_u32(&bars.mma_done[x]));
-            mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_cross_err);
+            tc::commit_warp(smem_u32(&bars.mma_done[0]));
+            mbar_wait_bounded(smem_u32(&bars.mma_done[0]), 0, &g_cross_err);
         }
     } else if (warp < 8) {
-        // ------------------------------------------------ softmax (slot x)
-        const int x = warp >> 2;
+        // ------------------------------------------------ softmax: warpgroup hf takes keys [64 hf, 64 hf + 64)
+        // of every tile (S and O buffer i & 1).  The half-row maxima meet through
+        // two spare TMEM columns past O_0's N (named barrier of both warpgroups);
+        // every thread runs all n tiles and the barrier of each, also after a
+        // wait gave up, so the barrier counts always match.
+        const int hf = warp >> 2;
         const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
-        const uint32_t s_col = x * 128;
+        const uint32_t xcol = 256 + 112;  // exchange columns [xcol, xcol + 4): O_0's columns past N (N <= 112)
         const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
+        const int k0 = hf * 64;  // first key of this half
         bool ok = true;
-        for (int i = x; i < n && ok; i += 2) {
-            ok = wait_bar(&bars, &bars.s_done[x], (i >> 1) & 1);
-            if (!ok) break;
-            tc::fence_after_sync();
-            // pass 1: row max over the text keys (scale > 0 commutes with max)
-            float mrow;
-            {
-                // two halves of 64 scores keep the register footprint low;
-                // eight independent 3-input max chains per half
+        for (int i = 0; i < n; ++i) {
+            const int x = i & 1;
+            const uint32_t s_col = x * 128;
+            if (ok) ok = wait_bar(&bars, &bars.s_done[x], (i >> 1) & 1);
+            float sv[64];
+            float mp = -INFINITY;
+            if (ok) {
+                tc::fence_after_sync();
+                uint32_t r0[32], r1[32];
+                tc::ld_32col(lane_addr + s_col + k0, r0);
+                tc::ld_32col(lane_addr + s_col + k0 + 32, r1);
+                tc::wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; ++c) {
+                    sv[c] = __uint_as_float(r0[c]);
+                    sv[32 + c] = __uint_as_float(r1[c]);
+                }
+                if (k0 + 64 > a.Lk) {  // uniform: this half holds the end of the keys
+#pragma unroll
+                    for (int c = 0; c < 64; ++c)
+                        if (k0 + c >= a.Lk) sv[c] = -INFINITY;
+                }
                 float mx[8];
 #pragma unroll
-                for (int k = 0; k < 8; ++k) mx[k] = -INFINITY;
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    uint32_t r0[32], r1[32];
-                    tc::ld_32col(lane_addr + s_col + half * 64, r0);
-                    tc::ld_32col(lane_addr + s_col + half * 64 + 32, r1);
-                    tc::wait_ld();
-                    float sv[64];
-#pragma unroll
-                    for (int c = 0; c < 32; ++c) {
-                        sv[c] = __uint_as_float(r0[c]);
-                        sv[32 + c] = __uint_as_float(r1[c]);
-                    }
-                    if ((half + 1) * 64 > a.Lk) {  // uniform: only the half holding the end of the keys
-#pragma unroll
-                        for (int c = 0; c < 64; ++c)
-                            if (half * 64 + c >= a.Lk) sv[c] = -INFINITY;
-                    }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        float m = tc::max3f(mx[k], sv[k], sv[k + 8]);
-                        m = tc::max3f(m, sv[k + 16], sv[k + 24]);
-                        m = tc::max3f(m, sv[k + 32], sv[k + 40]);
-                        mx[k] = tc::max3f(m, sv[k + 48], sv[k + 56]);
-                    }
+                for (int k = 0; k < 8; ++k) {
+                    float m = tc::max3f(sv[k], sv[k + 8], sv[k + 16]);
+                    m = tc::max3f(m, sv[k + 24], sv[k + 32]);
+                    m = tc::max3f(m, sv[k + 40], sv[k + 48]);
+                    mx[k] = fmaxf(m, sv[k + 56]);
                 }
-                mrow = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
-                                 fmaxf(mx[6], mx[7])) * a.scale_log2;
+                mp = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7]));
+                tc::st_1col(lane_addr + xcol + x * 2 + hf, __float_as_uint(mp));
+                tc::wait_st();
             }
-            // pass 2: S again, 32 columns at a time (next chunk's load in
-            // flight), exponentiated and written back as bf16 P over the
-            // columns already consumed (the row sums come out of the P Vt product)
-            const tc::f32x2 negm2 = tc::pack2(-mrow, -mrow);
-            uint32_t buf[2][32];
-            tc::ld_32col(lane_addr + s_col, buf[0]);
+            // both halves' scores are in registers before either writes P over them
+            tc::fence_before_sync();
+            tc::named_bar_sync(2, 256);  // id 1 is the epilogue warpgroup's
+            tc::fence_after_sync();
+            if (!ok) continue;
+            uint32_t mo_bits;
+            tc::ld_1col(lane_addr + xcol + x * 2 + (hf ^ 1), mo_bits);
             tc::wait_ld();
+            const float mo = __uint_as_float(mo_bits);
+            // the same value in both halves (max is exact and order-free)
+            const float mrow = (hf == 0 ? fmaxf(mp, mo) : fmaxf(mo, mp)) * a.scale_log2;
+            const tc::f32x2 negm2 = tc::pack2(-mrow, -mrow);
 #pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                if (c + 1 < kBN / 32) tc::ld_32col(lane_addr + s_col + (c + 1) * 32, buf[(c + 1) & 1]);
+            for (int c = 0; c < 2; ++c) {
                 uint32_t r[16];
-                if (c * 32 >= a.Lk) {
-                    // no key of this chunk exists: P = 0 (uniform branch)
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) r[e] = 0u;
-                    tc::st_16col(lane_addr + s_col + c * 16, r);
-                    if (c + 1 < kBN / 32) tc::wait_ld();
-                    continue;
-                }
-                const bool tail = (c + 1) * 32 > a.Lk;  // uniform: the chunk holding the end of the keys
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int idx = c * 32 + 2 * e;
-                    float s0 = __uint_as_float(buf[c & 1][2 * e]);
-                    float s1 = __uint_as_float(buf[c & 1][2 * e + 1]);
-                    if (tail) {
-                        if (idx >= a.Lk) s0 = -INFINITY;
-                        if (idx + 1 >= a.Lk) s1 = -INFINITY;
-                    }
-                    const tc::f32x2 t = tc::fma2(tc::pack2(s0, s1), scale2, negm2);
+                    const tc::f32x2 t = tc::fma2(tc::pack2(sv[idx], sv[idx + 1]), scale2, negm2);
                     float t0, t1, p0, p1;
                     tc::unpack2(t, t0, t1);
-                    if (((idx >> 1) & 7) < kPolyPairsOf8) {
+                    if ((e & 7) < kPolyPairsOf8) {
                         exp2_poly2(t0, t1, p0, p1);
                     } else {
                         p0 = ex2(t0);
@@ -399,15 +383,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     r[e] = pack_bf16x2(p0, p1);
                 }
-                tc::st_16col(lane_addr + s_col + c * 16, r);
-                if (c + 1 < kBN / 32) tc::wait_ld();
+                // P of keys [k0 + 32c, k0 + 32c + 32) as bf16 pairs: columns k0/2 + 16c
+                tc::st_16col(lane_addr + s_col + hf * 32 + c * 16, r);
             }
             tc::wait_st();
             tc::fence_before_sync();
             mbar_arrive(smem_u32(&bars.p_full[x]));
         }
     } else if (warp < 12) {
-        // ------------------------------------------------ epilogue (both slots, tiles in order)
+        // ------------------------------------------------ epilogue (tiles in order, buffer i & 1)
         // Every thread runs all n iterations and both named barriers of each,
         // also after a wait gave up (then the work is skipped), so the barrier
         // counts always match.
@@ -523,9 +507,9 @@ cudaError_t launch_ks(const CUtensorMap* m, const CrossArgs& a, cudaStream_t s) 
 cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,
                          int d, cudaStream_t s) {
     if (R == 0) return cudaSuccess;
-    // longer texts, and head dims whose P Vt product has no column to spare
-    // for the row sums, take the general flash kernel
-    if (Lk > kBN || d > 112) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s);
+    // longer texts, and head dims whose P Vt product leaves no columns for the
+    // row sums and the maxima exchange, take the general flash kernel
+    if (Lk > kBN || d > 96) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s);
     CrossArgs a;
     a.Lk = Lk;
     a.d = d;
@@ -546,7 +530,6 @@ cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* ou
         case 4: return extra ? launch_ks<4, 80>(m, a, s) : launch_ks<4, 64>(m, a, s);
         case 5: return extra ? launch_ks<5, 96>(m, a, s) : launch_ks<5, 80>(m, a, s);
         case 6: return extra ? launch_ks<6, 112>(m, a, s) : launch_ks<6, 96>(m, a, s);
-        case 7: return extra ? launch_ks<7, 128>(m, a, s) : launch_ks<7, 112>(m, a, s);
         default: return cudaErrorInvalidValue;
     }
 }
