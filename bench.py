@@ -64,6 +64,9 @@ def parse_args(argv=None):
                     help="distinct drifted input sets cycled over the diffusion steps")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0,
                     help="target seconds of oracle work for the CPU baseline sample")
+    ap.add_argument("--dit", action="store_true",
+                    help="time the synthetic DiT block (projections, norms, MLP around the library's "
+                         "attention) with the workload's PAB ranges and with ranges (1, 1, 1)")
     return ap.parse_args(argv)
 
 
@@ -601,10 +604,85 @@ def stack_inputs_shape(w, kind):
     return {"q": (w.T, w.N, w.C), "k": (w.T, w.N, w.C), "v": (w.T, w.N, w.C)}
 
 
+def dit_flops(w, counts):
+    """Algorithmic flops of one sampling run of the DiT block: per computing
+    kind 4 C x C projections (cross: q and the output on the video tokens, k and
+    v on the text) plus its attention; the MLP (C -> 4C -> C) at every step."""
+    R, C, L = w.T * w.N, w.C, w.text_len
+    att = w.flops()
+    per = {"spatial": 2 * 4 * R * C * C + att["spatial"], "temporal": 2 * 4 * R * C * C + att["temporal"],
+           "cross": 2 * 2 * R * C * C + 2 * 2 * L * C * C + att["cross"]}
+    mlp = 2 * 2 * R * C * 4 * C
+    return sum(counts[k] * per[k] for k in synth.KINDS) + w.steps * mlp
+
+
+def run_dit(args):
+    """The synthetic DiT block over whole sampling runs, PAB ranges against
+    ranges (1, 1, 1) (every step computes), device-timed; one JSON line."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    import step_reuse_b200 as pab
+    from step_reuse_b200 import dit
+
+    w = synth.WORKLOADS[args.workload]
+    xs, text = synth.dit_inputs(w, device=device, seed=rank)
+    wts = dit.make_weights(w.C, seed=rank + 1, device=device)
+    stream = torch.cuda.current_stream(device)
+    res = {}
+    runs = max(1, args.steps // 10)
+    for label, ranges in (("pab", w.ranges), ("no_broadcast", (1, 1, 1))):
+        block = dit.DiTBlock(pab, w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, ranges, wts, device)
+
+        def one():
+            block.reset()
+            for i in range(w.steps):
+                block.step(i, xs[i], text, stream)
+
+        for _ in range(args.warmup):
+            one()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(runs):
+            one()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(a.elapsed_time(b) / runs, device)
+        counts = {k: sum(block.plan.is_compute(k, i) for i in range(w.steps)) for k in synth.KINDS}
+        res[label] = {"ms_per_run": ms, "computes": counts, "tflops": dit_flops(w, counts) / (ms * 1e-3) / 1e12}
+        block.close()
+    assert pab.device_errors() == 0
+    if rank == 0:
+        speedup = res["no_broadcast"]["ms_per_run"] / res["pab"]["ms_per_run"]
+        line = {
+            "metric": "synthetic DiT block: denoising steps/s with PAB broadcast",
+            "value": world * w.steps / (res["pab"]["ms_per_run"] * 1e-3), "unit": "steps/s",
+            "n_gpus": world, "runs": runs, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "dtype": "bf16", "data": "synthetic (random weights, drifting N(0, 1) residual stream)",
+            "config": dict(workload_config(w),
+                           step="one sampling run of the DiT block (all diffusion steps)",
+                           block="LN -> QKV -> attention -> out-proj per kind, "
+                                 "LN -> MLP(4C, tanh GELU); fp32 residual"),
+            "speedup_vs_no_broadcast": speedup, "pab": res["pab"], "no_broadcast": res["no_broadcast"],
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.dit:
+        return run_dit(args)
     return run_ours(args)
 
 

@@ -125,3 +125,18 @@ def drift_(inputs: dict, sigma: float, g: torch.Generator) -> None:
 def randn(shape, seed: int, dtype=torch.float32, device="cpu", scale: float = 1.0):
     g = generator(seed, device)
     return (scale * torch.randn(shape, generator=g, device=device, dtype=torch.float32)).to(dtype)
+
+
+def dit_inputs(w: Workload, device="cpu", seed: int | None = None, steps: int | None = None):
+    """Inputs of the synthetic DiT block over a sampling run: the residual
+    stream x_i [T, N, C] (fp32, N(0, 1) at step 0, then drifting by
+    sigma * N(0, 1) per step) and one text embedding [text_len, C] (bf16,
+    N(0, 1), the same at every step).  Returns (xs, text)."""
+    g = generator(w.seed if seed is None else seed)
+    x = torch.randn((w.T, w.N, w.C), generator=g)
+    text = torch.randn((w.text_len, w.C), generator=g).to(torch.bfloat16)
+    xs = [x.clone()]
+    for _ in range(1, steps or w.steps):
+        x = x + w.sigma * torch.randn(x.shape, generator=g)
+        xs.append(x.clone())
+    return [t.to(device) for t in xs], text.to(device)
