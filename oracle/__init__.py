@@ -18,7 +18,11 @@ What each function computes (sources are the PAB pages):
     broadcasts each compute to the following (range - 1) steps;
   * mse -- the attention-difference diagnostic of Fig. 1 (MSE between the
     outputs of consecutive diffusion steps);
-  * layout -- the spatial view [T, N, C] <-> temporal view [N, T, C].
+  * layout -- the spatial view [T, N, C] <-> temporal view [N, T, C];
+  * sta_attention -- sliding tile attention as the spatial kind (sgqg.cn
+    summary of "Fast Video Generation with Sliding Tile Attention", section
+    "Sliding Tile Attention (STA)"): 2-D tiles per frame, a window of whole
+    tiles centred on the query's tile, cut off at the frame edge.
 """
 from __future__ import annotations
 
@@ -57,6 +61,7 @@ def _load():
         lib.oracle_spatial_attention.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 4
         lib.oracle_temporal_attention.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 4
         lib.oracle_cross_attention.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_long] + [ctypes.c_int] * 3
+        lib.oracle_sta_attention.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 8
         lib.oracle_pab_edge_steps.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.oracle_pab_schedule.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _ip, _ip]
         lib.oracle_mse.argtypes = [_dp, _dp, ctypes.c_long]
@@ -64,7 +69,7 @@ def _load():
         lib.oracle_layout.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 4
         lib.oracle_num_threads.restype = ctypes.c_int
         for name in ("oracle_spatial_attention", "oracle_temporal_attention",
-                     "oracle_cross_attention", "oracle_pab_edge_steps",
+                     "oracle_cross_attention", "oracle_sta_attention", "oracle_pab_edge_steps",
                      "oracle_pab_schedule", "oracle_layout", "oracle_num_threads"):
             if getattr(lib, name).restype is not ctypes.c_double:
                 getattr(lib, name).restype = ctypes.c_int
@@ -122,6 +127,24 @@ def cross_attention(q, kt, vt, heads: int) -> np.ndarray:
     if rc != 0:
         raise RuntimeError(f"oracle_cross_attention failed ({rc})")
     return o.reshape(shape)
+
+
+def sta_attention(q, k, v, H: int, W: int, heads: int, tile: int, win_h: int, win_w: int) -> np.ndarray:
+    """Sliding tile attention within each frame: q, k, v [T, H*W, C] ->
+    out [T, H*W, C].  Each query attends to the keys of the tiles (tile x tile
+    tokens) inside a window of win_h x win_w tokens (odd tile counts)
+    centred on its own tile, cut off at the frame edge."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, N, C = q.shape
+    assert N == H * W and k.shape == q.shape and v.shape == q.shape and C % heads == 0
+    o = np.empty_like(q)
+    rc = _load().oracle_sta_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), T, H, W, heads, C // heads,
+                                      tile, win_h, win_w)
+    if rc == -1:
+        raise ValueError("bad STA arguments (sizes must be whole tiles, windows odd tile counts)")
+    if rc != 0:
+        raise RuntimeError(f"oracle_sta_attention failed ({rc})")
+    return o
 
 
 def edge_steps(steps: int, edge_pct: int = 15) -> int:

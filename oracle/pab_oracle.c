@@ -168,6 +168,75 @@ int oracle_cross_attention(const double *q, const double *kt, const double *vt,
     return bad ? -2 : 0;
 }
 
+/* Sliding tile attention (STA) as the spatial kind: sgqg.cn summary of
+ * "Fast Video Generation with Sliding Tile Attention", section "Sliding Tile
+ * Attention (STA)" -- a frame is cut into non-overlapping tiles, every query
+ * of a tile attends to the keys of the tiles inside a window around its own
+ * tile, and frame and window sizes are whole numbers of tiles, so the tile
+ * fits the window exactly.  2-D reading (PAB's spatial attention is per
+ * frame): tiles of tile x tile tokens on the H x W token grid (token n = y*W
+ * + x, the [T][N][C] layout), a window of win_h x win_w tokens = an odd
+ * number of tiles in each direction centred on the query's tile, cut off at
+ * the frame edge (no shift).  Per (frame, head, query tile) the window's keys
+ * and values are gathered into scratch in row-major token order and every
+ * query of the tile attends to them with the textbook definition above.
+ * Returns -1 on arguments that break these rules. */
+int oracle_sta_attention(const double *q, const double *k, const double *v,
+                         double *o, int T, int H, int W, int heads, int d,
+                         int tile, int win_h, int win_w)
+{
+    if (T < 0 || H < 0 || W < 0 || heads <= 0 || d <= 0 || tile <= 0)
+        return -1;
+    if (H % tile || W % tile || win_h <= 0 || win_w <= 0 || win_h % tile || win_w % tile)
+        return -1;
+    if ((win_h / tile) % 2 == 0 || (win_w / tile) % 2 == 0)
+        return -1;
+    const long C = (long)heads * d;
+    const long N = (long)H * W;
+    const int th = H / tile, tw = W / tile;
+    const int rh = (win_h / tile - 1) / 2, rw = (win_w / tile - 1) / 2;
+    const long maxkeys = (long)(2 * rh + 1) * tile * (2 * rw + 1) * tile;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * (maxkeys > 0 ? maxkeys : 1));
+        double *kw = (double *)malloc(sizeof(double) * (size_t)(maxkeys > 0 ? maxkeys : 1) * d);
+        double *vw = (double *)malloc(sizeof(double) * (size_t)(maxkeys > 0 ? maxkeys : 1) * d);
+        if (!p || !kw || !vw) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for collapse(3) schedule(dynamic)
+            for (int t = 0; t < T; ++t)
+                for (int h = 0; h < heads; ++h)
+                    for (int qt = 0; qt < th * tw; ++qt) {
+                        const int ty = qt / tw, tx = qt % tw;
+                        const int y0 = (ty - rh < 0 ? 0 : ty - rh) * tile;
+                        const int y1 = (ty + rh >= th ? th : ty + rh + 1) * tile;
+                        const int x0 = (tx - rw < 0 ? 0 : tx - rw) * tile;
+                        const int x1 = (tx + rw >= tw ? tw : tx + rw + 1) * tile;
+                        const long frame = (long)t * N * C + (long)h * d;
+                        int nk = 0;
+                        for (int y = y0; y < y1; ++y)
+                            for (int x = x0; x < x1; ++x, ++nk) {
+                                const long src = frame + ((long)y * W + x) * C;
+                                memcpy(kw + (long)nk * d, k + src, sizeof(double) * d);
+                                memcpy(vw + (long)nk * d, v + src, sizeof(double) * d);
+                            }
+                        for (int y = ty * tile; y < (ty + 1) * tile; ++y)
+                            for (int x = tx * tile; x < (tx + 1) * tile; ++x) {
+                                const long at = frame + ((long)y * W + x) * C;
+                                attend_one_query(q + at, kw, d, vw, d, nk, d, o + at, p);
+                            }
+                    }
+        }
+        free(p);
+        free(kw);
+        free(vw);
+    }
+    return bad ? -2 : 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* PAB schedule, walked step by step in execution order (noisiest first).    */
 /*   edge steps (first and last edge_pct%): always compute;                  */
