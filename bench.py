@@ -56,7 +56,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny"))
+    ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny", "sta_48x80"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
@@ -64,6 +64,10 @@ def parse_args(argv=None):
                     help="distinct drifted input sets cycled over the diffusion steps")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0,
                     help="target seconds of oracle work for the CPU baseline sample")
+    ap.add_argument("--sta", action="store_true",
+                    help="sliding tile attention as the spatial kind (workload sta_48x80 unless "
+                         "--workload names another with a spatial window): the kernel against full "
+                         "spatial attention, and the PAB stack with each")
     ap.add_argument("--dit", action="store_true",
                     help="time the synthetic DiT block (projections, norms, MLP around the library's "
                          "attention) with the workload's PAB ranges and with ranges (1, 1, 1)")
@@ -210,12 +214,14 @@ class AttentionStack:
     fused=True: the temporal kernel reads and writes the spatial view itself
     (pab_plan_set_temporal_view), no layout launches."""
 
-    def __init__(self, pab, w, device, fused=False):
+    def __init__(self, pab, w, device, fused=False, window=()):
         self.pab, self.w, self.dev, self.fused = pab, w, device, fused
         self.plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges,
                              dtype=torch.bfloat16)
         if fused:
             self.plan.set_temporal_view(True)
+        if window:
+            self.plan.set_spatial_window(*window)
         self.plan.prepare()
         T, N, C = w.T, w.N, w.C
         # temporal-view scratch and the spatial-view copy of the temporal output
@@ -677,10 +683,129 @@ def run_dit(args):
     return 0
 
 
+def sta_pairs(w):
+    """Query-key pairs per frame of sliding tile attention: every query of
+    tile (ty, tx) meets the keys of the window's tiles, clipped at the edge."""
+    tile, win_h, win_w = w.spatial_window
+    th, tw = w.H // tile, w.W // tile
+    rh, rw = (win_h // tile - 1) // 2, (win_w // tile - 1) // 2
+    rows = [min(ty + rh + 1, th) - max(ty - rh, 0) for ty in range(th)]
+    cols = [min(tx + rw + 1, tw) - max(tx - rw, 0) for tx in range(tw)]
+    return (tile * tile) ** 2 * sum(rows) * sum(cols)
+
+
+def run_sta(args):
+    """Sliding tile attention as the spatial kind: the kernel alone against
+    full spatial attention on the same tensors, then one PAB sampling run of
+    the fused attention stack with each; device-timed; one JSON line."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    import step_reuse_b200 as pab
+
+    name = args.workload if synth.WORKLOADS[args.workload].spatial_window else "sta_48x80"
+    w = synth.WORKLOADS[name]
+    tile, win_h, win_w = w.spatial_window
+    T, N, C = w.T, w.N, w.C
+    sta_flops = 4.0 * T * w.heads * w.d * sta_pairs(w)
+    full_flops = w.flops()["spatial"]
+    n_sets = max(1, min(w.steps, args.input_sets))
+    inputs = make_inputs(w, device, n_sets, seed=rank)
+    stream = torch.cuda.current_stream(device)
+    out = torch.empty((T, N, C), dtype=torch.bfloat16, device=device)
+    launches = {
+        "sta": lambda x: pab.sta_attention(x["q"], x["k"], x["v"], w.H, w.W, w.heads, tile, win_h, win_w,
+                                           out=out, stream=stream),
+        "full": lambda x: pab.spatial_attention(x["q"], x["k"], x["v"], w.heads, out=out, stream=stream),
+    }
+    reps = max(5, args.steps)
+    kern = {}
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    clocks.mark_start()
+    for label, fn in launches.items():
+        for i in range(args.warmup):
+            fn(inputs[i % n_sets]["spatial"])
+        torch.cuda.synchronize(device)
+        barrier(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(reps):
+            fn(inputs[i % n_sets]["spatial"])
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        kern[label] = max_over_ranks(a.elapsed_time(b) / reps, device)
+    assert pab.device_errors() == 0
+    runs = max(3, args.steps // 10)
+    stacks = {}
+    for label, window in (("sta", w.spatial_window), ("full", ())):
+        st = AttentionStack(pab, w, device, fused=True, window=window)
+        for _ in range(args.warmup):
+            st.run(inputs, stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(runs):
+            st.run(inputs, stream)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        stacks[label] = {"ms_per_run": max_over_ranks(a.elapsed_time(b) / runs, device),
+                         "gpu_launches_per_run": st.launches_per_run}
+        st.close()
+    clocks.mark_end()
+    clk = clocks.stop()
+    assert pab.device_errors() == 0
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peak_src = "measured"
+    except (OSError, ValueError):
+        peak_src = "fallback"
+    tc_peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    achieved = sta_flops / (kern["sta"] * 1e-3) / 1e12
+    if rank == 0:
+        line = {
+            "metric": "sliding tile attention as the spatial kind: kernel TFLOP/s (window pairs) "
+                      "and PAB stack steps/s",
+            "value": world * sta_flops / (kern["sta"] * 1e-3) / 1e12, "unit": "TFLOP/s (algorithmic, window)",
+            "n_gpus": world, "steps": reps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(w), spatial_window={"tile": tile, "win_h": win_h, "win_w": win_w},
+                           l2=f"inputs larger than L2 ({n_sets} input sets cycled)"),
+            "roofline": {"kernel": "sliding tile attention (flash_tc, window geometry)", "bound": "tensor",
+                         "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
+                         "traffic": None, "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "algorithmic_flops_per_launch": sta_flops},
+            "kernel_ms": {"sta": kern["sta"], "full_spatial": kern["full"]},
+            "window_share_of_full": sta_flops / full_flops,
+            "kernel_speedup_vs_full": kern["full"] / kern["sta"],
+            "full_spatial_tflops": full_flops / (kern["full"] * 1e-3) / 1e12,
+            "stack": {k: dict(v, denoising_steps_per_s=world * w.steps / (v["ms_per_run"] * 1e-3))
+                      for k, v in stacks.items()},
+            "stack_speedup_vs_full": stacks["full"]["ms_per_run"] / stacks["sta"]["ms_per_run"],
+            "gpu_launches": reps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.sta:
+        return run_sta(args)
     if args.dit:
         return run_dit(args)
     return run_ours(args)

@@ -82,6 +82,23 @@ const char* pab_last_error_string(void);
 int pab_spatial_attention(const void* q, const void* k, const void* v, void* out,
                           int T, int N, int heads, int d, void* cuda_stream);
 
+/* Sliding tile attention (STA) as the spatial kind (sgqg.cn summary of
+ * "Fast Video Generation with Sliding Tile Attention", section "Sliding Tile
+ * Attention (STA)": non-overlapping tiles, each query tile attends to the
+ * key tiles inside a window around it, frame and window sizes in whole
+ * tiles).  Within each frame of q, k, v, out [T, H*W, C] (token n = y*W + x):
+ * tiles of tile x tile tokens; a query in tile (ty, tx) attends to every key
+ * whose tile (ky, kx) has |ky - ty| <= (win_h/tile - 1)/2 and
+ * |kx - tx| <= (win_w/tile - 1)/2 (the window is centred on the query's tile
+ * and cut off at the frame edge), with the softmax of the spatial kind over
+ * those keys.  tile must be 16 (the kernel's tile: one CTA's 256 queries);
+ * H, W, win_h, win_w must be multiples of it, with odd win_h/tile and
+ * win_w/tile (PAB_ERR_ARG else; PAB_ERR_UNSUPPORTED for another tile).
+ * A window covering the frame gives pab_spatial_attention's result.
+ * PAB_BF16 only. */
+int pab_sta_attention(const void* q, const void* k, const void* v, void* out, int T, int H, int W,
+                      int heads, int d, int tile, int win_h, int win_w, void* cuda_stream);
+
 /* Temporal attention (same section: attention across frames).
  * q, k, v, out: [N, T, C] (the temporal view).  For each position n, head h:
  *   out[n, t, h] = sum_s softmax_s(q[n, t, h] . k[n, s, h] / sqrt(d)) v[n, s, h].
@@ -186,6 +203,13 @@ int pab_plan_reset(pab_plan* plan);
  * spatial_view = 0 (default) -> [N, T, C]; 1 -> [T, N, C] (the spatial view,
  * no layout change needed around the call).  Call before the run starts. */
 int pab_plan_set_temporal_view(pab_plan* plan, int spatial_view);
+
+/* Make this plan's SPATIAL computes sliding tile attention
+ * (pab_sta_attention with the plan's H, W and these tile / window sizes)
+ * instead of full attention within the frame; win_h = win_w = 0 restores
+ * full attention.  Same argument rules as pab_sta_attention.  Call before
+ * the run starts (the broadcast schedule and cache are unchanged). */
+int pab_plan_set_spatial_window(pab_plan* plan, int tile, int win_h, int win_w);
 
 /* Allocate the cache (2 output slots per kind, plus bf16 staging for
  * PAB_FP32 plans) on the current device now instead of at each kind's first

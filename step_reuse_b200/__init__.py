@@ -33,7 +33,8 @@ BF16, FP32 = 0, 1
 # every symbol include/pab.h declares
 EXPORTS = (
     "pab_version", "pab_last_error_string", "pab_spatial_attention", "pab_temporal_attention",
-    "pab_temporal_attention_sv", "pab_plan_set_temporal_view",
+    "pab_temporal_attention_sv", "pab_plan_set_temporal_view", "pab_sta_attention",
+    "pab_plan_set_spatial_window",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
     "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
@@ -64,6 +65,8 @@ def _load() -> ctypes.CDLL:
         "pab_temporal_attention": ([vp, vp, vp, vp, i, i, i, i, vp], i),
         "pab_temporal_attention_sv": ([vp, vp, vp, vp, i, i, i, i, vp], i),
         "pab_plan_set_temporal_view": ([vp, i], i),
+        "pab_sta_attention": ([vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp], i),
+        "pab_plan_set_spatial_window": ([vp, i, i, i], i),
         "pab_cross_attention": ([vp, vp, vp, vp, ll, i, i, i, vp], i),
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
         "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
@@ -128,6 +131,20 @@ def spatial_attention(q, k, v, heads: int, out=None, stream=None):
     out = torch.empty_like(q) if out is None else out
     _check(lib.pab_spatial_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), T, N, heads, C // heads,
                                      _stream(stream)))
+    return out
+
+
+def sta_attention(q, k, v, H: int, W: int, heads: int, tile: int = 16, win_h: int = 48, win_w: int = 48,
+                  out=None, stream=None):
+    """Sliding tile attention within each frame: q, k, v [T, H*W, C] bf16
+    CUDA tensors -> [T, H*W, C]; tile x tile-token tiles, a win_h x win_w
+    window (odd tile counts) centred on each query's tile, cut at the edge."""
+    T, N, C = q.shape
+    if N != H * W:
+        raise ValueError(f"q has {N} tokens per frame, H*W = {H * W}")
+    out = torch.empty_like(q) if out is None else out
+    _check(lib.pab_sta_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), T, H, W, heads, C // heads,
+                                 tile, win_h, win_w, _stream(stream)))
     return out
 
 
@@ -243,6 +260,11 @@ class Plan:
         """True: TEMPORAL takes and returns [T, N, C] instead of [N, T, C]."""
         _check(lib.pab_plan_set_temporal_view(self._h, 1 if spatial_view else 0))
         self.temporal_sv = bool(spatial_view)
+
+    def set_spatial_window(self, tile: int = 16, win_h: int = 0, win_w: int = 0):
+        """Spatial computes become sliding tile attention with this window
+        (win_h = win_w = 0: full attention within the frame again)."""
+        _check(lib.pab_plan_set_spatial_window(self._h, tile, win_h, win_w))
 
     def prepare(self):
         _check(lib.pab_plan_prepare(self._h))

@@ -54,6 +54,7 @@ namespace pab {
 namespace {
 
 constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
+constexpr int kStaTile = 16;      // sliding tile attention: 16 x 16-token tiles (the CTA's 256 queries)
 constexpr int kBN = 64;           // keys per K/V tile
 constexpr int kQBox = 128 * 128;  // bytes of one [128 rows][64 cols] bf16 box (Q, O)
 constexpr int kKVBox = 64 * 128;  // bytes of one [64 rows][64 cols] bf16 box (K, V)
@@ -81,6 +82,9 @@ struct FlashTcArgs {
     int kv_batched;    // 1: K/V have a batch coordinate (spatial); 0: shared (cross)
     int d;             // head dim
     float scale_log2;  // log2(e) / sqrt(d)
+    // sliding tile attention only: the frame in 16 x 16 tiles and the
+    // window's reach in tiles on each side of the query tile
+    int tiles_h, tiles_w, reach_h, reach_w;
 };
 
 constexpr int kMaxStages = 8;
@@ -158,7 +162,13 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
 // column inside the PV product's N = 16 * KSTEPS -- is set to 1 once the tile
 // lands (warp 11), so O's column d accumulates the row sum of P with the same
 // bf16 P as the numerator; the softmax then keeps no running sum.
-template <int KSTEPS, int NST, bool ONES>
+// STA (sliding tile attention): the CTA's 256 queries are one 16 x 16 tile
+// of the frame (tile A its upper 8 rows, tile B the lower 8, each read as a
+// [8][16]-token TMA box of the [H][W] grid), and the key loop runs over the
+// 16 x 16 key tiles of the window around it, clipped at the frame edge, each
+// as four [4][16]-token blocks of 64 keys.  Every block is whole, so nothing
+// is masked.
+template <int KSTEPS, int NST, bool ONES, bool STA>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -179,8 +189,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qblk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    const int nkv = (a.Lk + kBN - 1) / kBN;
-    const bool has_b = qblk * 2 * kBM + kBM < a.Lq;
+    // STA geometry: query tile (ty, tx); window tiles [wy0, wy0 + rows) x [wx0, wx0 + cols)
+    int ty = 0, tx = 0, wy0 = 0, wx0 = 0, wcols = 1, nkv;
+    if constexpr (STA) {
+        ty = qblk / a.tiles_w;
+        tx = qblk - ty * a.tiles_w;
+        wy0 = max(ty - a.reach_h, 0);
+        wx0 = max(tx - a.reach_w, 0);
+        const int wy1 = min(ty + a.reach_h + 1, a.tiles_h), wx1 = min(tx + a.reach_w + 1, a.tiles_w);
+        wcols = wx1 - wx0;
+        nkv = (wy1 - wy0) * wcols * 4;
+    } else {
+        nkv = (a.Lk + kBN - 1) / kBN;
+    }
+    const bool has_b = STA || qblk * 2 * kBM + kBM < a.Lq;
     const int ntiles = has_b ? 2 : 1;
 
     if (threadIdx.x == 256) {
@@ -214,6 +236,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc::fence_after_sync();
     const uint32_t tmem = bars.tmem_base;
     const int kvb = a.kv_batched ? b : 0;
+    // TMA coordinates of query tile x's box and of key block j's box
+    auto load_q = [&](uint32_t dst, int x, int bx, uint32_t bar) {
+        if constexpr (STA)
+            tc::tma_load_5d(dst, &tm_q, bx * 64, h, tx * 16, ty * 16 + x * 8, b, bar);
+        else
+            tc::tma_load_4d(dst, &tm_q, bx * 64, h, (qblk * 2 + x) * kBM, b, bar);
+    };
+    auto load_kv = [&](uint32_t dst, const CUtensorMap* m, int j, int bx, uint32_t bar) {
+        if constexpr (STA) {
+            const int t = j >> 2, ky = wy0 + t / wcols, kx = wx0 + t % wcols;
+            tc::tma_load_5d(dst, m, bx * 64, h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
+        } else {
+            tc::tma_load_4d(dst, m, bx * 64, h, j * kBN, kvb, bar);
+        }
+    };
 
     if (warp == 8) {
         // ------------------------------------------------ TMA producer
@@ -221,16 +258,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int x = 0; x < ntiles; ++x) {
                 mbar_arrive_expect_tx(smem_u32(&bars.q_full[x]), kQTile);
                 for (int bx = 0; bx < NB; ++bx)
-                    tc::tma_load_4d(q_s + x * kQTile + bx * kQBox, &tm_q, bx * 64, h, (qblk * 2 + x) * kBM, b,
-                                    smem_u32(&bars.q_full[x]));
+                    load_q(q_s + x * kQTile + bx * kQBox, x, bx, smem_u32(&bars.q_full[x]));
             }
             const int n01 = nkv < 2 ? nkv : 2;
             if (n01 > 0) {
                 mbar_arrive_expect_tx(smem_u32(&bars.k01_full), n01 * kKVTile);
                 for (int j = 0; j < n01; ++j)
                     for (int bx = 0; bx < NB; ++bx)
-                        tc::tma_load_4d(k01_s + j * kKVTile + bx * kKVBox, &tm_k, bx * 64, h, j * kBN, kvb,
-                                        smem_u32(&bars.k01_full));
+                        load_kv(k01_s + j * kKVTile + bx * kKVBox, &tm_k, j, bx, smem_u32(&bars.k01_full));
             }
             int nslot = 0;  // slot loads issued
             bool ok = true;
@@ -242,12 +277,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool with_k = j + 2 < nkv;
                 const uint32_t bar = smem_u32(&bars.slot_full[st]);
                 mbar_arrive_expect_tx(bar, with_k ? 2 * kKVTile : kKVTile);
-                for (int bx = 0; bx < NB; ++bx)
-                    tc::tma_load_4d(v_s + st * kKVTile + bx * kKVBox, &tm_v, bx * 64, h, j * kBN, kvb, bar);
+                for (int bx = 0; bx < NB; ++bx) load_kv(v_s + st * kKVTile + bx * kKVBox, &tm_v, j, bx, bar);
                 if (with_k)
                     for (int bx = 0; bx < NB; ++bx)
-                        tc::tma_load_4d(k_s + st * kKVTile + bx * kKVBox, &tm_k, bx * 64, h, (j + 2) * kBN, kvb,
-                                        bar);
+                        load_kv(k_s + st * kKVTile + bx * kKVBox, &tm_k, j + 2, bx, bar);
                 nslot = j + 1;
             }
             if (!ok || *(volatile int*)&bars.abort) {
@@ -354,7 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_bar(&bars, &bars.slot_done[(j - 2) % NST][x], ((j - 2) / NST) & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            const int valid = a.Lk - j * kBN;  // keys of this tile that exist
+            const int valid = STA ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
             // the row's 64 scores fit in registers: one TMEM read
             float sv[kBN];
             {
@@ -482,8 +515,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc::named_bar_sync(1 + x, 128);
         if (ok && row == 0) {
-            for (int bx = 0; bx < NB; ++bx)
-                tc::tma_store_4d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
+            for (int bx = 0; bx < NB; ++bx) {
+                if constexpr (STA)
+                    tc::tma_store_5d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, tx * 16, ty * 16 + x * 8, b);
+                else
+                    tc::tma_store_4d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
+            }
             bulk_commit();
             bulk_wait<0>();
         }
@@ -531,25 +568,57 @@ bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows
     return r == CUDA_SUCCESS;
 }
 
-template <int KSTEPS, bool ONES>
+// 5-D map over the [frames][H][W][heads][d] bf16 spatial view: dims (d,
+// heads, W, H, frames), box (64, 1, 16, box_h, 1) -- 16 * box_h tokens of a
+// 16-wide tile, row-major, one 128-byte swizzled row each.
+bool make_map_grid(CUtensorMap* m, const void* base, int d, int heads, int H, int W, int frames, int box_h) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t C = (cuuint64_t)heads * d;
+    cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)frames};
+    cuuint64_t strides[4] = {(cuuint64_t)d * 2, C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
+    cuuint32_t box[5] = {64, 1, 16, (cuuint32_t)box_h, 1};
+    cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int KSTEPS, bool ONES, bool STA>
 cudaError_t launch_ks1(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                        const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
     constexpr int NST = NB == 1 ? 6 : 4;  // ring slots of (V_j, K_{j+2})
     const size_t smem = (size_t)NB * (2 * kQBox + (2 + 2 * NST) * kKVBox) + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST, ONES>,
+    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST, ONES, STA>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
     if (e != cudaSuccess) return e;
-    flash_tc_kernel<KSTEPS, NST, ONES><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    flash_tc_kernel<KSTEPS, NST, ONES, STA><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
-template <int KSTEPS>
+template <int KSTEPS, bool STA>
 cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     // a padding column inside the PV product carries the row sums when d % 16 != 0
-    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true>(mq, mk, mv, mo, a, grid, s);
-    return launch_ks1<KSTEPS, false>(mq, mk, mv, mo, a, grid, s);
+    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true, STA>(mq, mk, mv, mo, a, grid, s);
+    return launch_ks1<KSTEPS, false, STA>(mq, mk, mv, mo, a, grid, s);
+}
+template <bool STA>
+cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
+                     const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
+    switch ((a.d + 15) / 16) {
+        case 1: return launch_ks<1, STA>(mq, mk, mv, mo, a, grid, s);
+        case 2: return launch_ks<2, STA>(mq, mk, mv, mo, a, grid, s);
+        case 3: return launch_ks<3, STA>(mq, mk, mv, mo, a, grid, s);
+        case 4: return launch_ks<4, STA>(mq, mk, mv, mo, a, grid, s);
+        case 5: return launch_ks<5, STA>(mq, mk, mv, mo, a, grid, s);
+        case 6: return launch_ks<6, STA>(mq, mk, mv, mo, a, grid, s);
+        case 7: return launch_ks<7, STA>(mq, mk, mv, mo, a, grid, s);
+        case 8: return launch_ks<8, STA>(mq, mk, mv, mo, a, grid, s);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace
@@ -574,18 +643,35 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
     a.kv_batched = kv_bstride > 0 ? 1 : 0;
     a.d = d;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+    a.tiles_h = a.tiles_w = a.reach_h = a.reach_w = 0;
     dim3 grid((unsigned)qblocks, (unsigned)heads, (unsigned)batches);
-    switch ((d + 15) / 16) {
-        case 1: return launch_ks<1>(mq, mk, mv, mo, a, grid, s);
-        case 2: return launch_ks<2>(mq, mk, mv, mo, a, grid, s);
-        case 3: return launch_ks<3>(mq, mk, mv, mo, a, grid, s);
-        case 4: return launch_ks<4>(mq, mk, mv, mo, a, grid, s);
-        case 5: return launch_ks<5>(mq, mk, mv, mo, a, grid, s);
-        case 6: return launch_ks<6>(mq, mk, mv, mo, a, grid, s);
-        case 7: return launch_ks<7>(mq, mk, mv, mo, a, grid, s);
-        case 8: return launch_ks<8>(mq, mk, mv, mo, a, grid, s);
-        default: return cudaErrorInvalidValue;
-    }
+    return launch_d<false>(mq, mk, mv, mo, a, grid, s);
+}
+
+cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
+                             int heads, int d, int win_h, int win_w, cudaStream_t s) {
+    if (frames == 0 || H == 0 || W == 0) return cudaSuccess;
+    if (H % kStaTile || W % kStaTile || win_h % kStaTile || win_w % kStaTile || win_h <= 0 || win_w <= 0 ||
+        (win_h / kStaTile) % 2 == 0 || (win_w / kStaTile) % 2 == 0)
+        return cudaErrorInvalidValue;
+    const long long tiles = (long long)(H / kStaTile) * (W / kStaTile);
+    if (tiles > 0x7fffffffLL || frames > 65535 || heads > 65535) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map_grid(&mq, q, d, heads, H, W, frames, 8) || !make_map_grid(&mk, k, d, heads, H, W, frames, 4) ||
+        !make_map_grid(&mv, v, d, heads, H, W, frames, 4) || !make_map_grid(&mo, out, d, heads, H, W, frames, 8))
+        return cudaErrorInvalidValue;
+    FlashTcArgs a;
+    a.Lq = H * W;
+    a.Lk = H * W;
+    a.kv_batched = 1;
+    a.d = d;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+    a.tiles_h = H / kStaTile;
+    a.tiles_w = W / kStaTile;
+    a.reach_h = (win_h / kStaTile - 1) / 2;
+    a.reach_w = (win_w / kStaTile - 1) / 2;
+    dim3 grid((unsigned)tiles, (unsigned)heads, (unsigned)frames);
+    return launch_d<true>(mq, mk, mv, mo, a, grid, s);
 }
 
 unsigned int flash_device_errors(bool clear) {

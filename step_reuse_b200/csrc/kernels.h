@@ -39,6 +39,12 @@ unsigned int temporal_device_errors(bool clear);
 cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches,
                          long long Lq, int Lk, int heads, int d, long long q_bstride,
                          long long kv_bstride, cudaStream_t s);
+// Sliding tile attention within each frame of a [frames][H*W][heads*d] bf16
+// spatial view: 16 x 16-token tiles, a window of win_h x win_w tokens (odd
+// tile counts) centred on the query's tile and clipped at the frame edge.
+// H, W, win_h, win_w must be multiples of 16 (cudaErrorInvalidValue else).
+cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
+                             int heads, int d, int win_h, int win_w, cudaStream_t s);
 
 unsigned int flash_device_errors(bool clear);
 

@@ -108,6 +108,22 @@ int run_spatial(const void* q, const void* k, const void* v, void* out, int T, i
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "spatial attention launch");
 }
 
+int check_sta(int H, int W, int tile, int win_h, int win_w) {
+    if (tile != 16) return fail(PAB_ERR_UNSUPPORTED, "sliding tile attention tile %d unsupported (need 16)", tile);
+    if (H % tile || W % tile) return fail(PAB_ERR_ARG, "frame %d x %d is not whole %d-token tiles", H, W, tile);
+    if (win_h <= 0 || win_w <= 0 || win_h % tile || win_w % tile || (win_h / tile) % 2 == 0 ||
+        (win_w / tile) % 2 == 0)
+        return fail(PAB_ERR_ARG, "window %d x %d must be an odd number of %d-token tiles each way", win_h, win_w,
+                    tile);
+    return PAB_OK;
+}
+
+int run_sta(const void* q, const void* k, const void* v, void* out, int T, int H, int W, int heads, int d,
+            int win_h, int win_w, cudaStream_t s) {
+    cudaError_t e = pab::launch_flash_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, s);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "sliding tile attention launch");
+}
+
 int run_temporal(const void* q, const void* k, const void* v, void* out, int N, int T, int heads,
                  int d, int spatial_view, cudaStream_t s) {
     cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s);
@@ -154,6 +170,7 @@ struct pab_plan {
     int range[3];
     int edge_pct, lo, hi;
     int temporal_sv;  // temporal attention takes / returns the spatial view
+    int sta_win_h, sta_win_w;  // > 0: spatial computes are sliding tile attention (16-token tiles)
     // cache
     int device;
     void* slot[3][2];
@@ -239,7 +256,9 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
         oo = p->stage_out;
     }
     int rc;
-    if (kind == PAB_SPATIAL)
+    if (kind == PAB_SPATIAL && p->sta_win_h > 0)
+        rc = run_sta(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->sta_win_h, p->sta_win_w, s);
+    else if (kind == PAB_SPATIAL)
         rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s);
     else if (kind == PAB_TEMPORAL)
         rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, p->temporal_sv, s);
@@ -282,6 +301,23 @@ int pab_spatial_attention(const void* q, const void* k, const void* v, void* out
     rc = check_ptrs("q, k, v, out", q, k, v, out);
     if (rc) return rc;
     return run_spatial(q, k, v, out, T, N, heads, d, static_cast<cudaStream_t>(cuda_stream));
+    PAB_GUARD_END
+}
+
+int pab_sta_attention(const void* q, const void* k, const void* v, void* out, int T, int H, int W,
+                      int heads, int d, int tile, int win_h, int win_w, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || H < 0 || W < 0) return fail(PAB_ERR_ARG, "T, H, W must be >= 0 (got %d, %d, %d)", T, H, W);
+    rc = check_sta(H, W, tile, win_h, win_w);
+    if (rc) return rc;
+    if ((long long)T * H * W == 0) return PAB_OK;
+    if (T > 65535) return fail(PAB_ERR_UNSUPPORTED, "T=%d frames exceeds 65535", T);
+    if ((long long)H * W > (1LL << 30)) return fail(PAB_ERR_UNSUPPORTED, "H*W too large");
+    rc = check_ptrs("q, k, v, out", q, k, v, out);
+    if (rc) return rc;
+    return run_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, static_cast<cudaStream_t>(cuda_stream));
     PAB_GUARD_END
 }
 
@@ -485,6 +521,19 @@ int pab_plan_set_temporal_view(pab_plan* plan, int spatial_view) {
     if (!plan) return fail(PAB_ERR_ARG, "null plan");
     if (spatial_view != 0 && spatial_view != 1) return fail(PAB_ERR_ARG, "spatial_view must be 0 or 1");
     plan->temporal_sv = spatial_view;
+    return PAB_OK;
+}
+
+int pab_plan_set_spatial_window(pab_plan* plan, int tile, int win_h, int win_w) {
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    if (win_h == 0 && win_w == 0) {
+        plan->sta_win_h = plan->sta_win_w = 0;
+        return PAB_OK;
+    }
+    int rc = check_sta(plan->H, plan->W, tile, win_h, win_w);
+    if (rc) return rc;
+    plan->sta_win_h = win_h;
+    plan->sta_win_w = win_w;
     return PAB_OK;
 }
 

@@ -33,6 +33,9 @@ class Workload:
     sigma_edge: float = 0.0  # drift on edge steps (0 -> same as sigma)
     seed: int = 0
     extra_ranges: tuple = field(default_factory=tuple)
+    # (tile, win_h, win_w) in tokens when the spatial kind is sliding tile
+    # attention; () for full attention within the frame
+    spatial_window: tuple = field(default_factory=tuple)
 
     @property
     def N(self) -> int:
@@ -70,6 +73,10 @@ WORKLOADS = {
     "temporal_heavy": Workload("temporal_heavy", T=64, H=30, W=40, heads=16, d=64,
                                text_len=120, steps=30, ranges=(2, 4, 6), dtype="bf16",
                                sigma=0.02),
+    # a 720p-class frame rounded up to whole 16 x 16 tiles (768 x 1280 video),
+    # 3 x 3-tile windows: the sliding-tile spatial kind under the PAB schedule
+    "sta_48x80": Workload("sta_48x80", T=24, H=48, W=80, heads=24, d=128, text_len=256, steps=30,
+                          ranges=(2, 4, 6), dtype="bf16", sigma=0.02, spatial_window=(16, 48, 48)),
     "sweep": Workload("sweep", T=16, H=30, W=53, heads=16, d=72, text_len=120, steps=50,
                       ranges=(1, 1, 1), dtype="bf16", sigma=0.02, sigma_edge=0.2,
                       extra_ranges=((1, 1, 1), (2, 3, 4), (2, 4, 6), (3, 6, 9))),

@@ -127,3 +127,119 @@ def test_bad_sta_arguments_are_rejected(oracle_mod, H, W, win_h, win_w):
     x = np.zeros((1, H * W, 8))
     with pytest.raises(ValueError):
         oracle_mod.sta_attention(x, x, x, H, W, 1, TILE, win_h, win_w)
+
+
+# ------------------------------------------------------------------ GPU kernel vs oracle
+def _randn(shape, seed, scale=1.0):
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return (scale * torch.randn(shape, generator=g)).to(torch.bfloat16).cuda()
+
+
+@pytest.fixture(scope="module")
+def pab():
+    import step_reuse_b200
+    assert torch.cuda.is_available()
+    return step_reuse_b200
+
+
+def _no_device_errors(pab):
+    torch.cuda.synchronize()
+    assert pab.device_errors(clear=True) == 0
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("T,H,W,heads,d,win_h,win_w", [
+    (2, 32, 48, 2, 64, 48, 48),     # every tile's window clipped
+    (1, 48, 64, 3, 72, 16, 48),     # d = 72 (V's padding column carries the row sums)
+    (2, 64, 32, 2, 128, 48, 16),
+    (1, 16, 16, 2, 32, 16, 16),     # one tile: four 64-key blocks
+    (1, 48, 80, 2, 128, 48, 48),    # the 48 x 80 frame of the sliding-tile workload
+    (1, 32, 32, 1, 8, 80, 80),      # window beyond the frame on every side
+    (1, 80, 48, 2, 40, 48, 80),
+    (1, 96, 96, 1, 64, 80, 80),     # interior tiles see 25 key tiles (100 blocks)
+])
+def test_sta_kernel_parity(pab, oracle_mod, T, H, W, heads, d, win_h, win_w):
+    from parity import assert_attn_close, check_guards, guarded_empty, to_f64
+    C = heads * d
+    q, k, v = (_randn((T, H * W, C), s) for s in (21, 22, 23))
+    base, out = guarded_empty((T, H * W, C), torch.bfloat16)
+    pab.sta_attention(q, k, v, H, W, heads, TILE, win_h, win_w, out=out)
+    want = oracle_mod.sta_attention(to_f64(q), to_f64(k), to_f64(v), H, W, heads, TILE, win_h, win_w)
+    assert_attn_close(out, want, f"sta T={T} {H}x{W} h={heads} d={d} win {win_h}x{win_w}")
+    check_guards(base)
+    _no_device_errors(pab)
+
+
+@pytest.mark.gpu
+def test_sta_frame_covering_window_is_spatial_attention(pab, oracle_mod):
+    from parity import assert_attn_close, to_f64
+    T, H, W, heads, d = 2, 32, 64, 2, 64
+    C = heads * d
+    q, k, v = (_randn((T, H * W, C), s) for s in (24, 25, 26))
+    out = pab.sta_attention(q, k, v, H, W, heads, TILE, 48, 112)
+    want = oracle_mod.spatial_attention(to_f64(q), to_f64(k), to_f64(v), heads)
+    assert_attn_close(out, want, "sta, window covering the frame")
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("H,W,tile,win_h,win_w,code", [
+    (30, 32, 16, 48, 48, "PAB_ERR_ARG"),          # frame not whole tiles
+    (32, 32, 16, 32, 48, "PAB_ERR_ARG"),          # even tile count
+    (32, 32, 16, 40, 48, "PAB_ERR_ARG"),          # window not whole tiles
+    (32, 32, 8, 24, 24, "PAB_ERR_UNSUPPORTED"),   # another tile size
+])
+def test_sta_rejects_bad_geometry(pab, H, W, tile, win_h, win_w, code):
+    x = _randn((1, H * W, 64), 27)
+    with pytest.raises(pab.PabError) as e:
+        pab.sta_attention(x, x, x, H, W, 1, tile, win_h, win_w)
+    assert e.value.code == getattr(pab, code)
+
+
+@pytest.mark.gpu
+def test_plan_spatial_window_runs_sta_under_the_schedule(pab):
+    """A plan with a spatial window computes sliding tile attention at its
+    computing steps (bit-identical to the stateless call) and serves the
+    cached slot at its broadcast steps."""
+    T, H, W, heads, d, steps = 2, 32, 48, 2, 64, 10
+    C = heads * d
+    plan = pab.Plan(T, H, W, heads, d, 16, steps, (2, 3, 4), dtype=torch.bfloat16)
+    try:
+        plan.set_spatial_window(TILE, 48, 48)
+        last = None
+        for i in range(steps):
+            q, k, v = (_randn((T, H * W, C), 100 * i + s) for s in (1, 2, 3))
+            got = plan.attention("spatial", i, q, k, v)
+            if plan.is_compute("spatial", i):
+                want = pab.sta_attention(q, k, v, H, W, heads, TILE, 48, 48)
+                assert torch.equal(got, want), i
+            else:
+                assert got.data_ptr() == last.data_ptr() and torch.equal(got, last_val), i
+            last, last_val = got, got.clone()
+        plan.reset()
+        plan.set_spatial_window(TILE, 0, 0)  # back to full attention
+        q, k, v = (_randn((T, H * W, C), s) for s in (7, 8, 9))
+        assert torch.equal(plan.attention("spatial", 0, q, k, v), pab.spatial_attention(q, k, v, heads))
+        with pytest.raises(pab.PabError):
+            plan.set_spatial_window(TILE, 32, 48)
+    finally:
+        plan.close()
+    _no_device_errors(pab)
+
+
+@pytest.mark.gpu
+def test_sta_full_size_sampled(pab, oracle_mod):
+    """The sliding-tile workload at full size (24 frames of 48 x 80 tokens,
+    24 heads of d = 128, 3 x 3-tile windows) in the launch the benchmark
+    times; two frames (all heads) against the oracle."""
+    from parity import assert_attn_close, to_f64
+    T, H, W, heads, d = 24, 48, 80, 24, 128
+    C = heads * d
+    q, k, v = (_randn((T, H * W, C), s) for s in (31, 32, 33))
+    out = pab.sta_attention(q, k, v, H, W, heads, TILE, 48, 48)
+    torch.cuda.synchronize()
+    for fr in (0, T - 1):
+        want = oracle_mod.sta_attention(to_f64(q[fr:fr + 1]), to_f64(k[fr:fr + 1]), to_f64(v[fr:fr + 1]),
+                                        H, W, heads, TILE, 48, 48)
+        assert_attn_close(out[fr:fr + 1], want, f"sta full size, frame {fr}")
+    _no_device_errors(pab)
