@@ -45,8 +45,10 @@ UNIT = "TFLOP/s (dense-equivalent attention)"
 # keyed by (sha256 of the kernel's source, workload); a different source hash
 # or a workload without a capture means traffic is null.
 MEASURED_TRAFFIC = {
-    # flash_tc spatial, 480p-like, 1 launch: dram read 176.15 MB + write 42.39 MB
-    ("ca2dcfe83a42d92b", "480p"): 218539520,
+    # flash_tc spatial, 480p-like, 1 launch: dram read 175.92 MB + write 42.11 MB
+    ("07d5ce460e633017", "480p"): 218031104,
+    # flash_tc sliding tile attention, sta_48x80, 1 launch: read 1698.89 MB + write 547.61 MB
+    ("07d5ce460e633017", "sta_48x80"): 2246495296,
 }
 
 
@@ -782,8 +784,10 @@ def run_sta(args):
                            l2=f"inputs larger than L2 ({n_sets} input sets cycled)"),
             "roofline": {"kernel": "sliding tile attention (flash_tc, window geometry)", "bound": "tensor",
                          "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
-                         "traffic": None, "peak_source": f"{peak_src} bf16_tflops_sustained",
-                         "algorithmic_flops_per_launch": sta_flops},
+                         "traffic": MEASURED_TRAFFIC.get((kernel_source_hash("flash_tc.cu"), name)),
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "algorithmic_flops_per_launch": sta_flops,
+                         "algorithmic_bytes_per_launch": 4 * T * N * C * 2},
             "kernel_ms": {"sta": kern["sta"], "full_spatial": kern["full"]},
             "window_share_of_full": sta_flops / full_flops,
             "kernel_speedup_vs_full": kern["full"] / kern["sta"],
