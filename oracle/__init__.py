@@ -22,7 +22,11 @@ What each function computes (sources are the PAB pages):
   * sta_attention -- sliding tile attention as the spatial kind (sgqg.cn
     summary of "Fast Video Generation with Sliding Tile Attention", section
     "Sliding Tile Attention (STA)"): 2-D tiles per frame, a window of whole
-    tiles centred on the query's tile, cut off at the frame edge.
+    tiles centred on the query's tile, cut off at the frame edge;
+  * draft_select / region_sparse_attention / draft_attention -- draft
+    attention as the spatial kind (crisp3r.com article on "Draft Attention",
+    steps 1-4): pooled region sketch, draft scores, the best key regions of
+    each query region, attention restricted to them.
 """
 from __future__ import annotations
 
@@ -62,6 +66,8 @@ def _load():
         lib.oracle_temporal_attention.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 4
         lib.oracle_cross_attention.argtypes = [_dp, _dp, _dp, _dp, ctypes.c_long] + [ctypes.c_int] * 3
         lib.oracle_sta_attention.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 8
+        lib.oracle_draft_select.argtypes = [_dp, _dp] + [ctypes.c_int] * 7 + [_ip]
+        lib.oracle_region_sparse_attention.argtypes = [_dp, _dp, _dp, _dp] + [ctypes.c_int] * 7 + [_ip]
         lib.oracle_pab_edge_steps.argtypes = [ctypes.c_int, ctypes.c_int]
         lib.oracle_pab_schedule.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, _ip, _ip]
         lib.oracle_mse.argtypes = [_dp, _dp, ctypes.c_long]
@@ -69,7 +75,8 @@ def _load():
         lib.oracle_layout.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 4
         lib.oracle_num_threads.restype = ctypes.c_int
         for name in ("oracle_spatial_attention", "oracle_temporal_attention",
-                     "oracle_cross_attention", "oracle_sta_attention", "oracle_pab_edge_steps",
+                     "oracle_cross_attention", "oracle_sta_attention", "oracle_draft_select",
+                     "oracle_region_sparse_attention", "oracle_pab_edge_steps",
                      "oracle_pab_schedule", "oracle_layout", "oracle_num_threads"):
             if getattr(lib, name).restype is not ctypes.c_double:
                 getattr(lib, name).restype = ctypes.c_int
@@ -145,6 +152,49 @@ def sta_attention(q, k, v, H: int, W: int, heads: int, tile: int, win_h: int, wi
     if rc != 0:
         raise RuntimeError(f"oracle_sta_attention failed ({rc})")
     return o
+
+
+def draft_select(q, k, H: int, W: int, heads: int, region: int, keep: int) -> np.ndarray:
+    """Draft attention's region selection: q, k [T, H*W, C] -> int32
+    [T, heads, R, keep], R = (H/region)(W/region): per query region the
+    `keep` key regions with the highest pooled-sketch scores (ties to the
+    lower index), listed in ascending region index."""
+    q, k = _f64(q), _f64(k)
+    T, N, C = q.shape
+    assert N == H * W and k.shape == q.shape and C % heads == 0
+    R = (H // region) * (W // region) if region > 0 and H % region == 0 and W % region == 0 else 0
+    sel = np.zeros((T, heads, max(R, 1), max(keep, 1)), dtype=np.int32)
+    rc = _load().oracle_draft_select(_ptr(q), _ptr(k), T, H, W, heads, C // heads, region, keep,
+                                     sel.ctypes.data_as(_ip))
+    if rc == -1:
+        raise ValueError("bad draft-attention arguments")
+    if rc != 0:
+        raise RuntimeError(f"oracle_draft_select failed ({rc})")
+    return sel
+
+
+def region_sparse_attention(q, k, v, H: int, W: int, heads: int, region: int, sel) -> np.ndarray:
+    """Attention of every query region over the key regions sel lists
+    ([T, heads, R, keep] int): q, k, v [T, H*W, C] -> out [T, H*W, C]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    sel = np.ascontiguousarray(np.asarray(sel, dtype=np.int32))
+    T, N, C = q.shape
+    assert N == H * W and k.shape == q.shape and v.shape == q.shape and C % heads == 0
+    keep = sel.shape[-1]
+    o = np.empty_like(q)
+    rc = _load().oracle_region_sparse_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(o), T, H, W, heads,
+                                                C // heads, region, keep, sel.ctypes.data_as(_ip))
+    if rc == -1:
+        raise ValueError("bad region-sparse attention arguments")
+    if rc != 0:
+        raise RuntimeError(f"oracle_region_sparse_attention failed ({rc})")
+    return o
+
+
+def draft_attention(q, k, v, H: int, W: int, heads: int, region: int, keep: int) -> np.ndarray:
+    """Draft attention within each frame: the selection of draft_select, then
+    region_sparse_attention under it."""
+    return region_sparse_attention(q, k, v, H, W, heads, region, draft_select(q, k, H, W, heads, region, keep))
 
 
 def edge_steps(steps: int, edge_pct: int = 15) -> int:

@@ -237,6 +237,155 @@ int oracle_sta_attention(const double *q, const double *k, const double *v,
     return bad ? -2 : 0;
 }
 
+/* Draft attention as the spatial kind: crisp3r.com article on "Draft
+ * Attention" (low-resolution attention guidance), its steps 1-4 -- the
+ * latent frame is average-pooled into a low-resolution sketch of the queries
+ * and keys, the draft attention map of the sketch ranks regions, the
+ * best-scoring regions form a structured sparse mask for the full-resolution
+ * attention, and tokens are grouped so the kept blocks are contiguous.
+ * Readings: regions of `region` x `region` tokens per frame; the sketch of a
+ * region is the mean of its tokens' q (and k) per head; the draft score of
+ * query region i and key region j is qbar_i . kbar_j / sqrt(d) (the draft
+ * softmax is monotone along a row, so ranking scores ranks the map); every
+ * query region keeps its `keep` best key regions, ties to the lower region
+ * index; the selection is listed in ascending region index.
+ * sel: [T][heads][R][keep] with R = (H/region) * (W/region). */
+int oracle_draft_select(const double *q, const double *k, int T, int H, int W, int heads, int d,
+                        int region, int keep, int *sel)
+{
+    if (T < 0 || H < 0 || W < 0 || heads <= 0 || d <= 0 || region <= 0)
+        return -1;
+    if (H % region || W % region)
+        return -1;
+    const int rw = W / region, R = (H / region) * rw;
+    if (keep < 1 || keep > R)
+        return -1;
+    const long C = (long)heads * d;
+    const long N = (long)H * W;
+    const double scale = 1.0 / sqrt((double)d);
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *qb = (double *)malloc(sizeof(double) * (size_t)R * d);
+        double *kb = (double *)malloc(sizeof(double) * (size_t)R * d);
+        double *sc = (double *)malloc(sizeof(double) * (size_t)R);
+        char *taken = (char *)malloc((size_t)R);
+        if (!qb || !kb || !sc || !taken) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for collapse(2) schedule(dynamic)
+            for (int t = 0; t < T; ++t)
+                for (int h = 0; h < heads; ++h) {
+                    /* step 1: the sketch -- per region, the mean of q and of k */
+                    for (int r = 0; r < R; ++r) {
+                        const int y0 = (r / rw) * region, x0 = (r % rw) * region;
+                        for (int c = 0; c < d; ++c) {
+                            double sq = 0.0, sk = 0.0;
+                            for (int y = y0; y < y0 + region; ++y)
+                                for (int x = x0; x < x0 + region; ++x) {
+                                    const long at = (long)t * N * C + ((long)y * W + x) * C + (long)h * d + c;
+                                    sq += q[at];
+                                    sk += k[at];
+                                }
+                            qb[(long)r * d + c] = sq / ((double)region * region);
+                            kb[(long)r * d + c] = sk / ((double)region * region);
+                        }
+                    }
+                    /* steps 2-3: draft scores of each query region, keep the best */
+                    for (int i = 0; i < R; ++i) {
+                        for (int j = 0; j < R; ++j) {
+                            double s = 0.0;
+                            for (int c = 0; c < d; ++c)
+                                s += qb[(long)i * d + c] * kb[(long)j * d + c];
+                            sc[j] = s * scale;
+                            taken[j] = 0;
+                        }
+                        for (int n = 0; n < keep; ++n) {
+                            int best = -1;
+                            for (int j = 0; j < R; ++j)
+                                if (!taken[j] && (best < 0 || sc[j] > sc[best]))
+                                    best = j;
+                            taken[best] = 1;
+                        }
+                        int *row = sel + (((long)t * heads + h) * R + i) * keep;
+                        int n = 0;
+                        for (int j = 0; j < R; ++j)
+                            if (taken[j])
+                                row[n++] = j;
+                    }
+                }
+        }
+        free(qb);
+        free(kb);
+        free(sc);
+        free(taken);
+    }
+    return bad ? -2 : 0;
+}
+
+/* Full-resolution attention under a region selection (step 3's sparse
+ * mask): every query of region i attends to the tokens of the key regions
+ * sel[t][h][i][0..keep), gathered in list order then row-major within a
+ * region, with the textbook definition. */
+int oracle_region_sparse_attention(const double *q, const double *k, const double *v, double *o,
+                                   int T, int H, int W, int heads, int d, int region, int keep,
+                                   const int *sel)
+{
+    if (T < 0 || H < 0 || W < 0 || heads <= 0 || d <= 0 || region <= 0)
+        return -1;
+    if (H % region || W % region)
+        return -1;
+    const int rw = W / region, R = (H / region) * rw;
+    if (keep < 1 || keep > R)
+        return -1;
+    for (long i = 0; i < (long)T * heads * R * keep; ++i)
+        if (sel[i] < 0 || sel[i] >= R)
+            return -1;
+    const long C = (long)heads * d;
+    const long N = (long)H * W;
+    const long maxkeys = (long)keep * region * region;
+    int bad = 0;
+#pragma omp parallel
+    {
+        double *p = (double *)malloc(sizeof(double) * maxkeys);
+        double *kw = (double *)malloc(sizeof(double) * (size_t)maxkeys * d);
+        double *vw = (double *)malloc(sizeof(double) * (size_t)maxkeys * d);
+        if (!p || !kw || !vw) {
+#pragma omp atomic write
+            bad = 1;
+        } else {
+#pragma omp for collapse(3) schedule(dynamic)
+            for (int t = 0; t < T; ++t)
+                for (int h = 0; h < heads; ++h)
+                    for (int i = 0; i < R; ++i) {
+                        const int *row = sel + (((long)t * heads + h) * R + i) * keep;
+                        const long frame = (long)t * N * C + (long)h * d;
+                        int nk = 0;
+                        for (int n = 0; n < keep; ++n) {
+                            const int y0 = (row[n] / rw) * region, x0 = (row[n] % rw) * region;
+                            for (int y = y0; y < y0 + region; ++y)
+                                for (int x = x0; x < x0 + region; ++x, ++nk) {
+                                    const long src = frame + ((long)y * W + x) * C;
+                                    memcpy(kw + (long)nk * d, k + src, sizeof(double) * d);
+                                    memcpy(vw + (long)nk * d, v + src, sizeof(double) * d);
+                                }
+                        }
+                        const int y0 = (i / rw) * region, x0 = (i % rw) * region;
+                        for (int y = y0; y < y0 + region; ++y)
+                            for (int x = x0; x < x0 + region; ++x) {
+                                const long at = frame + ((long)y * W + x) * C;
+                                attend_one_query(q + at, kw, d, vw, d, nk, d, o + at, p);
+                            }
+                    }
+        }
+        free(p);
+        free(kw);
+        free(vw);
+    }
+    return bad ? -2 : 0;
+}
+
 /* ------------------------------------------------------------------------ */
 /* PAB schedule, walked step by step in execution order (noisiest first).    */
 /*   edge steps (first and last edge_pct%): always compute;                  */
