@@ -58,7 +58,7 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
-    ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny", "sta_48x80"))
+    ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny", "sta_48x80", "draft_48x80"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=2)
@@ -70,6 +70,10 @@ def parse_args(argv=None):
                     help="sliding tile attention as the spatial kind (workload sta_48x80 unless "
                          "--workload names another with a spatial window): the kernel against full "
                          "spatial attention, and the PAB stack with each")
+    ap.add_argument("--draft", action="store_true",
+                    help="draft attention as the spatial kind (workload draft_48x80): pooled sketch and "
+                         "selection, region-sparse attention against full spatial attention, and the PAB "
+                         "stack with each")
     ap.add_argument("--dit", action="store_true",
                     help="time the synthetic DiT block (projections, norms, MLP around the library's "
                          "attention) with the workload's PAB ranges and with ranges (1, 1, 1)")
@@ -216,7 +220,7 @@ class AttentionStack:
     fused=True: the temporal kernel reads and writes the spatial view itself
     (pab_plan_set_temporal_view), no layout launches."""
 
-    def __init__(self, pab, w, device, fused=False, window=()):
+    def __init__(self, pab, w, device, fused=False, window=(), draft=()):
         self.pab, self.w, self.dev, self.fused = pab, w, device, fused
         self.plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges,
                              dtype=torch.bfloat16)
@@ -224,6 +228,8 @@ class AttentionStack:
             self.plan.set_temporal_view(True)
         if window:
             self.plan.set_spatial_window(*window)
+        if draft:
+            self.plan.set_spatial_draft(*draft)
         self.plan.prepare()
         T, N, C = w.T, w.N, w.C
         # temporal-view scratch and the spatial-view copy of the temporal output
@@ -795,7 +801,134 @@ def run_sta(args):
             "stack": {k: dict(v, denoising_steps_per_s=world * w.steps / (v["ms_per_run"] * 1e-3))
                       for k, v in stacks.items()},
             "stack_speedup_vs_full": stacks["full"]["ms_per_run"] / stacks["sta"]["ms_per_run"],
-            "gpu_launches": reps,
+            # timed launches: the two kernel loops, then `runs` runs of each stack
+            "gpu_launches": 2 * reps + runs * sum(v["gpu_launches_per_run"] for v in stacks.values()),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+def run_draft(args):
+    """Draft attention as the spatial kind: the pooled-sketch selection and
+    the region-sparse attention against full spatial attention on the same
+    tensors, then one PAB sampling run of the fused stack with each;
+    device-timed; one JSON line."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    import step_reuse_b200 as pab
+
+    name = args.workload if synth.WORKLOADS[args.workload].spatial_draft else "draft_48x80"
+    w = synth.WORKLOADS[name]
+    region, keep = w.spatial_draft
+    T, N, C = w.T, w.N, w.C
+    R = (w.H // region) * (w.W // region)
+    sparse_flops = 4.0 * T * w.heads * w.d * R * keep * (region * region) ** 2
+    full_flops = w.flops()["spatial"]
+    pool_bytes = 2 * T * N * C * 2 + 2 * T * R * C * 4  # q, k read; the fp32 sketch written
+    n_sets = max(1, min(w.steps, args.input_sets))
+    inputs = make_inputs(w, device, n_sets, seed=rank)
+    stream = torch.cuda.current_stream(device)
+    out = torch.empty((T, N, C), dtype=torch.bfloat16, device=device)
+    sel = torch.empty((T, w.heads, R, keep), dtype=torch.int32, device=device)
+    ws = torch.empty(pab.draft_workspace_bytes(T, w.H, w.W, w.heads, w.d, region), dtype=torch.uint8,
+                     device=device)
+    launches = {
+        "select": lambda x: pab.draft_select(x["q"], x["k"], w.H, w.W, w.heads, keep, region, sel=sel,
+                                             workspace=ws, stream=stream),
+        "sparse": lambda x: pab.region_sparse_attention(x["q"], x["k"], x["v"], w.H, w.W, w.heads, sel, region,
+                                                        out=out, stream=stream),
+        "full": lambda x: pab.spatial_attention(x["q"], x["k"], x["v"], w.heads, out=out, stream=stream),
+    }
+    reps = max(5, args.steps)
+    kern = {}
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.5)
+    clocks.mark_start()
+    for label, fn in launches.items():
+        for i in range(args.warmup):
+            fn(inputs[i % n_sets]["spatial"])
+        torch.cuda.synchronize(device)
+        barrier(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(reps):
+            fn(inputs[i % n_sets]["spatial"])
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        kern[label] = max_over_ranks(a.elapsed_time(b) / reps, device)
+    assert pab.device_errors() == 0
+    runs = max(3, args.steps // 10)
+    stacks = {}
+    for label, draft in (("draft", w.spatial_draft), ("full", ())):
+        st = AttentionStack(pab, w, device, fused=True, draft=draft)
+        for _ in range(args.warmup):
+            st.run(inputs, stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(runs):
+            st.run(inputs, stream)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        extra = st.launches_per_run
+        if draft:  # each spatial compute is three launches: pool, select, region-sparse attention
+            extra += 2 * sum(st.sched["spatial"])
+        stacks[label] = {"ms_per_run": max_over_ranks(a.elapsed_time(b) / runs, device),
+                         "gpu_launches_per_run": extra}
+        st.close()
+    clocks.mark_end()
+    clk = clocks.stop()
+    assert pab.device_errors() == 0
+
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        peak_src = "measured"
+    except (OSError, ValueError):
+        peak_src = "fallback"
+    tc_peak = peaks.get("bf16_tflops_sustained", 1400.0)
+    hbm_peak = peaks.get("hbm_gbs", 6650.0)
+    achieved = sparse_flops / (kern["sparse"] * 1e-3) / 1e12
+    total_ms = kern["select"] + kern["sparse"]
+    if rank == 0:
+        line = {
+            "metric": "draft attention as the spatial kind: region-sparse TFLOP/s (kept pairs) and PAB stack "
+                      "steps/s",
+            "value": world * sparse_flops / (total_ms * 1e-3) / 1e12,
+            "unit": "TFLOP/s (algorithmic, kept regions; selection included)",
+            "n_gpus": world, "steps": reps, "warmup": args.warmup, "higher_is_better": True, "scaling": "weak",
+            "dtype": "bf16", "data": "synthetic",
+            "config": dict(workload_config(w), spatial_draft={"region": region, "keep": keep, "regions": R},
+                           l2=f"inputs larger than L2 ({n_sets} input sets cycled)"),
+            "roofline": {"kernel": "region-sparse attention (flash_tc, list geometry)", "bound": "tensor",
+                         "achieved": achieved, "peak": tc_peak, "unit": "TFLOP/s", "frac": achieved / tc_peak,
+                         "traffic": MEASURED_TRAFFIC.get((kernel_source_hash("flash_tc.cu"), name)),
+                         "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "algorithmic_flops_per_launch": sparse_flops},
+            "select_roofline": {"kernel": "draft pool + select", "bound": "hbm",
+                                "achieved": pool_bytes / (kern["select"] * 1e-3) / 1e9, "peak": hbm_peak,
+                                "unit": "GB/s", "frac": pool_bytes / (kern["select"] * 1e-3) / 1e9 / hbm_peak,
+                                "algorithmic_bytes_per_launch": pool_bytes},
+            "kernel_ms": {"select": kern["select"], "sparse": kern["sparse"], "full_spatial": kern["full"]},
+            "kept_share_of_full": sparse_flops / full_flops,
+            "speedup_vs_full": kern["full"] / total_ms,
+            "full_spatial_tflops": full_flops / (kern["full"] * 1e-3) / 1e12,
+            "stack": {k: dict(v, denoising_steps_per_s=world * w.steps / (v["ms_per_run"] * 1e-3))
+                      for k, v in stacks.items()},
+            "stack_speedup_vs_full": stacks["full"]["ms_per_run"] / stacks["draft"]["ms_per_run"],
+            # timed launches: pool + select, region-sparse and full loops, then `runs` runs of each stack
+            "gpu_launches": 4 * reps + runs * sum(v["gpu_launches_per_run"] for v in stacks.values()),
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
@@ -810,6 +943,8 @@ def main(argv=None):
         return run_reference(args)
     if args.sta:
         return run_sta(args)
+    if args.draft:
+        return run_draft(args)
     if args.dit:
         return run_dit(args)
     return run_ours(args)

@@ -99,6 +99,34 @@ int pab_spatial_attention(const void* q, const void* k, const void* v, void* out
 int pab_sta_attention(const void* q, const void* k, const void* v, void* out, int T, int H, int W,
                       int heads, int d, int tile, int win_h, int win_w, void* cuda_stream);
 
+/* Draft attention as the spatial kind (crisp3r.com article on "Draft
+ * Attention", steps 1-4: a pooled low-resolution sketch of the queries and
+ * keys, its draft attention map, the best regions as a structured sparse
+ * mask, kept blocks contiguous).  Two calls:
+ *
+ * pab_draft_select: per frame, average-pool q and k ([T, H*W, C], bf16) over
+ * region x region-token regions (R = (H/region)(W/region) per frame); the
+ * draft score of query region i and key region j for head h is
+ * qbar_i . kbar_j / sqrt(d); every query region keeps the `keep` key regions
+ * with the highest scores (equal scores: the lower index), written to sel
+ * ([T, heads, R, keep] int32, device memory, ascending index per row).
+ * Means and scores are fp32.  workspace: device scratch of at least
+ * pab_draft_workspace_bytes(...) bytes, 16-byte aligned, owned by the
+ * caller.  region must be 16; H, W multiples of 16; 1 <= keep <= R <= 4096.
+ *
+ * pab_region_sparse_attention: every query of region i attends to the tokens
+ * of the key regions sel[t][h][i][0..keep) (softmax over those only).  sel
+ * may come from pab_draft_select or from the caller; an index outside
+ * [0, R) sets bit 2 of pab_device_errors and is clamped.
+ * Keeping every region (keep = R) gives pab_spatial_attention's result.
+ * PAB_BF16 only. */
+int pab_draft_workspace_bytes(int T, int H, int W, int heads, int d, int region, long long* bytes);
+int pab_draft_select(const void* q, const void* k, int T, int H, int W, int heads, int d, int region,
+                     int keep, int* sel, void* workspace, long long workspace_bytes, void* cuda_stream);
+int pab_region_sparse_attention(const void* q, const void* k, const void* v, void* out, int T, int H,
+                                int W, int heads, int d, int region, int keep, const int* sel,
+                                void* cuda_stream);
+
 /* Temporal attention (same section: attention across frames).
  * q, k, v, out: [N, T, C] (the temporal view).  For each position n, head h:
  *   out[n, t, h] = sum_s softmax_s(q[n, t, h] . k[n, s, h] / sqrt(d)) v[n, s, h].
@@ -173,8 +201,10 @@ int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long n, int dty
 
 /* Device status word of the kernels that wait on asynchronous copies: bit 0
  * is set when a bounded wait gave up (the kernel then returns early and its
- * output is incomplete).  Synchronises the device to read it; clear != 0
- * resets it.  A healthy run reads 0. */
+ * output is incomplete); bit 2 when a region index read from device memory
+ * (pab_region_sparse_attention's selection) lay outside the frame (it was
+ * clamped; that output is not meaningful).  Synchronises the device to read
+ * it; clear != 0 resets it.  A healthy run reads 0. */
 int pab_device_errors(int clear, unsigned int* flags);
 
 /* ---------------------------------------------------------------------- */
@@ -210,6 +240,13 @@ int pab_plan_set_temporal_view(pab_plan* plan, int spatial_view);
  * full attention.  Same argument rules as pab_sta_attention.  Call before
  * the run starts (the broadcast schedule and cache are unchanged). */
 int pab_plan_set_spatial_window(pab_plan* plan, int tile, int win_h, int win_w);
+
+/* Make this plan's SPATIAL computes draft attention (pab_draft_select then
+ * pab_region_sparse_attention with the plan's H, W, region and keep; the
+ * plan owns the scratch and the selection); keep = 0 restores full
+ * attention.  A spatial window (pab_plan_set_spatial_window) and a draft
+ * setting replace each other.  Same argument rules as pab_draft_select. */
+int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep);
 
 /* Allocate the cache (2 output slots per kind, plus bf16 staging for
  * PAB_FP32 plans) on the current device now instead of at each kind's first

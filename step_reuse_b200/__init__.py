@@ -34,7 +34,8 @@ BF16, FP32 = 0, 1
 EXPORTS = (
     "pab_version", "pab_last_error_string", "pab_spatial_attention", "pab_temporal_attention",
     "pab_temporal_attention_sv", "pab_plan_set_temporal_view", "pab_sta_attention",
-    "pab_plan_set_spatial_window",
+    "pab_plan_set_spatial_window", "pab_draft_workspace_bytes", "pab_draft_select",
+    "pab_region_sparse_attention", "pab_plan_set_spatial_draft",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
     "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
@@ -67,6 +68,10 @@ def _load() -> ctypes.CDLL:
         "pab_plan_set_temporal_view": ([vp, i], i),
         "pab_sta_attention": ([vp, vp, vp, vp, i, i, i, i, i, i, i, i, vp], i),
         "pab_plan_set_spatial_window": ([vp, i, i, i], i),
+        "pab_draft_workspace_bytes": ([i, i, i, i, i, i, ctypes.POINTER(ll)], i),
+        "pab_draft_select": ([vp, vp, i, i, i, i, i, i, i, vp, vp, ll, vp], i),
+        "pab_region_sparse_attention": ([vp, vp, vp, vp, i, i, i, i, i, i, i, vp, vp], i),
+        "pab_plan_set_spatial_draft": ([vp, i, i], i),
         "pab_cross_attention": ([vp, vp, vp, vp, ll, i, i, i, vp], i),
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
         "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
@@ -146,6 +151,51 @@ def sta_attention(q, k, v, H: int, W: int, heads: int, tile: int = 16, win_h: in
     _check(lib.pab_sta_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), T, H, W, heads, C // heads,
                                  tile, win_h, win_w, _stream(stream)))
     return out
+
+
+def draft_workspace_bytes(T: int, H: int, W: int, heads: int, d: int, region: int = 16) -> int:
+    n = ctypes.c_longlong(0)
+    _check(lib.pab_draft_workspace_bytes(T, H, W, heads, d, region, ctypes.byref(n)))
+    return n.value
+
+
+def draft_select(q, k, H: int, W: int, heads: int, keep: int, region: int = 16, sel=None, workspace=None,
+                 stream=None):
+    """Draft attention's region selection: q, k [T, H*W, C] bf16 CUDA tensors
+    -> int32 [T, heads, R, keep] (per query region the keep key regions with
+    the highest pooled-sketch scores, ascending)."""
+    T, N, C = q.shape
+    if N != H * W:
+        raise ValueError(f"q has {N} tokens per frame, H*W = {H * W}")
+    R = (H // region) * (W // region)
+    if sel is None:
+        sel = torch.empty((T, heads, R, keep), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(draft_workspace_bytes(T, H, W, heads, C // heads, region),
+                                dtype=torch.uint8, device=q.device)
+    _check(lib.pab_draft_select(_ptr(q), _ptr(k), T, H, W, heads, C // heads, region, keep, _ptr(sel),
+                                _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)))
+    return sel
+
+
+def region_sparse_attention(q, k, v, H: int, W: int, heads: int, sel, region: int = 16, out=None, stream=None):
+    """Attention of every query region over the key regions sel
+    ([T, heads, R, keep] int32 CUDA tensor) lists: q, k, v [T, H*W, C]."""
+    T, N, C = q.shape
+    if N != H * W:
+        raise ValueError(f"q has {N} tokens per frame, H*W = {H * W}")
+    if sel.dtype != torch.int32 or not sel.is_contiguous():
+        raise ValueError("sel must be a contiguous int32 tensor")
+    out = torch.empty_like(q) if out is None else out
+    _check(lib.pab_region_sparse_attention(_ptr(q), _ptr(k), _ptr(v), _ptr(out), T, H, W, heads, C // heads,
+                                           region, sel.shape[-1], _ptr(sel), _stream(stream)))
+    return out
+
+
+def draft_attention(q, k, v, H: int, W: int, heads: int, keep: int, region: int = 16, stream=None):
+    """Draft attention within each frame: draft_select then region_sparse_attention."""
+    sel = draft_select(q, k, H, W, heads, keep, region, stream=stream)
+    return region_sparse_attention(q, k, v, H, W, heads, sel, region, stream=stream)
 
 
 def temporal_attention(q, k, v, heads: int, out=None, stream=None):
@@ -265,6 +315,11 @@ class Plan:
         """Spatial computes become sliding tile attention with this window
         (win_h = win_w = 0: full attention within the frame again)."""
         _check(lib.pab_plan_set_spatial_window(self._h, tile, win_h, win_w))
+
+    def set_spatial_draft(self, region: int = 16, keep: int = 0):
+        """Spatial computes become draft attention keeping `keep` key regions
+        per query region (keep = 0: full attention within the frame again)."""
+        _check(lib.pab_plan_set_spatial_draft(self._h, region, keep))
 
     def prepare(self):
         _check(lib.pab_plan_prepare(self._h))

@@ -15,6 +15,7 @@ namespace pab {
 enum : unsigned int {
     kDevErrWaitTimeout = 1u,  // a bounded wait on an mbarrier gave up
     kDevErrBadLaunch = 2u,    // launch geometry did not match the plan
+    kDevErrBadIndex = 4u,     // an index read from device memory was out of range (clamped)
 };
 
 // A wait that has not completed after this many nanoseconds is abandoned.

@@ -82,10 +82,19 @@ struct FlashTcArgs {
     int kv_batched;    // 1: K/V have a batch coordinate (spatial); 0: shared (cross)
     int d;             // head dim
     float scale_log2;  // log2(e) / sqrt(d)
-    // sliding tile attention only: the frame in 16 x 16 tiles and the
-    // window's reach in tiles on each side of the query tile
+    // tile geometries only: the frame in 16 x 16 tiles; the window's reach
+    // in tiles on each side of the query tile (window geometry); the key
+    // tiles of every query tile, [batches][heads][tiles][kv_count] (list
+    // geometry)
     int tiles_h, tiles_w, reach_h, reach_w;
+    const int* kv_list;
+    int kv_count;
 };
+
+// Key geometries of the flash kernel: every key of the (frame, head) row
+// range; the window of 16 x 16 tiles around the query tile (sliding tile
+// attention); a per-query-tile list of 16 x 16 key tiles (draft attention).
+enum { kGeoFull = 0, kGeoWindow = 1, kGeoList = 2 };
 
 constexpr int kMaxStages = 8;
 
@@ -162,13 +171,14 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
 // column inside the PV product's N = 16 * KSTEPS -- is set to 1 once the tile
 // lands (warp 11), so O's column d accumulates the row sum of P with the same
 // bf16 P as the numerator; the softmax then keeps no running sum.
-// STA (sliding tile attention): the CTA's 256 queries are one 16 x 16 tile
-// of the frame (tile A its upper 8 rows, tile B the lower 8, each read as a
-// [8][16]-token TMA box of the [H][W] grid), and the key loop runs over the
-// 16 x 16 key tiles of the window around it, clipped at the frame edge, each
-// as four [4][16]-token blocks of 64 keys.  Every block is whole, so nothing
-// is masked.
-template <int KSTEPS, int NST, bool ONES, bool STA>
+// Tile geometries (GEO != kGeoFull): the CTA's 256 queries are one 16 x 16
+// tile of the frame (tile A its upper 8 rows, tile B the lower 8, each read
+// as a [8][16]-token TMA box of the [H][W] grid), and the key loop runs over
+// 16 x 16 key tiles, each as four [4][16]-token blocks of 64 keys: the tiles
+// of the window around the query tile, clipped at the frame edge (window),
+// or the tiles listed for it (list; an index outside the frame raises the
+// error word and is clamped).  Every block is whole, so nothing is masked.
+template <int KSTEPS, int NST, bool ONES, int GEO>
 __global__ void __launch_bounds__(kThreads, 1)
     flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
@@ -189,20 +199,28 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int qblk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    // STA geometry: query tile (ty, tx); window tiles [wy0, wy0 + rows) x [wx0, wx0 + cols)
+    // tile geometries: query tile (ty, tx); window tiles [wy0, wy0 + rows) x
+    // [wx0, wx0 + wcols); the list of key tiles
+    constexpr bool TILED = GEO != kGeoFull;
     int ty = 0, tx = 0, wy0 = 0, wx0 = 0, wcols = 1, nkv;
-    if constexpr (STA) {
+    const int* klist = nullptr;
+    if constexpr (TILED) {
         ty = qblk / a.tiles_w;
         tx = qblk - ty * a.tiles_w;
+    }
+    if constexpr (GEO == kGeoWindow) {
         wy0 = max(ty - a.reach_h, 0);
         wx0 = max(tx - a.reach_w, 0);
         const int wy1 = min(ty + a.reach_h + 1, a.tiles_h), wx1 = min(tx + a.reach_w + 1, a.tiles_w);
         wcols = wx1 - wx0;
         nkv = (wy1 - wy0) * wcols * 4;
+    } else if constexpr (GEO == kGeoList) {
+        klist = a.kv_list + (((long long)b * gridDim.y + h) * gridDim.x + qblk) * a.kv_count;
+        nkv = a.kv_count * 4;
     } else {
         nkv = (a.Lk + kBN - 1) / kBN;
     }
-    const bool has_b = STA || qblk * 2 * kBM + kBM < a.Lq;
+    const bool has_b = TILED || qblk * 2 * kBM + kBM < a.Lq;
     const int ntiles = has_b ? 2 : 1;
 
     if (threadIdx.x == 256) {
@@ -238,14 +256,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int kvb = a.kv_batched ? b : 0;
     // TMA coordinates of query tile x's box and of key block j's box
     auto load_q = [&](uint32_t dst, int x, int bx, uint32_t bar) {
-        if constexpr (STA)
+        if constexpr (TILED)
             tc::tma_load_5d(dst, &tm_q, bx * 64, h, tx * 16, ty * 16 + x * 8, b, bar);
         else
             tc::tma_load_4d(dst, &tm_q, bx * 64, h, (qblk * 2 + x) * kBM, b, bar);
     };
     auto load_kv = [&](uint32_t dst, const CUtensorMap* m, int j, int bx, uint32_t bar) {
-        if constexpr (STA) {
+        if constexpr (GEO == kGeoWindow) {
             const int t = j >> 2, ky = wy0 + t / wcols, kx = wx0 + t % wcols;
+            tc::tma_load_5d(dst, m, bx * 64, h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
+        } else if constexpr (GEO == kGeoList) {
+            int tile = __ldg(klist + (j >> 2));
+            if (tile < 0 || tile >= a.tiles_h * a.tiles_w) {
+                atomicOr(&g_flash_err, kDevErrBadIndex);
+                tile = tile < 0 ? 0 : a.tiles_h * a.tiles_w - 1;
+            }
+            const int ky = tile / a.tiles_w, kx = tile - ky * a.tiles_w;
             tc::tma_load_5d(dst, m, bx * 64, h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
         } else {
             tc::tma_load_4d(dst, m, bx * 64, h, j * kBN, kvb, bar);
@@ -387,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ok = wait_bar(&bars, &bars.slot_done[(j - 2) % NST][x], ((j - 2) / NST) & 1);
             if (!ok) break;
             tc::fence_after_sync();
-            const int valid = STA ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
+            const int valid = TILED ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
             // the row's 64 scores fit in registers: one TMEM read
             float sv[kBN];
             {
@@ -516,7 +542,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::named_bar_sync(1 + x, 128);
         if (ok && row == 0) {
             for (int bx = 0; bx < NB; ++bx) {
-                if constexpr (STA)
+                if constexpr (TILED)
                     tc::tma_store_5d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, tx * 16, ty * 16 + x * 8, b);
                 else
                     tc::tma_store_4d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
@@ -585,38 +611,38 @@ bool make_map_grid(CUtensorMap* m, const void* base, int d, int heads, int H, in
     return r == CUDA_SUCCESS;
 }
 
-template <int KSTEPS, bool ONES, bool STA>
+template <int KSTEPS, bool ONES, int GEO>
 cudaError_t launch_ks1(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                        const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     constexpr int NB = (KSTEPS + 3) / 4;
     constexpr int NST = NB == 1 ? 6 : 4;  // ring slots of (V_j, K_{j+2})
     const size_t smem = (size_t)NB * (2 * kQBox + (2 + 2 * NST) * kKVBox) + 1024;
     const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST, ONES, STA>,
+    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST, ONES, GEO>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
     if (e != cudaSuccess) return e;
-    flash_tc_kernel<KSTEPS, NST, ONES, STA><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    flash_tc_kernel<KSTEPS, NST, ONES, GEO><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
     return cudaGetLastError();
 }
-template <int KSTEPS, bool STA>
+template <int KSTEPS, int GEO>
 cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     // a padding column inside the PV product carries the row sums when d % 16 != 0
-    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true, STA>(mq, mk, mv, mo, a, grid, s);
-    return launch_ks1<KSTEPS, false, STA>(mq, mk, mv, mo, a, grid, s);
+    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true, GEO>(mq, mk, mv, mo, a, grid, s);
+    return launch_ks1<KSTEPS, false, GEO>(mq, mk, mv, mo, a, grid, s);
 }
-template <bool STA>
+template <int GEO>
 cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
                      const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
     switch ((a.d + 15) / 16) {
-        case 1: return launch_ks<1, STA>(mq, mk, mv, mo, a, grid, s);
-        case 2: return launch_ks<2, STA>(mq, mk, mv, mo, a, grid, s);
-        case 3: return launch_ks<3, STA>(mq, mk, mv, mo, a, grid, s);
-        case 4: return launch_ks<4, STA>(mq, mk, mv, mo, a, grid, s);
-        case 5: return launch_ks<5, STA>(mq, mk, mv, mo, a, grid, s);
-        case 6: return launch_ks<6, STA>(mq, mk, mv, mo, a, grid, s);
-        case 7: return launch_ks<7, STA>(mq, mk, mv, mo, a, grid, s);
-        case 8: return launch_ks<8, STA>(mq, mk, mv, mo, a, grid, s);
+        case 1: return launch_ks<1, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 2: return launch_ks<2, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 3: return launch_ks<3, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 4: return launch_ks<4, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 5: return launch_ks<5, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 6: return launch_ks<6, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 7: return launch_ks<7, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 8: return launch_ks<8, GEO>(mq, mk, mv, mo, a, grid, s);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -644,8 +670,10 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
     a.d = d;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
     a.tiles_h = a.tiles_w = a.reach_h = a.reach_w = 0;
+    a.kv_list = nullptr;
+    a.kv_count = 0;
     dim3 grid((unsigned)qblocks, (unsigned)heads, (unsigned)batches);
-    return launch_d<false>(mq, mk, mv, mo, a, grid, s);
+    return launch_d<kGeoFull>(mq, mk, mv, mo, a, grid, s);
 }
 
 cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
@@ -670,8 +698,35 @@ cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* 
     a.tiles_w = W / kStaTile;
     a.reach_h = (win_h / kStaTile - 1) / 2;
     a.reach_w = (win_w / kStaTile - 1) / 2;
+    a.kv_list = nullptr;
+    a.kv_count = 0;
     dim3 grid((unsigned)tiles, (unsigned)heads, (unsigned)frames);
-    return launch_d<true>(mq, mk, mv, mo, a, grid, s);
+    return launch_d<kGeoWindow>(mq, mk, mv, mo, a, grid, s);
+}
+
+cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
+                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s) {
+    if (frames == 0 || H == 0 || W == 0) return cudaSuccess;
+    if (H % kStaTile || W % kStaTile || kv_count < 1 || !kv_list) return cudaErrorInvalidValue;
+    const long long tiles = (long long)(H / kStaTile) * (W / kStaTile);
+    if (kv_count > tiles || tiles > 0x7fffffffLL || frames > 65535 || heads > 65535) return cudaErrorInvalidValue;
+    CUtensorMap mq, mk, mv, mo;
+    if (!make_map_grid(&mq, q, d, heads, H, W, frames, 8) || !make_map_grid(&mk, k, d, heads, H, W, frames, 4) ||
+        !make_map_grid(&mv, v, d, heads, H, W, frames, 4) || !make_map_grid(&mo, out, d, heads, H, W, frames, 8))
+        return cudaErrorInvalidValue;
+    FlashTcArgs a;
+    a.Lq = H * W;
+    a.Lk = H * W;
+    a.kv_batched = 1;
+    a.d = d;
+    a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+    a.tiles_h = H / kStaTile;
+    a.tiles_w = W / kStaTile;
+    a.reach_h = a.reach_w = 0;
+    a.kv_list = kv_list;
+    a.kv_count = kv_count;
+    dim3 grid((unsigned)tiles, (unsigned)heads, (unsigned)frames);
+    return launch_d<kGeoList>(mq, mk, mv, mo, a, grid, s);
 }
 
 unsigned int flash_device_errors(bool clear) {

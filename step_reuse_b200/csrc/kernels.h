@@ -46,7 +46,22 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
 cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
                              int heads, int d, int win_h, int win_w, cudaStream_t s);
 
+// Attention of every 16 x 16 query tile of each frame over the 16 x 16 key
+// tiles kv_list names for it: [frames][heads][tiles][kv_count] tile indices
+// (ty * (W/16) + tx) of the same frame.  An index outside the frame raises
+// kDevErrBadIndex in the flash status word and is clamped.
+cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
+                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s);
+
 unsigned int flash_device_errors(bool clear);
+
+// --- draft attention's low-resolution half: pooled sketch + region selection
+// sketch: draft_sketch_bytes(...) of device scratch (fp32 means of q and k
+// over 16 x 16-token regions); sel: [T][heads][R][keep] int32, per query
+// region the keep key regions with the highest draft scores, ascending.
+size_t draft_sketch_bytes(int T, int H, int W, int heads, int d);
+cudaError_t launch_draft_select(const void* q, const void* k, int T, int H, int W, int heads, int d, int keep,
+                                int* sel, void* sketch, cudaStream_t s);
 
 // --- cross attention (text_len <= 128: persistent cross_tc; longer: flash) --
 cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,

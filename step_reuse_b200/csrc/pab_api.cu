@@ -124,6 +124,23 @@ int run_sta(const void* q, const void* k, const void* v, void* out, int T, int H
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "sliding tile attention launch");
 }
 
+int check_draft(int H, int W, int region, int keep) {
+    if (region != 16) return fail(PAB_ERR_UNSUPPORTED, "draft attention region %d unsupported (need 16)", region);
+    if (H % region || W % region) return fail(PAB_ERR_ARG, "frame %d x %d is not whole %d-token regions", H, W, region);
+    const long long R = (long long)(H / region) * (W / region);
+    if (R > 4096) return fail(PAB_ERR_UNSUPPORTED, "%lld regions per frame exceed 4096", R);
+    if (keep < 1 || keep > R) return fail(PAB_ERR_ARG, "keep=%d outside [1, %lld]", keep, R);
+    return PAB_OK;
+}
+
+int run_draft(const void* q, const void* k, const void* v, void* out, int T, int H, int W, int heads, int d,
+              int keep, int* sel, void* sketch, cudaStream_t s) {
+    cudaError_t e = pab::launch_draft_select(q, k, T, H, W, heads, d, keep, sel, sketch, s);
+    if (e != cudaSuccess) return cuda_fail(e, "draft selection launch");
+    e = pab::launch_flash_tile_list(q, k, v, out, T, H, W, heads, d, sel, keep, s);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "region-sparse attention launch");
+}
+
 int run_temporal(const void* q, const void* k, const void* v, void* out, int N, int T, int heads,
                  int d, int spatial_view, cudaStream_t s) {
     cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s);
@@ -171,6 +188,10 @@ struct pab_plan {
     int edge_pct, lo, hi;
     int temporal_sv;  // temporal attention takes / returns the spatial view
     int sta_win_h, sta_win_w;  // > 0: spatial computes are sliding tile attention (16-token tiles)
+    int draft_keep;            // > 0: spatial computes are draft attention (16 x 16 regions)
+    int* draft_sel;            // [T][heads][R][draft_keep]
+    void* draft_sketch;
+    size_t draft_sel_bytes, draft_sketch_bytes;
     // cache
     int device;
     void* slot[3][2];
@@ -207,6 +228,10 @@ void plan_free_device(pab_plan* p) {
     }
     if (p->stage_out) cudaFree(p->stage_out);
     p->stage_out = nullptr;
+    if (p->draft_sel) cudaFree(p->draft_sel);
+    if (p->draft_sketch) cudaFree(p->draft_sketch);
+    p->draft_sel = nullptr;
+    p->draft_sketch = nullptr;
     p->device = -1;
 }
 
@@ -222,6 +247,16 @@ int plan_alloc_kind(pab_plan* p, int kind) {
             cudaError_t e = cudaMalloc(&p->slot[kind][j], p->slot_bytes[kind]);
             if (e != cudaSuccess) return cuda_fail(e, "broadcast cache allocation");
         }
+    if (kind == PAB_SPATIAL && p->draft_keep > 0) {
+        if (!p->draft_sel) {
+            cudaError_t e = cudaMalloc(reinterpret_cast<void**>(&p->draft_sel), p->draft_sel_bytes);
+            if (e != cudaSuccess) return cuda_fail(e, "draft selection allocation");
+        }
+        if (!p->draft_sketch) {
+            cudaError_t e = cudaMalloc(&p->draft_sketch, p->draft_sketch_bytes);
+            if (e != cudaSuccess) return cuda_fail(e, "draft sketch allocation");
+        }
+    }
     if (p->dtype == PAB_FP32) {
         for (int j = 0; j < 3; ++j)
             if (!p->stage_in[j] && p->stage_in_bytes > 0) {
@@ -256,7 +291,10 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
         oo = p->stage_out;
     }
     int rc;
-    if (kind == PAB_SPATIAL && p->sta_win_h > 0)
+    if (kind == PAB_SPATIAL && p->draft_keep > 0)
+        rc = run_draft(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->draft_keep, p->draft_sel,
+                       p->draft_sketch, s);
+    else if (kind == PAB_SPATIAL && p->sta_win_h > 0)
         rc = run_sta(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->sta_win_h, p->sta_win_w, s);
     else if (kind == PAB_SPATIAL)
         rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s);
@@ -318,6 +356,57 @@ int pab_sta_attention(const void* q, const void* k, const void* v, void* out, in
     rc = check_ptrs("q, k, v, out", q, k, v, out);
     if (rc) return rc;
     return run_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, static_cast<cudaStream_t>(cuda_stream));
+    PAB_GUARD_END
+}
+
+int pab_draft_workspace_bytes(int T, int H, int W, int heads, int d, int region, long long* bytes) {
+    if (!bytes) return fail(PAB_ERR_ARG, "null bytes");
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || H < 0 || W < 0) return fail(PAB_ERR_ARG, "T, H, W must be >= 0 (got %d, %d, %d)", T, H, W);
+    rc = check_draft(H, W, region, 1);
+    if (rc && H * W > 0) return rc;
+    *bytes = (long long)pab::draft_sketch_bytes(T, H, W, heads, d);
+    return PAB_OK;
+}
+
+int pab_draft_select(const void* q, const void* k, int T, int H, int W, int heads, int d, int region, int keep,
+                     int* sel, void* workspace, long long workspace_bytes, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || H < 0 || W < 0) return fail(PAB_ERR_ARG, "T, H, W must be >= 0 (got %d, %d, %d)", T, H, W);
+    if ((long long)T * H * W == 0) return PAB_OK;
+    rc = check_draft(H, W, region, keep);
+    if (rc) return rc;
+    if (T > 65535) return fail(PAB_ERR_UNSUPPORTED, "T=%d frames exceeds 65535", T);
+    rc = check_ptrs("q, k, sel, workspace", q, k, sel, workspace);
+    if (rc) return rc;
+    if (workspace_bytes < (long long)pab::draft_sketch_bytes(T, H, W, heads, d))
+        return fail(PAB_ERR_ARG, "workspace of %lld bytes is smaller than %lld", workspace_bytes,
+                    (long long)pab::draft_sketch_bytes(T, H, W, heads, d));
+    cudaError_t e = pab::launch_draft_select(q, k, T, H, W, heads, d, keep, sel, workspace,
+                                             static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "draft selection launch");
+    PAB_GUARD_END
+}
+
+int pab_region_sparse_attention(const void* q, const void* k, const void* v, void* out, int T, int H, int W,
+                                int heads, int d, int region, int keep, const int* sel, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    int rc = check_dims(heads, d);
+    if (rc) return rc;
+    if (T < 0 || H < 0 || W < 0) return fail(PAB_ERR_ARG, "T, H, W must be >= 0 (got %d, %d, %d)", T, H, W);
+    if ((long long)T * H * W == 0) return PAB_OK;
+    rc = check_draft(H, W, region, keep);
+    if (rc) return rc;
+    if (T > 65535) return fail(PAB_ERR_UNSUPPORTED, "T=%d frames exceeds 65535", T);
+    rc = check_ptrs("q, k, v, out", q, k, v, out);
+    if (rc) return rc;
+    if (!sel) return fail(PAB_ERR_ARG, "null selection");
+    cudaError_t e = pab::launch_flash_tile_list(q, k, v, out, T, H, W, heads, d, sel, keep,
+                                                static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "region-sparse attention launch");
     PAB_GUARD_END
 }
 
@@ -534,7 +623,31 @@ int pab_plan_set_spatial_window(pab_plan* plan, int tile, int win_h, int win_w) 
     if (rc) return rc;
     plan->sta_win_h = win_h;
     plan->sta_win_w = win_w;
+    plan->draft_keep = 0;
     return PAB_OK;
+}
+
+int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep) {
+    PAB_GUARD_BEGIN
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    if (keep == 0) {
+        plan->draft_keep = 0;
+        return PAB_OK;
+    }
+    int rc = check_draft(plan->H, plan->W, region, keep);
+    if (rc) return rc;
+    const long long R = (long long)(plan->H / region) * (plan->W / region);
+    const size_t sel_bytes = (size_t)plan->T * plan->heads * R * keep * sizeof(int);
+    if (plan->draft_sel && sel_bytes > plan->draft_sel_bytes) {  // a larger keep: reallocate on next use
+        cudaFree(plan->draft_sel);
+        plan->draft_sel = nullptr;
+    }
+    if (!plan->draft_sel) plan->draft_sel_bytes = sel_bytes;
+    plan->draft_sketch_bytes = pab::draft_sketch_bytes(plan->T, plan->H, plan->W, plan->heads, plan->d);
+    plan->draft_keep = keep;
+    plan->sta_win_h = plan->sta_win_w = 0;
+    return PAB_OK;
+    PAB_GUARD_END
 }
 
 int pab_plan_prepare(pab_plan* plan) {

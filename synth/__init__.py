@@ -36,6 +36,8 @@ class Workload:
     # (tile, win_h, win_w) in tokens when the spatial kind is sliding tile
     # attention; () for full attention within the frame
     spatial_window: tuple = field(default_factory=tuple)
+    # (region, keep) when the spatial kind is draft attention; () otherwise
+    spatial_draft: tuple = field(default_factory=tuple)
 
     @property
     def N(self) -> int:
@@ -77,6 +79,10 @@ WORKLOADS = {
     # 3 x 3-tile windows: the sliding-tile spatial kind under the PAB schedule
     "sta_48x80": Workload("sta_48x80", T=24, H=48, W=80, heads=24, d=128, text_len=256, steps=30,
                           ranges=(2, 4, 6), dtype="bf16", sigma=0.02, spatial_window=(16, 48, 48)),
+    # the same frames under draft attention: 16 x 16 regions (15 per frame),
+    # 4 kept per query region (75% sparsity, the low end of the pages' range)
+    "draft_48x80": Workload("draft_48x80", T=24, H=48, W=80, heads=24, d=128, text_len=256, steps=30,
+                            ranges=(2, 4, 6), dtype="bf16", sigma=0.02, spatial_draft=(16, 4)),
     "sweep": Workload("sweep", T=16, H=30, W=53, heads=16, d=72, text_len=120, steps=50,
                       ranges=(1, 1, 1), dtype="bf16", sigma=0.02, sigma_edge=0.2,
                       extra_ranges=((1, 1, 1), (2, 3, 4), (2, 4, 6), (3, 6, 9))),
