@@ -5,16 +5,19 @@
 // region, and the best `keep` of them form the sparse mask that the
 // region-sparse flash kernel (flash_tc.cu, list geometry) runs under.
 //
-//   draft_pool_kernel    one CTA per (region, frame, tensor): thread c owns
-//                        channels [8c, 8c + 8) and sums the region's 256
-//                        tokens in a fixed order (deterministic), 16-byte
-//                        loads, a 16-token row in flight; writes the fp32
-//                        mean.
-//                        HBM-bound: q and k are read once.
-//   draft_select_kernel  one warp per (query region, head, frame): lane l
-//                        scores key regions l, l + 32, ... (fp32 dot products
-//                        of the pooled rows over d, scaled by 1/sqrt(d)),
-//                        then `keep` rounds of a warp arg-max (higher score
+//   draft_pool_kernel    one CTA per (region, frame, tensor, 1024-channel
+//                        slice): thread c owns 8 channels and sums the
+//                        region's 256 tokens in a fixed order
+//                        (deterministic), 16-byte loads, a 16-token row in
+//                        flight; writes the fp32 mean.  Small CTAs, many of
+//                        them: the grid is several waves, so no SM is left
+//                        with a long tail.  HBM-bound: q and k are read once.
+//   draft_select_kernel  one warp per (query region, head, frame): for each
+//                        key region the lanes split the d channels (the
+//                        query's sketch row in registers, the key's read as
+//                        one coalesced row) and a fixed butterfly sums the
+//                        fp32 products; the score is scaled by 1/sqrt(d).
+//                        Then `keep` rounds of a warp arg-max (higher score
 //                        wins, equal scores go to the lower index) mark the
 //                        kept regions, which are written in ascending order.
 #include "common.cuh"
@@ -25,16 +28,20 @@ namespace {
 
 constexpr int kRegion = 16;
 constexpr int kSelectWarps = 4;
+constexpr int kPoolThreads = 128;  // 8 channels each: a CTA pools a 1024-channel slice
+constexpr int kMaxD = 128;         // head dims the library accepts
 
 // q, k: [T][H][W][C] bf16; sketch: [2][T][R][C] fp32 (q's, then k's)
-__global__ void draft_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                                  float* __restrict__ sketch, int T, int H, int W, int C) {
-    const int r = blockIdx.x, t = blockIdx.y, which = blockIdx.z;
+__global__ void __launch_bounds__(kPoolThreads)
+    draft_pool_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
+                      float* __restrict__ sketch, int T, int H, int W, int C, int slices) {
+    const int r = blockIdx.x, t = blockIdx.y, which = blockIdx.z / slices;
     const int rw = W / kRegion, R = (H / kRegion) * rw;
     const int y0 = (r / rw) * kRegion, x0 = (r % rw) * kRegion;
     const __nv_bfloat16* src = (which == 0 ? q : k) + (long long)t * H * W * C;
     float* dst = sketch + ((long long)which * T + t) * R * C + (long long)r * C;
-    for (int c8 = threadIdx.x; c8 < C / 8; c8 += blockDim.x) {
+    const int c8 = (blockIdx.z % slices) * kPoolThreads + threadIdx.x;
+    if (c8 < C / 8) {
         float acc[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[i] = 0.f;
@@ -73,13 +80,22 @@ __global__ void draft_select_kernel(const float* __restrict__ sketch, int* __res
     const float* kb = sketch + ((long long)(T + t) * R) * C + (long long)h * d;
     float* sc = sm + warp * R;
     unsigned char* taken = reinterpret_cast<unsigned char*>(sm + kSelectWarps * R) + warp * R;
-    for (int j = lane; j < R; j += 32) {
+    float qv[kMaxD / 32];
+#pragma unroll
+    for (int m = 0; m < kMaxD / 32; ++m) qv[m] = lane + 32 * m < d ? qb[lane + 32 * m] : 0.f;
+    for (int j = 0; j < R; ++j) {
         const float* kj = kb + (long long)j * C;
-        float s = 0.f;
-        for (int c = 0; c < d; ++c) s = fmaf(qb[c], kj[c], s);
-        s *= scale;
-        sc[j] = s == s ? s : -INFINITY;  // a NaN score ranks last, so every round still picks a region
-        taken[j] = 0;
+        float part = 0.f;
+#pragma unroll
+        for (int m = 0; m < kMaxD / 32; ++m)
+            if (lane + 32 * m < d) part = fmaf(qv[m], kj[lane + 32 * m], part);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+        if (lane == 0) {
+            const float s = part * scale;
+            sc[j] = s == s ? s : -INFINITY;  // a NaN score ranks last, so every round still picks a region
+            taken[j] = 0;
+        }
     }
     __syncwarp();
     for (int n = 0; n < keep; ++n) {
@@ -128,10 +144,12 @@ cudaError_t launch_draft_select(const void* q, const void* k, int T, int H, int 
     const int R = (H / kRegion) * (W / kRegion);
     if (H % kRegion || W % kRegion || C % 8 || keep < 1 || keep > R || R > 4096 || T > 65535 || heads > 65535)
         return cudaErrorInvalidValue;
-    const int threads = C / 8 < 1024 ? ((C / 8 + 31) / 32) * 32 : 1024;
-    draft_pool_kernel<<<dim3(R, T, 2), threads, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
-                                                        static_cast<const __nv_bfloat16*>(k),
-                                                        static_cast<float*>(sketch), T, H, W, C);
+    const int slices = (C / 8 + kPoolThreads - 1) / kPoolThreads;
+    if (2LL * slices > 65535) return cudaErrorInvalidValue;
+    draft_pool_kernel<<<dim3(R, T, 2 * slices), kPoolThreads, 0, s>>>(static_cast<const __nv_bfloat16*>(q),
+                                                                      static_cast<const __nv_bfloat16*>(k),
+                                                                      static_cast<float*>(sketch), T, H, W, C,
+                                                                      slices);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     const size_t smem = (size_t)kSelectWarps * R * (sizeof(float) + 1);
