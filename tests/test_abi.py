@@ -164,3 +164,52 @@ def test_stateless_argument_checks(pab):
     assert lib.pab_attn_diff_mse(None, None, 10, 0, ctypes.byref(res), None) == pab.PAB_ERR_ARG
     assert lib.pab_attn_diff_mse(None, None, 10, 7, ctypes.byref(res), None) == pab.PAB_ERR_ARG
     assert lib.pab_attn_diff_mse(None, None, 10, 0, None, None) == pab.PAB_ERR_ARG
+
+
+def test_spatial_alternatives_argument_checks(pab):
+    """Sliding tile and draft attention reject bad geometry before any device
+    work (no GPU needed); the plan options validate against the plan's frame."""
+    lib = pab.lib
+    ARG, UNS = pab.PAB_ERR_ARG, pab.PAB_ERR_UNSUPPORTED
+    # pab_sta_attention(q, k, v, out, T, H, W, heads, d, tile, win_h, win_w, stream)
+    assert lib.pab_sta_attention(None, None, None, None, 1, 30, 32, 2, 64, 16, 48, 48, None) == ARG  # H not tiles
+    assert lib.pab_sta_attention(None, None, None, None, 1, 32, 32, 2, 64, 16, 32, 48, None) == ARG  # even window
+    assert lib.pab_sta_attention(None, None, None, None, 1, 32, 32, 2, 64, 16, 40, 48, None) == ARG  # window not tiles
+    assert lib.pab_sta_attention(None, None, None, None, 1, 32, 32, 2, 64, 8, 24, 24, None) == UNS   # tile size
+    assert lib.pab_sta_attention(None, None, None, None, 1, 32, 32, 2, 64, 16, 48, 48, None) == ARG  # null pointers
+    assert lib.pab_sta_attention(None, None, None, None, 0, 32, 32, 2, 64, 16, 48, 48, None) == pab.PAB_OK
+    # draft attention
+    n = ctypes.c_longlong(0)
+    assert lib.pab_draft_workspace_bytes(2, 48, 80, 24, 128, 16, ctypes.byref(n)) == pab.PAB_OK
+    assert n.value == 2 * 2 * 15 * 24 * 128 * 4
+    assert lib.pab_draft_workspace_bytes(2, 48, 80, 24, 128, 8, ctypes.byref(n)) == UNS
+    sel = ctypes.c_void_p(1 << 20)
+    assert lib.pab_draft_select(None, None, 1, 30, 32, 1, 64, 16, 1, sel, sel, 1 << 20, None) == ARG
+    assert lib.pab_draft_select(None, None, 1, 32, 32, 1, 64, 16, 0, sel, sel, 1 << 20, None) == ARG
+    assert lib.pab_draft_select(None, None, 1, 32, 32, 1, 64, 16, 5, sel, sel, 1 << 20, None) == ARG
+    assert lib.pab_draft_select(None, None, 1, 32, 32, 1, 64, 8, 1, sel, sel, 1 << 20, None) == UNS
+    big = ctypes.c_void_p(1 << 24)
+    assert lib.pab_draft_select(big, big, 1, 32, 32, 1, 64, 16, 2, sel, sel, 16, None) == ARG  # workspace too small
+    assert lib.pab_region_sparse_attention(big, big, big, big, 1, 32, 32, 1, 64, 16, 2, None, None) == ARG
+    # plan options: validated against the plan's 48 x 80 frame
+    plan = pab.Plan(2, 48, 80, 2, 64, 16, 10, (2, 3, 4), dtype=torch.bfloat16)
+    try:
+        plan.set_spatial_window(16, 48, 48)
+        plan.set_spatial_draft(16, 4)
+        plan.set_spatial_draft(16, 0)
+        for bad in ((16, 32, 48), (8, 24, 24)):
+            with pytest.raises(pab.PabError):
+                plan.set_spatial_window(*bad)
+        for bad in ((16, 16), (8, 2)):
+            with pytest.raises(pab.PabError):
+                plan.set_spatial_draft(*bad)
+    finally:
+        plan.close()
+    odd = pab.Plan(2, 30, 53, 2, 64, 16, 10, (2, 3, 4), dtype=torch.bfloat16)
+    try:
+        with pytest.raises(pab.PabError):
+            odd.set_spatial_window(16, 48, 48)
+        with pytest.raises(pab.PabError):
+            odd.set_spatial_draft(16, 2)
+    finally:
+        odd.close()
