@@ -45,10 +45,12 @@ UNIT = "TFLOP/s (dense-equivalent attention)"
 # keyed by (sha256 of the kernel's source, workload); a different source hash
 # or a workload without a capture means traffic is null.
 MEASURED_TRAFFIC = {
-    # flash_tc spatial, 480p-like, 1 launch: dram read 175.92 MB + write 42.11 MB
-    ("07d5ce460e633017", "480p"): 218031104,
-    # flash_tc sliding tile attention, sta_48x80, 1 launch: read 1698.89 MB + write 547.61 MB
-    ("07d5ce460e633017", "sta_48x80"): 2246495296,
+    # flash_tc spatial, 480p-like, 1 launch: dram read 175.92 MB + write 44.08 MB
+    ("b78a0851064cded0", "480p"): 220001536,
+    # flash_tc sliding tile attention, sta_48x80, 1 launch: read 1700.31 MB + write 546.97 MB
+    ("b78a0851064cded0", "sta_48x80"): 2247280640,
+    # flash_tc region-sparse (draft) attention, draft_48x80, 1 launch: read 1688.63 MB + write 546.71 MB
+    ("b78a0851064cded0", "draft_48x80"): 2235336960,
 }
 
 
