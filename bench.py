@@ -76,6 +76,10 @@ def parse_args(argv=None):
                     help="draft attention as the spatial kind (workload draft_48x80): pooled sketch and "
                          "selection, region-sparse attention against full spatial attention, and the PAB "
                          "stack with each")
+    ap.add_argument("--dsp", action="store_true",
+                    help="broadcast sequence parallel: one video's frames sharded over the ranks, two "
+                         "all-to-all exchanges per temporal compute (none on broadcast steps); the PAB "
+                         "ranges against ranges (1, 1, 1)")
     ap.add_argument("--dit", action="store_true",
                     help="time the synthetic DiT block (projections, norms, MLP around the library's "
                          "attention) with the workload's PAB ranges and with ranges (1, 1, 1)")
@@ -939,6 +943,84 @@ def run_draft(args):
     return 0
 
 
+def run_dsp(args):
+    """One video sharded over the ranks (strong scaling): a sampling run of
+    the three attention kinds through DSPStack with the workload's ranges and
+    with ranges (1, 1, 1); device-timed, max over ranks; one JSON line with
+    the exchanges and bytes each rank sent."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    import step_reuse_b200 as pab
+    from step_reuse_b200 import dsp
+
+    w = synth.WORKLOADS[args.workload]
+    if w.T % world or w.N % world:
+        raise SystemExit(f"{w.name}: T={w.T} and N={w.N} must divide by {world} ranks")
+    Tl = w.T // world
+    n_sets = max(1, min(w.steps, args.input_sets))
+    full = make_inputs(w, device, n_sets, seed=0)  # the same video on every rank; each takes its frames
+    fr = slice(rank * Tl, (rank + 1) * Tl)
+    inputs = [{k: {n: (x[k][n] if k == "cross" and n != "q" else
+                       x[k][n].view(w.T, w.N, w.C)[fr].contiguous() if k != "cross" else
+                       x[k][n].view(w.T, w.N, w.C)[fr].reshape(Tl * w.N, w.C).contiguous())
+                   for n in ("q", "k", "v")} for k in synth.KINDS} for x in full]
+    del full
+    stream = torch.cuda.current_stream(device)
+    runs = max(2, args.steps // 10)
+    res = {}
+    for label, ranges in (("pab", w.ranges), ("no_broadcast", (1, 1, 1))):
+        st = dsp.DSPStack(pab, w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, ranges, device=device)
+
+        def one():
+            st.reset()
+            for i in range(w.steps):
+                x = inputs[i % n_sets]
+                for k in synth.KINDS:
+                    if st.is_compute(k, i) or k == "temporal":
+                        st.attention(k, i, x[k]["q"], x[k]["k"], x[k]["v"], stream)
+
+        for _ in range(args.warmup):
+            one()
+        torch.cuda.synchronize(device)
+        barrier(device)
+        ex0, by0 = st.exchanges, st.bytes_sent
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(runs):
+            one()
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(a.elapsed_time(b) / runs, device)
+        res[label] = {"ms_per_run": ms, "denoising_steps_per_s": w.steps / (ms * 1e-3),
+                      "exchanges_per_run": (st.exchanges - ex0) // runs,
+                      "bytes_sent_per_run_per_rank": (st.bytes_sent - by0) // runs,
+                      "temporal_computes": sum(st.is_compute("temporal", i) for i in range(w.steps))}
+        st.close()
+    assert pab.device_errors() == 0
+    if rank == 0:
+        ex_p, ex_n = res["pab"]["exchanges_per_run"], res["no_broadcast"]["exchanges_per_run"]
+        line = {
+            "metric": "broadcast sequence parallel: denoising steps/s of one video over the ranks",
+            "value": res["pab"]["denoising_steps_per_s"], "unit": "steps/s", "n_gpus": world, "runs": runs,
+            "warmup": args.warmup, "higher_is_better": True, "scaling": "strong", "dtype": "bf16",
+            "data": "synthetic",
+            "config": dict(workload_config(w), parallelism=f"sequence parallel x{world} (frames; positions "
+                                                            f"for temporal attention)"),
+            "pab": res["pab"], "no_broadcast": res["no_broadcast"],
+            "exchange_reduction": 1.0 - ex_p / ex_n if ex_n else None,
+            "speedup_vs_no_broadcast": res["no_broadcast"]["ms_per_run"] / res["pab"]["ms_per_run"],
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
@@ -947,6 +1029,8 @@ def main(argv=None):
         return run_sta(args)
     if args.draft:
         return run_draft(args)
+    if args.dsp:
+        return run_dsp(args)
     if args.dit:
         return run_dit(args)
     return run_ours(args)

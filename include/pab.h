@@ -161,6 +161,17 @@ int pab_cross_attention(const void* q, const void* kt, const void* vt, void* out
 int pab_layout(int to_temporal, const void* src, void* dst, int T, int N, int C,
                int dtype, void* cuda_stream);
 
+/* Swap the two outer dimensions of a block array: src [P, Q, block_rows, C]
+ * -> dst [Q, P, block_rows, C], i.e. dst[q][p] = src[p][q] for blocks of
+ * block_rows consecutive C-element rows.  pab_layout is the case
+ * block_rows = 1; with P = frames per rank, Q = ranks and block_rows =
+ * positions per rank it packs a frame-sharded [T/G, N, C] tensor into the
+ * per-destination chunks of a sequence-parallel all-to-all (and back).
+ * Same element types, alignment, row-size and no-overlap rules as
+ * pab_layout; bytes are moved unchanged. */
+int pab_permute_blocks(const void* src, void* dst, int P, int Q, long long block_rows, int C, int dtype,
+                       void* cuda_stream);
+
 /* ---------------------------------------------------------------------- */
 /* Attention-difference diagnostic (PAB report, Fig. 1: the difference      */
 /* between consecutive diffusion steps' attention outputs, as MSE).        */

@@ -19,6 +19,8 @@ What each function computes (sources are the PAB pages):
   * mse -- the attention-difference diagnostic of Fig. 1 (MSE between the
     outputs of consecutive diffusion steps);
   * layout -- the spatial view [T, N, C] <-> temporal view [N, T, C];
+  * permute_blocks -- [P, Q, block, C] -> [Q, P, block, C], the packing of a
+    sequence-parallel all-to-all (PAB report, "Parallel");
   * sta_attention -- sliding tile attention as the spatial kind (sgqg.cn
     summary of "Fast Video Generation with Sliding Tile Attention", section
     "Sliding Tile Attention (STA)"): 2-D tiles per frame, a window of whole
@@ -73,11 +75,13 @@ def _load():
         lib.oracle_mse.argtypes = [_dp, _dp, ctypes.c_long]
         lib.oracle_mse.restype = ctypes.c_double
         lib.oracle_layout.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p] + [ctypes.c_int] * 4
+        lib.oracle_permute_blocks.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_long, ctypes.c_int, ctypes.c_int]
         lib.oracle_num_threads.restype = ctypes.c_int
         for name in ("oracle_spatial_attention", "oracle_temporal_attention",
                      "oracle_cross_attention", "oracle_sta_attention", "oracle_draft_select",
                      "oracle_region_sparse_attention", "oracle_pab_edge_steps",
-                     "oracle_pab_schedule", "oracle_layout", "oracle_num_threads"):
+                     "oracle_pab_schedule", "oracle_layout", "oracle_permute_blocks", "oracle_num_threads"):
             if getattr(lib, name).restype is not ctypes.c_double:
                 getattr(lib, name).restype = ctypes.c_int
         _lib = lib
@@ -232,4 +236,18 @@ def layout(x: np.ndarray, to_temporal: bool) -> np.ndarray:
                                T, N, C, x.dtype.itemsize)
     if rc != 0:
         raise RuntimeError("oracle_layout failed")
+    return out
+
+
+def permute_blocks(x: np.ndarray, P: int, Q: int) -> np.ndarray:
+    """x viewed as [P, Q, block, C] -> [Q, P, block, C]; bytes moved unchanged
+    (sequence-parallel packing, PAB report, "Parallel")."""
+    x = np.ascontiguousarray(x)
+    C = x.shape[-1]
+    block = x.size // (P * Q * C) if P * Q * C else 0
+    assert P * Q * block * C == x.size
+    out = np.empty((Q, P, block, C), dtype=x.dtype)
+    rc = _load().oracle_permute_blocks(x.ctypes.data, out.ctypes.data, P, Q, block, C, x.dtype.itemsize)
+    if rc != 0:
+        raise RuntimeError("oracle_permute_blocks failed")
     return out

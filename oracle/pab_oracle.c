@@ -467,6 +467,24 @@ int oracle_layout(int to_temporal, const void *src, void *dst, int T, int N, int
     return 0;
 }
 
+/* Sequence-parallel packing (PAB report, "Parallel", Fig. 3: dynamic sequence
+ * parallel moves each rank's frames of every position chunk to the rank
+ * that owns the chunk, and back): swap the two outer dimensions of
+ * [P][Q][block][C] -> [Q][P][block][C]; blocks of `block` rows of C
+ * elements move unchanged. */
+int oracle_permute_blocks(const void *src, void *dst, int P, int Q, long block, int C, int elem_size)
+{
+    if (P < 0 || Q < 0 || block < 0 || C < 0 || elem_size <= 0)
+        return -1;
+    const char *s = (const char *)src;
+    char *o = (char *)dst;
+    const size_t blk = (size_t)block * C * elem_size;
+    for (int p = 0; p < P; ++p)
+        for (int q = 0; q < Q; ++q)
+            memcpy(o + ((size_t)q * P + p) * blk, s + ((size_t)p * Q + q) * blk, blk);
+    return 0;
+}
+
 int oracle_num_threads(void)
 {
 #ifdef _OPENMP

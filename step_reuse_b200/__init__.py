@@ -35,7 +35,7 @@ EXPORTS = (
     "pab_version", "pab_last_error_string", "pab_spatial_attention", "pab_temporal_attention",
     "pab_temporal_attention_sv", "pab_plan_set_temporal_view", "pab_sta_attention",
     "pab_plan_set_spatial_window", "pab_draft_workspace_bytes", "pab_draft_select",
-    "pab_region_sparse_attention", "pab_plan_set_spatial_draft",
+    "pab_region_sparse_attention", "pab_plan_set_spatial_draft", "pab_permute_blocks",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
     "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
@@ -74,6 +74,7 @@ def _load() -> ctypes.CDLL:
         "pab_plan_set_spatial_draft": ([vp, i, i], i),
         "pab_cross_attention": ([vp, vp, vp, vp, ll, i, i, i, vp], i),
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
+        "pab_permute_blocks": ([vp, vp, i, i, ll, i, i, vp], i),
         "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
         "pab_attn_diff_mse_async": ([vp, vp, ll, i, vp, vp], i),
         "pab_attn_diff_mse_noalloc": ([vp, vp, ll, i, vp, vp], i),
@@ -233,6 +234,18 @@ def layout(x, to_temporal: bool, out=None, stream=None):
     T, N = (A, B) if to_temporal else (B, A)
     _check(lib.pab_layout(1 if to_temporal else 0, _ptr(x), _ptr(out), T, N, C, _dtype_code(x),
                           _stream(stream)))
+    return out
+
+
+def permute_blocks(x, P: int, Q: int, out=None, stream=None):
+    """x viewed as [P, Q, block_rows, C] -> out [Q, P, block_rows, C] (same
+    total shape as x unless `out` gives one)."""
+    C = x.shape[-1]
+    block_rows = x.numel() // (P * Q * C) if P * Q * C else 0
+    if P * Q * block_rows * C != x.numel():
+        raise ValueError(f"{tuple(x.shape)} is not [{P}, {Q}, rows, {C}]")
+    out = torch.empty((Q, P, block_rows, C), dtype=x.dtype, device=x.device) if out is None else out
+    _check(lib.pab_permute_blocks(_ptr(x), _ptr(out), P, Q, block_rows, C, _dtype_code(x), _stream(stream)))
     return out
 
 

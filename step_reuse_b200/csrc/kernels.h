@@ -25,6 +25,10 @@ cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, dou
 // --- layout change [T,N,C] <-> [N,T,C] (bulk-copy engine) ----------------
 cudaError_t launch_layout(int to_temporal, const void* src, void* dst, int T, int N,
                           int row_bytes, cudaStream_t s);
+// Swap the two outer dimensions of [P][Q][block] rows of row_bytes each:
+// dst[q][p][w] = src[p][q][w] (blocks of `block` rows move together).
+cudaError_t launch_swap_outer(const void* src, void* dst, int P, int Q, long long block, int row_bytes,
+                              cudaStream_t s);
 unsigned int layout_device_errors(bool clear);
 
 // --- temporal short-sequence attention ([N,T,C], L = T) -------------------

@@ -5,7 +5,11 @@
 // "Implementation").
 //
 // Every token row of C channels is contiguous in both views, so the change
-// is a permutation of rows of C*elem bytes.  A persistent grid works as a
+// is a permutation of rows of C*elem bytes.  The same engine swaps the two
+// outer dimensions of [P][Q][block][C] (blocks of `block` consecutive rows
+// move together): with block = 1 that is the view change, with block = N/G
+// it packs and unpacks the per-rank chunks of a sequence-parallel
+// all-to-all.  A persistent grid works as a
 // row-gather DMA engine on the bulk-copy (TMA) unit: each unit of work is R
 // consecutive DESTINATION rows; one elected thread issues R untiled
 // cp.async.bulk loads (one per source row) into a shared-memory stage,
@@ -28,16 +32,19 @@ struct LayoutArgs {
     char* dst;
     long long rows;      // T*N
     long long units;     // ceil(rows / R)
-    int A;               // destination outer extent (dst row = a*B + b)
-    int B;               // destination inner extent; source row = b*A + a
+    int A;               // destination outer extent (dst block = a*B + b)
+    int B;               // destination inner extent; source block = b*A + a
+    long long inner;     // rows per block
     int row_bytes;
     int R;               // rows per unit
 };
 
-PAB_DEV long long src_row_of(long long dst_row, int A, int B) {
-    const long long a = dst_row / B;
-    const long long b = dst_row - a * B;
-    return b * A + a;
+PAB_DEV long long src_row_of(long long dst_row, int A, int B, long long inner) {
+    const long long blk = dst_row / inner;
+    const long long w = dst_row - blk * inner;
+    const long long a = blk / B;
+    const long long b = blk - a * B;
+    return (b * A + a) * inner + w;
 }
 
 __global__ void __launch_bounds__(32) layout_bulk_kernel(LayoutArgs p) {
@@ -58,7 +65,7 @@ __global__ void __launch_bounds__(32) layout_bulk_kernel(LayoutArgs p) {
         mbar_arrive_expect_tx(bar, (uint32_t)(cnt * p.row_bytes));
         const uint32_t dst = smem_base + s * stage_bytes;
         for (long long j = 0; j < cnt; ++j) {
-            const long long sr = src_row_of(r0 + j, p.A, p.B);
+            const long long sr = src_row_of(r0 + j, p.A, p.B, p.inner);
             bulk_g2s(dst + (uint32_t)(j * p.row_bytes), p.src + sr * p.row_bytes,
                      (uint32_t)p.row_bytes, bar);
         }
@@ -121,18 +128,22 @@ __global__ void __launch_bounds__(32) layout_bulk_kernel(LayoutArgs p) {
 
 cudaError_t launch_layout(int to_temporal, const void* src, void* dst, int T, int N,
                           int row_bytes, cudaStream_t s) {
+    // to_temporal: src [T][N] -> dst [N][T]; else src [N][T] -> dst [T][N]
+    return to_temporal ? launch_swap_outer(src, dst, T, N, 1, row_bytes, s)
+                       : launch_swap_outer(src, dst, N, T, 1, row_bytes, s);
+}
+
+cudaError_t launch_swap_outer(const void* src, void* dst, int P, int Q, long long block, int row_bytes,
+                              cudaStream_t s) {
+    // src [P][Q][block] rows -> dst [Q][P][block]: dst block q*P + p <- src block p*Q + q
     LayoutArgs p;
     p.src = static_cast<const char*>(src);
     p.dst = static_cast<char*>(dst);
-    p.rows = (long long)T * N;
+    p.rows = (long long)P * Q * block;
     p.row_bytes = row_bytes;
-    if (to_temporal) {  // dst [N][T]: dst row n*T + t  <- src row t*N + n
-        p.A = N;
-        p.B = T;
-    } else {            // dst [T][N]: dst row t*N + n  <- src row n*T + t
-        p.A = T;
-        p.B = N;
-    }
+    p.A = Q;
+    p.B = P;
+    p.inner = block;
     int R = kStageBytes / row_bytes;
     if (R < 1) R = 1;
     p.R = R;

@@ -475,6 +475,28 @@ int pab_layout(int to_temporal, const void* src, void* dst, int T, int N, int C,
     PAB_GUARD_END
 }
 
+int pab_permute_blocks(const void* src, void* dst, int P, int Q, long long block_rows, int C, int dtype,
+                       void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (dtype != PAB_BF16 && dtype != PAB_FP32) return fail(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (P < 0 || Q < 0 || block_rows < 0 || C < 0) return fail(PAB_ERR_ARG, "negative size");
+    const int elem = dtype == PAB_FP32 ? 4 : 2;
+    const long long row = (long long)C * elem;
+    if ((long long)P * Q * block_rows * C == 0) return PAB_OK;
+    if (row % 16 != 0) return fail(PAB_ERR_UNSUPPORTED, "row of %lld bytes is not a multiple of 16", row);
+    if (row > 48 * 1024) return fail(PAB_ERR_UNSUPPORTED, "row of %lld bytes exceeds 48 KiB", row);
+    if (!src || !dst) return fail(PAB_ERR_ARG, "null src/dst");
+    if (!aligned16(src) || !aligned16(dst)) return fail(PAB_ERR_ARG, "src/dst not 16-byte aligned");
+    const char* s0 = static_cast<const char*>(src);
+    const char* d0 = static_cast<const char*>(dst);
+    const long long bytes = (long long)P * Q * block_rows * row;
+    if (s0 < d0 + bytes && d0 < s0 + bytes) return fail(PAB_ERR_ARG, "src and dst overlap");
+    cudaError_t e = pab::launch_swap_outer(src, dst, P, Q, block_rows, (int)row,
+                                           static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "block permute launch");
+    PAB_GUARD_END
+}
+
 int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype, double* result_dev,
                             void* cuda_stream) {
     PAB_GUARD_BEGIN
