@@ -111,8 +111,9 @@ int pab_sta_attention(const void* q, const void* k, const void* v, void* out, in
  * with the highest scores (equal scores: the lower index), written to sel
  * ([T, heads, R, keep] int32, device memory, ascending index per row).
  * Means and scores are fp32.  workspace: device scratch of at least
- * pab_draft_workspace_bytes(...) bytes, 16-byte aligned, owned by the
- * caller.  region must be 16; H, W multiples of 16; 1 <= keep <= R <= 4096.
+ * pab_draft_workspace_bytes(...) bytes, owned by the caller; q, k, sel and
+ * workspace must be 16-byte aligned.  region must be 16; H, W multiples of
+ * 16; 1 <= keep <= R <= 4096.
  *
  * pab_region_sparse_attention: every query of region i attends to the tokens
  * of the key regions sel[t][h][i][0..keep) (softmax over those only).  sel
