@@ -20,6 +20,7 @@ host<->device copies inside the timed region.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -80,6 +81,9 @@ def parse_args(argv=None):
                     help="broadcast sequence parallel: one video's frames sharded over the ranks, two "
                          "all-to-all exchanges per temporal compute (none on broadcast steps); the PAB "
                          "ranges against ranges (1, 1, 1)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="the 50-step sweep (480p shapes): every range set of the sweep workload timed, "
+                         "with the per-step attention difference (MSE) of the all-compute run")
     ap.add_argument("--dit", action="store_true",
                     help="time the synthetic DiT block (projections, norms, MLP around the library's "
                          "attention) with the workload's PAB ranges and with ranges (1, 1, 1)")
@@ -517,6 +521,27 @@ def run_ours(args):
         "clocks": clk,
     }
 
+    # the same stack with every step computing (ranges 1, 1, 1): the speedup
+    # the broadcast buys on this workload
+    nstack = AttentionStack(pab, dataclasses.replace(w, ranges=(1, 1, 1)), device)
+    nstack.run(inputs, stream)
+    nsteps = max(3, args.steps // 10)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    n0 = torch.cuda.Event(enable_timing=True)
+    n1 = torch.cuda.Event(enable_timing=True)
+    n0.record(stream)
+    for _ in range(nsteps):
+        nstack.run(inputs, stream)
+    n1.record(stream)
+    torch.cuda.synchronize(device)
+    nms = max_over_ranks(n0.elapsed_time(n1) / nsteps, device)
+    line["no_broadcast"] = {"ms_per_step": nms, "steps": nsteps,
+                            "denoising_steps_per_s": world * w.steps / (nms * 1e-3),
+                            "gpu_launches": nstack.launches_per_run * nsteps, "ranges": [1, 1, 1]}
+    line["speedup_vs_no_broadcast"] = nms / ms
+    nstack.close()
+
     # the same stack with the temporal kernel reading / writing the spatial
     # view itself (no layout launches): reported beside the main figure
     fstack = AttentionStack(pab, w, device, fused=True)
@@ -943,6 +968,77 @@ def run_draft(args):
     return 0
 
 
+def run_sweep(args):
+    """The sweep workload (480p shapes, 50 steps, inputs drifting 0.2 per
+    step on the edge steps and 0.02 in the middle): one sampling run of the
+    fused attention stack per range set, device-timed, and the attention
+    difference of consecutive steps (MSE) of the all-compute run per kind,
+    edges against the middle (the U shape of the PAB report's Fig. 1)."""
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    import step_reuse_b200 as pab
+
+    w = synth.WORKLOADS["sweep"]
+    e = -(-15 * w.steps // 100)
+    traj = make_inputs(w, device, 1, seed=rank)  # step 0, then one drift per step
+    g = synth.generator(rank + 7, device)
+    for i in range(1, w.steps):
+        nxt = {k: {n: t.clone() for n, t in v.items()} for k, v in traj[-1].items()}
+        synth.drift_(nxt, synth.sigma_at(w, i, e), g)
+        traj.append(nxt)
+    stream = torch.cuda.current_stream(device)
+    runs = max(2, args.steps // 20)
+    res, mse = {}, None
+    for ranges in w.extra_ranges:
+        st = AttentionStack(pab, dataclasses.replace(w, ranges=ranges), device, fused=True)
+        for _ in range(max(1, args.warmup)):
+            st.run(traj, stream)
+        torch.cuda.synchronize(device)
+        barrier(device)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(runs):
+            st.run(traj, stream)
+        b.record(stream)
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(a.elapsed_time(b) / runs, device)
+        res[str(tuple(ranges))] = {"ms_per_run": ms, "denoising_steps_per_s": world * w.steps / (ms * 1e-3),
+                                   "computes": {k: sum(st.sched[k]) for k in synth.KINDS}}
+        if tuple(ranges) == (1, 1, 1):
+            mse = st.mse.cpu().numpy()
+        st.close()
+    assert pab.device_errors() == 0
+    if rank == 0:
+        base = res[str((1, 1, 1))]["ms_per_run"]
+        for v in res.values():
+            v["speedup_vs_no_broadcast"] = base / v["ms_per_run"]
+        u = {}
+        for ki, k in enumerate(synth.KINDS):
+            edge = [float(mse[ki, i]) for i in list(range(1, e)) + list(range(w.steps - e + 1, w.steps))]
+            mid = [float(mse[ki, i]) for i in range(e + 1, w.steps - e)]
+            u[k] = {"edge_mean": sum(edge) / len(edge), "middle_mean": sum(mid) / len(mid),
+                    "edge_over_middle": (sum(edge) / len(edge)) / (sum(mid) / len(mid))}
+        line = {
+            "metric": "PAB sweep: denoising steps/s of the attention stack per broadcast range set "
+                      "(value: ranges 2/4/6)",
+            "value": res[str((2, 4, 6))]["denoising_steps_per_s"],
+            "unit": "steps/s", "n_gpus": world, "runs": runs, "higher_is_better": True, "scaling": "weak",
+            "dtype": "bf16", "data": "synthetic (drift 0.2 per edge step, 0.02 per middle step)",
+            "config": dict(workload_config(w), ranges=[list(r) for r in w.extra_ranges],
+                           step="one 50-step sampling run of the fused attention stack"),
+            "per_range_set": res, "attention_difference_all_compute": u,
+        }
+        print(json.dumps(line), flush=True)
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
 def run_dsp(args):
     """One video sharded over the ranks (strong scaling): a sampling run of
     the three attention kinds through DSPStack with the workload's ranges and
@@ -1031,6 +1127,8 @@ def main(argv=None):
         return run_draft(args)
     if args.dsp:
         return run_dsp(args)
+    if args.sweep:
+        return run_sweep(args)
     if args.dit:
         return run_dit(args)
     return run_ours(args)
