@@ -39,14 +39,23 @@ struct LayoutArgs {
     int R;               // rows per unit
 };
 
+// BLOCKED = false is the view change (one-row blocks): one division per row
+// on the issuing thread's path instead of two more for the block split
+template <bool BLOCKED>
 PAB_DEV long long src_row_of(long long dst_row, int A, int B, long long inner) {
-    const long long blk = dst_row / inner;
-    const long long w = dst_row - blk * inner;
-    const long long a = blk / B;
-    const long long b = blk - a * B;
-    return (b * A + a) * inner + w;
+    if constexpr (!BLOCKED) {
+        const long long a = dst_row / B;
+        return (dst_row - a * B) * A + a;
+    } else {
+        const long long blk = dst_row / inner;
+        const long long w = dst_row - blk * inner;
+        const long long a = blk / B;
+        const long long b = blk - a * B;
+        return (b * A + a) * inner + w;
+    }
 }
 
+template <bool BLOCKED>
 __global__ void __launch_bounds__(32) layout_bulk_kernel(LayoutArgs p) {
     extern __shared__ __align__(128) unsigned char smem[];
     __shared__ __align__(8) unsigned long long full_bar[kStages];
@@ -65,7 +74,7 @@ __global__ void __launch_bounds__(32) layout_bulk_kernel(LayoutArgs p) {
         mbar_arrive_expect_tx(bar, (uint32_t)(cnt * p.row_bytes));
         const uint32_t dst = smem_base + s * stage_bytes;
         for (long long j = 0; j < cnt; ++j) {
-            const long long sr = src_row_of(r0 + j, p.A, p.B, p.inner);
+            const long long sr = src_row_of<BLOCKED>(r0 + j, p.A, p.B, p.inner);
             bulk_g2s(dst + (uint32_t)(j * p.row_bytes), p.src + sr * p.row_bytes,
                      (uint32_t)p.row_bytes, bar);
         }
@@ -151,13 +160,13 @@ cudaError_t launch_swap_outer(const void* src, void* dst, int P, int Q, long lon
     if (p.rows == 0) return cudaSuccess;
     const size_t smem = (size_t)kStages * R * row_bytes;
     // the kernel's static shared memory (barriers) comes on top of `smem`
-    cudaError_t e = cudaFuncSetAttribute(layout_bulk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    auto kern = block == 1 ? layout_bulk_kernel<false> : layout_bulk_kernel<true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int per_sm = (int)((200 * 1024) / (smem + 1024));
     long long grid = (long long)device_sm_count() * (per_sm < 1 ? 1 : per_sm);
     if (grid > p.units) grid = p.units;
-    layout_bulk_kernel<<<(unsigned)grid, 32, smem, s>>>(p);
+    kern<<<(unsigned)grid, 32, smem, s>>>(p);
     return cudaGetLastError();
 }
 
