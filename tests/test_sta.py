@@ -243,3 +243,15 @@ def test_sta_full_size_sampled(pab, oracle_mod):
                                         H, W, heads, TILE, 48, 48)
         assert_attn_close(out[fr:fr + 1], want, f"sta full size, frame {fr}")
     _no_device_errors(pab)
+
+
+@pytest.mark.parametrize("H,W,win_h,win_w", [(48, 80, 48, 48), (32, 48, 16, 80), (64, 96, 80, 48), (16, 16, 48, 48)])
+def test_bench_window_pair_count_is_the_mask_count(H, W, win_h, win_w):
+    """The benchmark's algorithmic flops count query-key pairs in closed form;
+    they equal the pairs the window mask admits."""
+    import dataclasses
+
+    import bench
+    import synth
+    w = dataclasses.replace(synth.WORKLOADS["sta_48x80"], H=H, W=W, spatial_window=(TILE, win_h, win_w))
+    assert bench.sta_pairs(w) == int(window_mask(H, W, TILE, win_h, win_w).sum())
