@@ -324,7 +324,7 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
 
 extern "C" {
 
-int pab_version(void) { return (0 << 16) | 1; }
+int pab_version(void) { return (0 << 16) | 2; }  // 0.2: sliding tile, draft attention, block permute
 
 const char* pab_last_error_string(void) { return g_last_error.c_str(); }
 
