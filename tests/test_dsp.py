@@ -2,7 +2,7 @@
 frame-sharded attention stack with its two all-to-all exchanges per temporal
 compute, none on a temporal broadcast step.
 
-CPU (gloo, two ranks): DSPStack from the product, driven through a stand-in
+CPU (gloo, two and four ranks): DSPStack from the product, driven through a stand-in
 binding whose plan and block permute are the oracle's functions, must give
 every rank exactly the oracle's attention of the whole video restricted to
 its frames, at every step of a PAB run; the exchange, collective and byte
@@ -136,8 +136,8 @@ def _dsp_worker(rank, world, port, ranges, q):
             dist.destroy_process_group()
 
 
-def _run_two_ranks(ranges):
-    world, port = 2, _free_port()
+def _run_ranks(ranges, world=2):
+    port = _free_port()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     procs = [ctx.Process(target=_dsp_worker, args=(r, world, port, ranges, q)) for r in range(world)]
@@ -150,10 +150,10 @@ def _run_two_ranks(ranges):
 
 
 @pytest.mark.timeout(300)
-@pytest.mark.parametrize("ranges", [(2, 3, 4), (1, 1, 1)])
-def test_two_rank_sequence_parallel_matches_the_whole_video(oracle_mod, ranges):
-    res = _run_two_ranks(ranges)
-    steps, T, N, C, elem, G = 10, 4, 24, 16, 8, 2
+@pytest.mark.parametrize("ranges,world", [((2, 3, 4), 2), ((1, 1, 1), 2), ((2, 3, 4), 4)])
+def test_sequence_parallel_matches_the_whole_video(oracle_mod, ranges, world):
+    res = _run_ranks(ranges, world)
+    steps, T, N, C, elem, G = 10, 4, 24, 16, 8, world
     computes = int(oracle_mod.schedule(steps, ranges[1])[0].sum())
     for rank, worst, exchanges, collectives, sent in res:
         for kind, err in worst.items():
