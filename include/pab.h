@@ -53,7 +53,9 @@ enum { PAB_SPATIAL = 0, PAB_TEMPORAL = 1, PAB_CROSS = 2 };
 enum { PAB_BF16 = 0, PAB_FP32 = 1 };
 
 /* Broadcast ranges per kind (each >= 1; 1 = never broadcast) and the edge
- * share in percent (0 -> the pages' 15).  The pages order the ranges
+ * share in percent: a negative value selects the pages' 15, 0 gives no edge
+ * steps (every step follows the range rule), 1..50 as given; other values
+ * are rejected with PAB_ERR_ARG.  The pages order the ranges
  * r_cross >= r_temporal >= r_spatial (Fig. 2); that order is not enforced. */
 typedef struct {
     int spatial;
@@ -155,7 +157,10 @@ int pab_cross_attention(const void* q, const void* kt, const void* vt, void* out
 /* Layout change between the two views of a video token tensor.            */
 /* ---------------------------------------------------------------------- */
 
-/* to_temporal = 1: src [T, N, C] (spatial view) -> dst [N, T, C];
+/* The PAB report ("Implementation") attends spatially within each frame and
+ * temporally across the frames at each position: the two views of one video
+ * token tensor, [T, N, C] (frames outer) and [N, T, C] (positions outer).
+ * to_temporal = 1: src [T, N, C] (spatial view) -> dst [N, T, C];
  * to_temporal = 0: src [N, T, C] -> dst [T, N, C].
  * dtype PAB_BF16 or PAB_FP32; bytes are moved unchanged.  src and dst must
  * not overlap.  C * element size must be a multiple of 16 bytes. */
@@ -178,8 +183,12 @@ int pab_permute_blocks(const void* src, void* dst, int P, int Q, long long block
 /* between consecutive diffusion steps' attention outputs, as MSE).        */
 /* ---------------------------------------------------------------------- */
 
-/* *result (HOST pointer) = mean over n elements of (a - b)^2, accumulated in
- * fp64 in a fixed order (bitwise reproducible for a given n).  a and b hold n
+/* *result (HOST pointer) = mean over n elements of (a - b)^2.  For PAB_FP32
+ * every squared difference is formed and accumulated in fp64; for PAB_BF16
+ * the squared differences of each 16-byte vector (8 elements) are summed in
+ * fp32 (exact differences, relative error < 1e-6 per vector) and that sum
+ * is accumulated in fp64.  The order is fixed (bitwise reproducible for a
+ * given n and device).  a and b hold n
  * elements of dtype (PAB_BF16 or PAB_FP32).  n == 0 gives 0.  Uses a
  * per-device scratch buffer (fp64 partial sums and a completion ticket) that
  * the library allocates on first use.  SYNCHRONISES cuda_stream before
@@ -203,11 +212,14 @@ int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype
  * static device array of 4096 doubles (32 KiB) that every GPU loading the
  * library holds until exit; the call allocates nothing.  A call that would
  * need more than 4095 partial sums (only on devices with more than 1023 SMs)
- * returns PAB_ERR_UNSUPPORTED.  The first call on each device looks up the
- * array's device address (cudaGetSymbolAddress), caches it and clears the
- * array's completion ticket on cuda_stream; make that first call before any
- * stream capture.  All calls share the array: calls whose kernels overlap on
- * the GPU race and must be serialised by the caller. */
+ * returns PAB_ERR_UNSUPPORTED.  Every call looks up the array's device
+ * address in the current device's context (cudaGetSymbolAddress; nothing is
+ * cached, so a call after cudaDeviceReset finds the reloaded array).  The
+ * array's completion ticket starts at zero when the library's module is
+ * loaded on a device and every call returns it to zero; no call clears it.
+ * All calls share the array and it keeps the last call's contents: calls
+ * whose kernels overlap on the GPU race and must be serialised by the
+ * caller. */
 int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long n, int dtype,
                               double* result_dev, void* cuda_stream);
 
@@ -234,11 +246,14 @@ int pab_plan_create(int T, int H, int W, int heads, int d, int text_len, int ste
                     pab_ranges ranges, int dtype, pab_plan** out_plan);
 
 /* Free the plan and its cache (device memory freed; no pointer returned by
- * pab_attention stays valid).  NULL is accepted. */
+ * pab_attention stays valid).  NULL is accepted.  The cache is the store of
+ * broadcast attention outputs (PAB report, "Implementation" and Fig. 2). */
 int pab_plan_destroy(pab_plan* plan);
 
 /* Start a new sampling run: the cache is invalidated and step order restarts.
- * Device memory is kept. */
+ * Device memory is kept.  A broadcast reuses an output of the same run only
+ * (PAB report, "Implementation" and Fig. 2: one step's attention output is
+ * reused by the next few steps of that sampling run). */
 int pab_plan_reset(pab_plan* plan);
 
 /* Choose the layout of TEMPORAL q, k, v and of its output for this plan:
@@ -265,7 +280,10 @@ int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep);
  * compute.  Idempotent. */
 int pab_plan_prepare(pab_plan* plan);
 
-/* *is_compute = 1 if (kind, step) computes, 0 if it is a broadcast hit.
+/* *is_compute = 1 if (kind, step) computes, 0 if it is a broadcast hit, by
+ * the rule of pab_plan_create (PAB report, "Implementation" and Fig. 2: every
+ * attention computes in the first and last 15% of the steps; in between each
+ * kind is computed once per window of its range and broadcast to the rest).
  * Host only, no GPU needed. */
 int pab_schedule_query(const pab_plan* plan, int kind, int step, int* is_compute);
 

@@ -295,7 +295,7 @@ class Plan:
     the second following compute of the same kind, reset() or close()."""
 
     def __init__(self, T, H, W, heads, d, text_len, steps, ranges, dtype=torch.bfloat16,
-                 edge_pct: int = 0):
+                 edge_pct: int = 15):
         self.T, self.H, self.W, self.heads, self.d = T, H, W, heads, d
         self.N, self.C, self.text_len, self.steps = H * W, heads * d, text_len, steps
         self.dtype = dtype

@@ -51,7 +51,6 @@ constexpr int kBox = 128 * 128;   // bytes of one [128 rows][64 cols] bf16 box
 constexpr int kThreads = 448;     // 2 softmax warpgroups (key halves) + epilogue warpgroup + producer + MMA warp
 constexpr uint32_t kTmemCols = 512;
 constexpr int kPolyPairsOf8 = 3;  // share of exponentials on the FMA pipes
-constexpr float kC0 = 1.0f, kC1 = 0.693282962f, kC2 = 0.242210999f, kC3 = 0.0550089180f;
 
 __device__ unsigned int g_cross_err = 0;
 
@@ -79,33 +78,6 @@ struct Bars {
     uint32_t tmem_base;
     int abort;
 };
-
-PAB_DEV float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// 2^x on the FMA pipes for a pair, x <= 0 here (no running max): range
-// reduction x = rint(x) + f, f in [-0.5, 0.5], a degree-3 polynomial for 2^f
-// fitted here as a minimax of the relative error with p(0) = 1 fixed (so
-// integer x, the row maximum in particular, give exact powers of two; max
-// relative error 1.0e-4) and the exponent added directly; x < -120 is
-// clamped (result ~1e-36).
-PAB_DEV void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-    const tc::f32x2 x = tc::pack2(fmaxf(x0, -120.0f), fmaxf(x1, -120.0f));
-    const tc::f32x2 magic = tc::pack2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-    const tc::f32x2 y = tc::add2(x, magic);
-    const tc::f32x2 f = tc::sub2(x, tc::sub2(y, magic));
-    tc::f32x2 p = tc::fma2(tc::pack2(kC3, kC3), f, tc::pack2(kC2, kC2));
-    p = tc::fma2(p, f, tc::pack2(kC1, kC1));
-    p = tc::fma2(p, f, tc::pack2(kC0, kC0));
-    float q0, q1, y0, y1;
-    tc::unpack2(p, q0, q1);
-    tc::unpack2(y, y0, y1);
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(y0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(y1) << 23));
-}
 
 // bounded wait that gives up at once when the CTA has already aborted (a
 // phase that has completed is taken without reading the abort flag)
@@ -376,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float t0, t1, p0, p1;
                     tc::unpack2(t, t0, t1);
                     if ((e & 7) < kPolyPairsOf8) {
-                        exp2_poly2(t0, t1, p0, p1);
+                        tc::exp2_poly2(t0, t1, p0, p1);
                     } else {
                         p0 = ex2(t0);
                         p1 = ex2(t1);

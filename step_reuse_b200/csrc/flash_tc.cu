@@ -71,8 +71,6 @@ constexpr int kPolyPairsOf8 = PAB_POLY_PAIRS_OF_8;
 #ifndef PAB_FLASH_ONES
 #define PAB_FLASH_ONES 1
 #endif
-// 2^f ~ kP0 + kP1 f + kP2 f^2 + kP3 f^3 on [-0.5, 0.5] (see exp2_poly2)
-constexpr float kP0 = 1.0f, kP1 = 0.693282962f, kP2 = 0.242210999f, kP3 = 0.0550089180f;
 
 __device__ unsigned int g_flash_err = 0;
 
@@ -122,38 +120,6 @@ struct Bars {
     uint32_t tmem_base;
     int abort;
 };
-
-PAB_DEV float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
-// 2^x on the FMA/ALU pipes for two values at once, for x <= 8 (the lazily
-// rescaled softmax never exceeds 2^8).  Cody-Waite style range reduction:
-// x = n + f with n = rint(x) (the 1.5*2^23 rounding trick) and f in
-// [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted here by minimising the
-// maximum relative error on [-0.5, 0.5] with p(0) = 1 fixed, so integer x
-// give exact powers of two (linear-programming minimax fit; max relative
-// error 1.0e-4, far below the bf16 rounding of P); 2^n is added to the
-// exponent field.  x below -120 is clamped (the result, ~1e-36, is
-// negligible next to the row maximum's weight 1).
-PAB_DEV void exp2_poly2(float x0, float x1, float& p0, float& p1) {
-    const tc::f32x2 x = tc::pack2(fmaxf(x0, -120.0f), fmaxf(x1, -120.0f));
-    const tc::f32x2 magic = tc::pack2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
-    const tc::f32x2 y = tc::add2(x, magic);
-    const tc::f32x2 f = tc::sub2(x, tc::sub2(y, magic));  // x - rint(x)
-    tc::f32x2 p = tc::fma2(tc::pack2(kP3, kP3), f, tc::pack2(kP2, kP2));
-    p = tc::fma2(p, f, tc::pack2(kP1, kP1));
-    p = tc::fma2(p, f, tc::pack2(kP0, kP0));
-    float q0, q1, y0, y1;
-    tc::unpack2(p, q0, q1);
-    tc::unpack2(y, y0, y1);
-    // bits(y) << 23 == rint(x) << 23 (mod 2^32): the constant part of y's
-    // bit pattern has no bits below position 22.
-    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(y0) << 23));
-    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(y1) << 23));
-}
 
 // bounded wait that gives up at once when the CTA has already aborted (a
 // phase that has completed is taken without reading the abort flag)
@@ -489,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float t0, t1, p0, p1;
                     tc::unpack2(t, t0, t1);
                     if (((idx >> 1) & 7) < kPolyPairsOf8) {
-                        exp2_poly2(t0, t1, p0, p1);
+                        tc::exp2_poly2(t0, t1, p0, p1);
                     } else {
                         p0 = ex2(t0);
                         p1 = ex2(t1);

@@ -13,8 +13,6 @@
 // depends only on n and the SM count, and the final sum's order does not
 // depend on which block finishes last, so the result is bitwise reproducible
 // on a given device.
-#include <mutex>
-
 #include "../../include/pab.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -188,12 +186,14 @@ cudaError_t launch_mse(const void* a, const void* b, long long n, int dtype, dou
 // completion ticket, the rest are partial sums (at most kNoAllocMaxPartials).
 // Every GPU that loads this library keeps it until the process exits.  Every
 // call shares it and it keeps the last call's contents.  Only the ticket must
-// start at zero: the first call on a device clears it (stream-ordered before
-// its kernel), and every call's last block returns it to zero.  The partial
-// slots need no clearing: each block overwrites its own slot and the final
-// sum reads only the slots this call wrote.  Calls whose kernels overlap on
-// the GPU (different streams, or different host threads on one device) race
-// on the array and must be serialised by the caller.
+// start at zero: a file-scope device array is zero when the module is loaded
+// on a device, and every call's last block returns the ticket to zero, so no
+// call clears it (a clear issued by one call could land under another call's
+// kernel still running on another stream).  The partial slots need no
+// clearing: each block overwrites its own slot and the final sum reads only
+// the slots this call wrote.  Calls whose kernels overlap on the GPU
+// (different streams, or different host threads on one device) race on the
+// array and must be serialised by the caller.
 // ===========================================================================
 namespace {
 
@@ -201,36 +201,19 @@ constexpr int kNoAllocScratch = 4096;
 constexpr int kNoAllocMaxPartials = kNoAllocScratch - 1;
 static __device__ __align__(256) double g_mse_noalloc_scratch[kNoAllocScratch];
 
-constexpr int kNoAllocMaxDevices = 64;
-std::mutex g_noalloc_mu;
-double* g_noalloc_ptr[kNoAllocMaxDevices] = {nullptr};
-
-// Device address of the array on the current device.  Host code cannot use
-// the array's name as a device pointer (it names a host-side stand-in), so
-// the address is looked up once per device with cudaGetSymbolAddress while
-// that device is current, and cached; that first call also clears the
-// completion ticket on `stream`.
-int noalloc_scratch(double** out, cudaStream_t stream) {
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess)
-        return pab::report_error(PAB_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
-    if (dev < 0 || dev >= kNoAllocMaxDevices)
-        return pab::report_error(PAB_ERR_UNSUPPORTED, "device index %d", dev);
-    std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, g_mse_noalloc_scratch);
-        if (e != cudaSuccess || !p)
-            return pab::report_error(PAB_ERR_CUDA, "cudaGetSymbolAddress of the MSE scratch array: %s",
-                                     cudaGetErrorString(e));
-        e = cudaMemsetAsync(p, 0, sizeof(unsigned long long), stream);
-        if (e != cudaSuccess)
-            return pab::report_error(PAB_ERR_CUDA, "clearing the MSE completion ticket: %s",
-                                     cudaGetErrorString(e));
-        g_noalloc_ptr[dev] = static_cast<double*>(p);
-    }
-    *out = g_noalloc_ptr[dev];
+// Device address of the array in the current device's context.  Host code
+// cannot use the array's name as a device pointer (it names a host-side
+// stand-in), so every call looks the address up with cudaGetSymbolAddress
+// while the caller's device is current.  Nothing is cached: after a
+// cudaDeviceReset the module is loaded again (with a zeroed array) at a
+// possibly different address, and the next call sees that address.
+int noalloc_scratch(double** out) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_mse_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+        return pab::report_error(PAB_ERR_CUDA, "cudaGetSymbolAddress of the MSE scratch array: %s",
+                                 cudaGetErrorString(e));
+    *out = static_cast<double*>(p);
     return PAB_OK;
 }
 
@@ -253,7 +236,7 @@ extern "C" int pab_attn_diff_mse_noalloc(const void* a, const void* b, long long
                                  "this call needs %d partial sums; the static scratch array holds %d",
                                  parts, kNoAllocMaxPartials);
     double* scratch = nullptr;
-    const int rc = noalloc_scratch(&scratch, static_cast<cudaStream_t>(cuda_stream));
+    const int rc = noalloc_scratch(&scratch);
     if (rc != PAB_OK) return rc;
     const cudaError_t e = pab::launch_mse(a, b, n, dtype, scratch, parts, result_dev,
                                           static_cast<cudaStream_t>(cuda_stream));

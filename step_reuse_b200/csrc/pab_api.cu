@@ -572,8 +572,9 @@ int pab_plan_create(int T, int H, int W, int heads, int d, int text_len, int ste
     if (ranges.spatial < 1 || ranges.temporal < 1 || ranges.cross < 1)
         return fail(PAB_ERR_ARG, "broadcast ranges must be >= 1 (got %d, %d, %d)", ranges.spatial,
                     ranges.temporal, ranges.cross);
-    const int edge = ranges.edge_pct == 0 ? 15 : ranges.edge_pct;
-    if (edge < 0 || edge > 50) return fail(PAB_ERR_ARG, "edge_pct=%d outside [0, 50]", ranges.edge_pct);
+    // a negative edge share selects the pages' 15%; 0 means no edge steps
+    const int edge = ranges.edge_pct < 0 ? 15 : ranges.edge_pct;
+    if (edge > 50) return fail(PAB_ERR_ARG, "edge_pct=%d outside [0, 50] (negative: 15)", ranges.edge_pct);
     const long long N = (long long)H * W;
     if (N > (1LL << 30)) return fail(PAB_ERR_UNSUPPORTED, "H*W too large");
     pab_plan* p = new pab_plan;

@@ -203,6 +203,34 @@ PAB_DEV float max3f(float a, float b, float c) {
     return r;
 }
 
+// 2^x on the FMA/ALU pipes for two values at once, for x <= 8 (the lazily
+// rescaled softmax never exceeds 2^8).  Cody-Waite style range reduction:
+// x = n + f with n = rint(x) (the 1.5*2^23 rounding trick) and f in
+// [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted by minimising the
+// maximum relative error on [-0.5, 0.5] with p(0) = 1 fixed, so integer x
+// give exact powers of two (linear-programming minimax fit; max relative
+// error 1.0e-4, far below the bf16 rounding of P); 2^n is added to the
+// exponent field.  x below -120 is clamped (the result, ~1e-36, is
+// negligible next to the row maximum's weight 1).  The softmax kernels move
+// part of their exponentials from the MUFU unit to the FMA pipes with it.
+constexpr float kExpP0 = 1.0f, kExpP1 = 0.693282962f, kExpP2 = 0.242210999f, kExpP3 = 0.0550089180f;
+PAB_DEV void exp2_poly2(float x0, float x1, float& p0, float& p1) {
+    const f32x2 x = pack2(fmaxf(x0, -120.0f), fmaxf(x1, -120.0f));
+    const f32x2 magic = pack2(12582912.0f, 12582912.0f);  // 1.5 * 2^23
+    const f32x2 y = add2(x, magic);
+    const f32x2 f = sub2(x, sub2(y, magic));  // x - rint(x)
+    f32x2 p = fma2(pack2(kExpP3, kExpP3), f, pack2(kExpP2, kExpP2));
+    p = fma2(p, f, pack2(kExpP1, kExpP1));
+    p = fma2(p, f, pack2(kExpP0, kExpP0));
+    float q0, q1, y0, y1;
+    unpack2(p, q0, q1);
+    unpack2(y, y0, y1);
+    // bits(y) << 23 == rint(x) << 23 (mod 2^32): the constant part of y's
+    // bit pattern has no bits below position 22.
+    p0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(y0) << 23));
+    p1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(y1) << 23));
+}
+
 PAB_DEV void named_bar_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" :: "r"(id), "r"(threads) : "memory");
 }

@@ -53,12 +53,6 @@ struct TemporalArgs {
     float scale_log2;  // log2(e) / sqrt(d)
 };
 
-PAB_DEV float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
-
 // smem layout of one stage: [3 tensors][G heads][RT rows][P cols] bf16
 template <int DN>
 __global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constant__ CUtensorMap tm_q,

@@ -72,9 +72,10 @@ def test_schedule_exhaustive_small(pab, oracle_mod):
 
 
 def test_edge_pct_parameter(pab, oracle_mod):
-    for edge in (5, 15, 25, 50):
+    for edge in (0, 5, 15, 25, 50, -1):
         plan = pab.Plan(2, 2, 2, 1, 8, 4, 40, (3, 3, 3), edge_pct=edge)
-        comp, _ = oracle_mod.schedule(40, 3, edge_pct=edge)
+        # a negative share selects the default 15%; 0 means no edge steps
+        comp, _ = oracle_mod.schedule(40, 3, edge_pct=15 if edge < 0 else edge)
         assert [plan.is_compute(1, i) for i in range(40)] == [bool(c) for c in comp]
         plan.close()
 

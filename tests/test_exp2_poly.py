@@ -1,4 +1,4 @@
-"""The flash kernel's software exp2 (exp2_poly2 in flash_tc.cu), emulated bit
+"""The softmax kernels' software exp2 (exp2_poly2 in tc.cuh), emulated bit
 for bit in numpy float32 with the coefficients read from the kernel source,
 against numpy's exp2 in float64 over the whole input range the softmax
 produces (x <= 8; x < -120 clamped).  The kernel moves part of the softmax
@@ -10,19 +10,22 @@ import re
 import numpy as np
 
 SRC = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))),
-                   "step_reuse_b200", "csrc", "flash_tc.cu")
+                   "step_reuse_b200", "csrc", "tc.cuh")
 
 
 def kernel_coefficients():
     text = open(SRC).read()
-    vals = dict(re.findall(r"\b(kP[0-3]) = ([-0-9.e]+)f", text))
-    return [np.float32(vals[f"kP{i}"]) for i in range(4)]
+    vals = dict(re.findall(r"\b(kExpP[0-3]) = ([-0-9.e]+)f", text))
+    return [np.float32(vals[f"kExpP{i}"]) for i in range(4)]
 
 
-def test_kernels_share_the_coefficients():
-    other = open(SRC.replace("flash_tc.cu", "cross_tc.cu")).read()
-    vals = dict(re.findall(r"\b(kC[0-3]) = ([-0-9.e]+)f", other))
-    assert [np.float32(vals[f"kC{i}"]) for i in range(4)] == kernel_coefficients()
+def test_kernels_share_one_polynomial():
+    # one definition (tc.cuh); the kernels that use it define no copy of their own
+    csrc = os.path.dirname(SRC)
+    for name in os.listdir(csrc):
+        if name.endswith(".cu"):
+            text = open(os.path.join(csrc, name)).read()
+            assert "void exp2_poly2" not in text and "kExpP0 =" not in text, name
 
 
 def exp2_poly_emulated(x):
