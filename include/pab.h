@@ -178,6 +178,50 @@ int pab_layout(int to_temporal, const void* src, void* dst, int T, int N, int C,
 int pab_permute_blocks(const void* src, void* dst, int P, int Q, long long block_rows, int C, int dtype,
                        void* cuda_stream);
 
+/* Sequence-parallel exchange (PAB report, "Parallel", Fig. 3): dynamic
+ * sequence parallelism gives every rank T/G frames, and a temporal compute
+ * first moves every rank's frames of position chunk g to rank g (all frames
+ * of N/G positions) and afterwards moves the output back; a temporal
+ * broadcast step moves nothing.  This call performs one such move for up to
+ * three tensors in one launch, writing every block straight into its
+ * destination buffer -- on this GPU, or a peer GPU's buffer mapped into this
+ * process with pab_ipc_open -- so no packing copy and no collective carries
+ * the data.
+ *   src[t], t < ntensors (1..3): P * G blocks of block_rows rows of C
+ *     elements; src_order 0: block (p, g) is block p * G + g
+ *     ([P][G][block_rows][C], e.g. the spatial view [T/G, N, C] with
+ *     P = T/G and block_rows = N/G); src_order 1: block g * P + p
+ *     ([G][P][block_rows][C], e.g. the temporal output [T, N/G, C]).
+ *   dst: HOST array of ntensors * G device pointers, tensor-major
+ *     (dst[t * G + g]); block (p, g) of tensor t is written to rows
+ *     dst_offset_rows + p * dst_stride_rows ... + block_rows - 1 of
+ *     dst[t * G + g].
+ * Pack (rank r of G): src_order 0, P = T/G, block_rows = N/G,
+ *   dst_offset_rows = r * (T/G) * (N/G), dst_stride_rows = N/G.
+ * Unpack (rank r): src_order 1, P = T/G, block_rows = N/G,
+ *   dst_offset_rows = r * (N/G), dst_stride_rows = N.
+ * 1 <= G <= 32; dtype PAB_BF16 or PAB_FP32; bytes are moved unchanged.
+ * C * element size and every pointer 16-byte aligned.  Sources and
+ * destinations must not overlap.  The writes are complete when this call's
+ * work on cuda_stream is; a caller whose destinations are other GPUs' memory
+ * orders them before the readers with a stream-ordered barrier (for example
+ * a one-element collective after this call on every rank). */
+int pab_scatter_blocks(const void* const* src, void* const* dst, int ntensors, int G, int P,
+                       long long block_rows, int C, int src_order, long long dst_offset_rows,
+                       long long dst_stride_rows, int dtype, void* cuda_stream);
+
+/* Device memory that the other processes of this node can map (CUDA IPC),
+ * for the destinations of pab_scatter_blocks.  pab_ipc_alloc allocates
+ * `bytes` on the current device (cudaMalloc, so the handle covers exactly
+ * this buffer) and writes its 64-byte IPC handle; pab_ipc_free releases it.
+ * pab_ipc_open maps another process's buffer from its handle into this
+ * process (peer access enabled on demand); pab_ipc_close unmaps it.  A
+ * process cannot open its own handle (CUDA returns an error). */
+int pab_ipc_alloc(long long bytes, void** ptr, unsigned char handle[64]);
+int pab_ipc_free(void* ptr);
+int pab_ipc_open(const unsigned char handle[64], void** ptr);
+int pab_ipc_close(void* ptr);
+
 /* ---------------------------------------------------------------------- */
 /* Attention-difference diagnostic (PAB report, Fig. 1: the difference      */
 /* between consecutive diffusion steps' attention outputs, as MSE).        */

@@ -36,6 +36,7 @@ EXPORTS = (
     "pab_temporal_attention_sv", "pab_plan_set_temporal_view", "pab_sta_attention",
     "pab_plan_set_spatial_window", "pab_draft_workspace_bytes", "pab_draft_select",
     "pab_region_sparse_attention", "pab_plan_set_spatial_draft", "pab_permute_blocks",
+    "pab_scatter_blocks", "pab_ipc_alloc", "pab_ipc_free", "pab_ipc_open", "pab_ipc_close",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
     "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
@@ -75,6 +76,11 @@ def _load() -> ctypes.CDLL:
         "pab_cross_attention": ([vp, vp, vp, vp, ll, i, i, i, vp], i),
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
         "pab_permute_blocks": ([vp, vp, i, i, ll, i, i, vp], i),
+        "pab_scatter_blocks": ([ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, ll, i, i, ll, ll, i, vp], i),
+        "pab_ipc_alloc": ([ll, ctypes.POINTER(vp), ctypes.c_char_p], i),
+        "pab_ipc_free": ([vp], i),
+        "pab_ipc_open": ([ctypes.c_char_p, ctypes.POINTER(vp)], i),
+        "pab_ipc_close": ([vp], i),
         "pab_attn_diff_mse": ([vp, vp, ll, i, ctypes.POINTER(ctypes.c_double), vp], i),
         "pab_attn_diff_mse_async": ([vp, vp, ll, i, vp, vp], i),
         "pab_attn_diff_mse_noalloc": ([vp, vp, ll, i, vp, vp], i),
@@ -247,6 +253,71 @@ def permute_blocks(x, P: int, Q: int, out=None, stream=None):
     out = torch.empty((Q, P, block_rows, C), dtype=x.dtype, device=x.device) if out is None else out
     _check(lib.pab_permute_blocks(_ptr(x), _ptr(out), P, Q, block_rows, C, _dtype_code(x), _stream(stream)))
     return out
+
+
+def scatter_blocks(srcs, dsts, G: int, P: int, block_rows: int, src_order: int, dst_offset_rows: int,
+                   dst_stride_rows: int, stream=None):
+    """One move of broadcast sequence parallelism's exchange: every source
+    tensor in `srcs` (1..3, each P*G blocks of block_rows rows) has block
+    (p, g) written to rows dst_offset_rows + p*dst_stride_rows.. of the
+    g-th destination.  `dsts[t]` lists G destinations of tensor t, each a
+    CUDA tensor or a raw device address (int) -- e.g. a peer GPU's buffer
+    mapped with ipc_open."""
+    nt = len(srcs)
+    if nt < 1 or nt > 3 or len(dsts) != nt or any(len(d) != G for d in dsts):
+        raise ValueError("need 1..3 sources, each with G destinations")
+    C = srcs[0].shape[-1]
+    for x in srcs:
+        if x.dtype != srcs[0].dtype or x.shape[-1] != C or x.numel() != P * G * block_rows * C:
+            raise ValueError(f"source {tuple(x.shape)} is not {P * G} blocks of [{block_rows}, {C}]")
+    src_arr = (ctypes.c_void_p * nt)(*[x.data_ptr() for x in srcs])
+    flat = [d if isinstance(d, int) else d.data_ptr() for row in dsts for d in row]
+    dst_arr = (ctypes.c_void_p * len(flat))(*flat)
+    _check(lib.pab_scatter_blocks(src_arr, dst_arr, nt, G, P, block_rows, C, src_order, dst_offset_rows,
+                                  dst_stride_rows, _dtype_code(srcs[0]), _stream(stream)))
+
+
+def ipc_alloc(nbytes: int):
+    """(device address, 64-byte handle) of a new buffer that other processes
+    of this node can map with ipc_open; release it with ipc_free."""
+    ptr = ctypes.c_void_p()
+    handle = ctypes.create_string_buffer(64)
+    _check(lib.pab_ipc_alloc(nbytes, ctypes.byref(ptr), handle))
+    return ptr.value, handle.raw
+
+
+def ipc_free(ptr: int):
+    _check(lib.pab_ipc_free(ctypes.c_void_p(ptr)))
+
+
+def ipc_open(handle: bytes) -> int:
+    """Map another process's ipc_alloc buffer into this process."""
+    if len(handle) != 64:
+        raise ValueError("IPC handles are 64 bytes")
+    ptr = ctypes.c_void_p()
+    _check(lib.pab_ipc_open(handle, ctypes.byref(ptr)))
+    return ptr.value
+
+
+def ipc_close(ptr: int):
+    _check(lib.pab_ipc_close(ctypes.c_void_p(ptr)))
+
+
+def ipc_tensor(shape, dtype, device):
+    """A new CUDA tensor in a buffer the other processes of this node can map
+    (ipc_open_tensor): (tensor, 64-byte handle, address for ipc_free)."""
+    n = 1
+    for x in shape:
+        n *= int(x)
+    ptr, handle = ipc_alloc(n * torch.tensor([], dtype=dtype).element_size())
+    return _wrap(ptr, shape, dtype, device), handle, ptr
+
+
+def ipc_open_tensor(handle: bytes, shape, dtype, device):
+    """Another process's ipc_tensor mapped into this one: (tensor, address for
+    ipc_close)."""
+    ptr = ipc_open(handle)
+    return _wrap(ptr, shape, dtype, device), ptr
 
 
 def attn_diff_mse(a, b, stream=None) -> float:

@@ -4,45 +4,67 @@
 // tokens against one shared set of text keys/values) -- PAB report,
 // "Implementation".  softmax(Q K^T / sqrt(d)) V per (batch, head).
 //
-// A CTA owns 256 query rows of one (batch, head) as two 128-row tiles A and B
-// that share every K/V tile, and runs four roles:
-//   warp 8 (one thread)   TMA producer: Q_A, Q_B, K_0, K_1 once, then per
-//                          step j one ring slot with V_j and K_{j+2} (tiles of
-//                          64 keys; K is consumed two steps before V);
-//   warps 9, 10 (one thread each)  MMA issuers, one per query tile X:
-//                          S_X(j) = Q_X K_j^T (SS form, fp32 in TMEM) and
-//                          O_X += P_X(j) V_j (TS form: P from TMEM, V from
-//                          shared memory).  S is double-buffered per tile, so
-//                          S_X(j+2) is issued right behind PV_X(j) and is
-//                          ready before the softmax needs it: the softmax
-//                          never waits for a round trip through the tensor
-//                          cores.  Warp 9 also owns TMEM;
-//   warps 0-3 / 4-7       softmax of tile A / B: thread i owns query row i =
-//                          TMEM lane i.  It reads its row of S with tcgen05.ld,
-//                          keeps the running max and sum in registers (tree
-//                          reductions, no shuffles), writes P as bf16 over S's
-//                          columns and rescales O in TMEM only when the running
-//                          max grew by more than 2^8 (the final O / l is exact
-//                          either way).  Exponentials: 5/8 on the MUFU ex2
-//                          unit, 3/8 on the FMA pipes (exp2_poly2).
-//                          At the end it normalises O and writes it through
-//                          shared memory with a TMA tensor store.
-// Rescaling O_X at step j needs PV_X(j-1) retired: the softmax then waits for
-// step j-1's slot to be done.
+// Persistent CTAs, one per SM, walk a static list of work items: CTA c takes
+// items c, c + gridDim.x, ...  An item is 256 query rows of one (batch, head)
+// as two 128-row tiles A and B that share every K/V tile (for the tile
+// geometries, one 16 x 16 query tile of a frame: A its upper 8 rows, B the
+// lower 8).  Consecutive items share (batch, head), so the CTAs running at
+// one time read the same K/V from L2.
+// The 64-key K/V tiles of all of a CTA's items form ONE sequence of global
+// steps g = 0, 1, ...; use s of the ring carries K_s and V_{s-2} in slot
+// s mod NST.  Roles:
+//   producer warp         TMA producer (one thread): per item the two Q
+//                          tiles (Q is double-buffered by item parity), per
+//                          ring use one slot;
+//   two MMA warps         MMA issuers, one per query tile X, warp-uniform
+//                          (one elected lane issues): once P_X(g) is written,
+//                          O_X += P_X(g) V_g (TS form: P from TMEM, V from
+//                          shared memory) and S_X(g+2) = Q_X K_{g+2}^T (SS
+//                          form, fp32 in TMEM) into the S buffer that P_X(g)
+//                          is read from (the tensor core executes in order),
+//                          then one commit for the slot.  S_X(g+2) may belong
+//                          to the next item, so the next item's first two
+//                          score tiles are ready when the softmax finishes the
+//                          current item's epilogue;
+//   V-ones warp           (d % 16 != 0): sets V's padding column
+//                          d to 1 as each V tile lands, so O's column d
+//                          accumulates the row sums of P with the same bf16 P
+//                          as the numerator (the softmax keeps no running sum);
+//   softmax warps         per tile X one warp per TMEM lane quarter (for
+//                          head dims up to 96 two, each taking 32 of every 64
+//                          keys): the thread of query row i (TMEM lane i)
+//                          reads its scores of S with
+//                          tcgen05.ld, keeps the running max in registers,
+//                          writes P as bf16 over S's columns and rescales O in
+//                          TMEM only when the running max grew by more than
+//                          2^8 (the final O / l is exact either way);
+//                          exponentials 5/8 on the MUFU ex2 unit, 3/8 on the
+//                          FMA pipes (tc::exp2_poly2).  Then the item's
+//                          epilogue: O / l -> bf16 -> the item's Q buffer (no
+//                          score product reads it any more) -> TMA store.  The
+//                          store's read of shared memory is waited for during
+//                          the next item's first step, which then frees the
+//                          buffer for the Q of the item after next.
+// Rescaling O_X at step g needs PV_X(g-1) retired: the softmax then waits for
+// the commit of ring use g+1 (PV_X(g-1), S_X(g+1)).
 //
 // TMEM columns: S_A0 [0,64), S_A1 [64,128), S_B0 [128,192), S_B1 [192,256),
 //               O_A [256,256+NO), O_B [384,384+NO).
-// Operand layouts (128-byte swizzle, TMA-written):
-//   Q, K: [rows][64 cols] boxes (128 rows for Q, 64 for K), K-major (d
-//         contiguous); a 16-wide K step advances the descriptor start by 32
-//         bytes inside the box.
+// Operand layouts (TMA-written):
+//   Q, K: [rows][64 cols] boxes (128 rows for Q, 64 for K; 128-byte swizzle),
+//         K-major (d contiguous), plus for head dims whose 16-column K steps
+//         leave one or two over a [rows][16 or 32 cols] tail box (32- or
+//         64-byte swizzle); a 16-wide K step advances the descriptor start by
+//         32 bytes inside a box.  The output is staged in Q's layout.
 //   V:    [64 rows][64 cols] boxes read MN-major (B of the PV product has
 //         N = d contiguous); a 16-key K step advances by 16 rows = 2048 bytes,
 //         the next 64 columns of d are one box (8 KB) further (LBO).
-// Head dims that are not a multiple of 64 read zero-filled columns past d
-// (the tensor map's innermost extent is d); keys past Lk are masked to -inf;
+// Columns past d read as zero (the tensor map's innermost extent is d) and
+// are not stored; keys past Lk are masked to -inf;
 // query rows past Lq are zero-filled on load and clipped by the TMA store; a
-// B tile that lies wholly past Lq is skipped.
+// B tile that lies wholly past Lq issues no MMAs, computes no softmax and
+// stores nothing (its barriers still complete, so every role counts the
+// same steps).
 // Every wait on an mbarrier is bounded; on time-out the CTA raises the error
 // word, lets its own asynchronous copies and MMAs drain, frees TMEM and exits.
 #include <cuda.h>
@@ -53,17 +75,16 @@
 namespace pab {
 namespace {
 
-constexpr int kBM = 128;          // query rows per tile (two tiles per CTA)
-constexpr int kStaTile = 16;      // sliding tile attention: 16 x 16-token tiles (the CTA's 256 queries)
+constexpr int kBM = 128;          // query rows per tile (two tiles per item)
+constexpr int kStaTile = 16;      // sliding tile attention: 16 x 16-token tiles (the item's 256 queries)
 constexpr int kBN = 64;           // keys per K/V tile
 constexpr int kQBox = 128 * 128;  // bytes of one [128 rows][64 cols] bf16 box (Q, O)
 constexpr int kKVBox = 64 * 128;  // bytes of one [64 rows][64 cols] bf16 box (K, V)
-constexpr int kThreads = 384;     // 2 softmax warpgroups + producer warp + 2 MMA warps + V-ones warp
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleLog2 = 8.0f;
 // Exponentials: of every 8 consecutive pairs of a row's scores, this many go
-// to exp2_poly2 on the FMA pipes and the rest to the MUFU ex2 unit, which
-// alone would bound the softmax (16 results per clock per SM).
+// to tc::exp2_poly2 on the FMA pipes and the rest to the MUFU ex2 unit,
+// which alone would bound the softmax (16 results per clock per SM).
 #ifndef PAB_POLY_PAIRS_OF_8
 #define PAB_POLY_PAIRS_OF_8 3
 #endif
@@ -76,10 +97,13 @@ __device__ unsigned int g_flash_err = 0;
 
 struct FlashTcArgs {
     int Lq;            // query rows per batch
-    int Lk;            // keys per batch
+    int Lk;            // keys per batch (>= 1)
     int kv_batched;    // 1: K/V have a batch coordinate (spatial); 0: shared (cross)
     int d;             // head dim
     float scale_log2;  // log2(e) / sqrt(d)
+    int heads;
+    int per_bh;        // items per (batch, head): 256-row query blocks, or query tiles
+    int items;         // batches * heads * per_bh
     // tile geometries only: the frame in 16 x 16 tiles; the window's reach
     // in tiles on each side of the query tile (window geometry); the key
     // tiles of every query tile, [batches][heads][tiles][kv_count] (list
@@ -96,26 +120,92 @@ enum { kGeoFull = 0, kGeoWindow = 1, kGeoList = 2 };
 
 constexpr int kMaxStages = 8;
 
-// The pipeline is built around ONE commit per tile and K/V step: slot s of
-// the ring holds V_j and K_{j+2} (j = s mod NST); after issuing PV_X(j) and
-// S_X(j+2) tile X's issuer commits slot_done[s][X] once.  Its completion
-// tells tile X's softmax that S_X(j+2) is in TMEM and proves PV_X(j) retired
-// (in-order completion); the producer refills the slot once both tiles'
-// barriers of the slot completed.  The tiles never wait on each other's
-// MMAs, and tile B's softmax starts only once tile A's first row maximum is
-// done: the two tiles' score reads and maxima then fall into each other's
-// exponential phases instead of coinciding (measured 5-10% faster at
-// d = 64-72; the offset fades over a long key loop).
+// One work item, decoded from its index.
+struct Item {
+    int b, h, qblk;        // batch, head, query block (full) or query tile index (tiled)
+    int ty, tx;            // tile geometries: the query tile's position
+    int wy0, wx0, wcols;   // window geometry: first window tile and window width in tiles
+    int nkv;               // 64-key steps (>= 1)
+    bool has_b;            // tile B holds query rows
+    const int* klist;      // list geometry: this query tile's key tiles
+};
+
+template <int GEO>
+PAB_DEV Item decode_item(const FlashTcArgs& a, int it) {
+    Item m;
+    const int bh = it / a.per_bh;
+    m.qblk = it - bh * a.per_bh;
+    m.h = bh % a.heads;
+    m.b = bh / a.heads;
+    m.ty = m.tx = m.wy0 = m.wx0 = 0;
+    m.wcols = 1;
+    m.klist = nullptr;
+    if constexpr (GEO != kGeoFull) {
+        m.ty = m.qblk / a.tiles_w;
+        m.tx = m.qblk - m.ty * a.tiles_w;
+        m.has_b = true;
+    } else {
+        m.has_b = m.qblk * 2 * kBM + kBM < a.Lq;
+    }
+    if constexpr (GEO == kGeoWindow) {
+        m.wy0 = max(m.ty - a.reach_h, 0);
+        m.wx0 = max(m.tx - a.reach_w, 0);
+        const int wy1 = min(m.ty + a.reach_h + 1, a.tiles_h), wx1 = min(m.tx + a.reach_w + 1, a.tiles_w);
+        m.wcols = wx1 - m.wx0;
+        m.nkv = (wy1 - m.wy0) * m.wcols * 4;
+    } else if constexpr (GEO == kGeoList) {
+        m.klist = a.kv_list + (long long)it * a.kv_count;  // items are ordered (batch, head, tile)
+        m.nkv = a.kv_count * 4;
+    } else {
+        m.nkv = (a.Lk + kBN - 1) / kBN;
+    }
+    return m;
+}
+
+// Position in the CTA's sequence of (item, key step).
+template <int GEO>
+struct Cursor {
+    int it;  // item index (>= a.items once the CTA's items are exhausted)
+    int k;   // the item's position among this CTA's items
+    int j;   // key step within the item
+    Item m;
+    PAB_DEV void start(const FlashTcArgs& a) {
+        it = blockIdx.x;
+        k = j = 0;
+        if (it < a.items) m = decode_item<GEO>(a, it);
+    }
+    PAB_DEV bool valid(const FlashTcArgs& a) const { return it < a.items; }
+    PAB_DEV void next_item(const FlashTcArgs& a) {
+        j = 0;
+        ++k;
+        it += gridDim.x;
+        if (it < a.items) m = decode_item<GEO>(a, it);
+    }
+    PAB_DEV void next(const FlashTcArgs& a) {
+        if (++j == m.nkv) next_item(a);
+    }
+};
+
+// Every barrier completes exactly once per use, so each role derives its
+// wait parities from counters it keeps anyway:
+//   q_full[b][X], q_free[b][X]  once per item with Q buffer b (item k uses k & 1)
+//   slot_full/ready/done[s]     once per ring use s (use u of slot s: u / NST)
+//   p_full[X][b]                once per global step g with g & 1 == b
+//   o_done[X], stage[X]         once per item
+//   xmax_done[X][q][b]          once per exchange of maxima with b == its count & 1
+//   xsum_done[X][q]             once per exchange of row sums
 struct Bars {
-    unsigned long long q_full[2];
-    unsigned long long k01_full;               // K_0, K_1 (own buffer)
-    unsigned long long s01_done[2];            // [tile]: S_X(0), S_X(1) retired
-    unsigned long long b_go;                   // tile A's step-0 maximum is done
-    unsigned long long slot_full[kMaxStages];  // V_j (+ K_{j+2}) landed
-    unsigned long long slot_ready[kMaxStages]; // ... and (ONES) V_j's column d set to 1
-    unsigned long long slot_done[kMaxStages][2];  // [slot][tile]: PV_X(j), S_X(j+2) retired
-    unsigned long long p_full[2][2];           // [tile][S buffer]
-    unsigned long long o_done[2];              // the last PV_X retired
+    unsigned long long q_full[2][2];              // [Q buffer][tile]: Q landed
+    unsigned long long q_free[2][2];              // [Q buffer][tile]: the output staged there was stored
+    unsigned long long b_go;                      // tile A's first row maximum is done
+    unsigned long long slot_full[kMaxStages];     // K_s, V_{s-2} landed
+    unsigned long long slot_ready[kMaxStages];    // ... and (ONES) V's column d set to 1
+    unsigned long long slot_done[kMaxStages][2];  // [slot][tile]: PV_X(s-2), S_X(s) retired
+    unsigned long long p_full[2][2];              // [tile][S buffer]: P written
+    unsigned long long o_done[2];                 // [tile]: the item's last PV retired
+    unsigned long long stage[2];                  // [tile]: the item's output is staged
+    unsigned long long xmax_done[2][4][2];        // [tile][lane quarter][buffer]: both halves' maxima written
+    unsigned long long xsum_done[2][4];           // [tile][lane quarter]: both halves' row sums written
     unsigned long long mma_done[2];
     uint32_t tmem_base;
     int abort;
@@ -137,68 +227,102 @@ PAB_DEV bool wait_bar(Bars* b, unsigned long long* bar, uint32_t parity) {
 // column inside the PV product's N = 16 * KSTEPS -- is set to 1 once the tile
 // lands (warp 11), so O's column d accumulates the row sum of P with the same
 // bf16 P as the numerator; the softmax then keeps no running sum.
-// Tile geometries (GEO != kGeoFull): the CTA's 256 queries are one 16 x 16
+// Tile geometries (GEO != kGeoFull): an item's 256 queries are one 16 x 16
 // tile of the frame (tile A its upper 8 rows, tile B the lower 8, each read
 // as a [8][16]-token TMA box of the [H][W] grid), and the key loop runs over
 // 16 x 16 key tiles, each as four [4][16]-token blocks of 64 keys: the tiles
 // of the window around the query tile, clipped at the frame edge (window),
 // or the tiles listed for it (list; an index outside the frame raises the
 // error word and is clamped).  Every block is whole, so nothing is masked.
+// Operand boxes along d.  Q, K and the staged output of one tile are NB0 full
+// 64-column boxes (128-byte swizzle) plus, when the 16-column K steps leave
+// one or two over, one narrow tail box of 16 or 32 columns (32- or 64-byte
+// swizzle), so a head dim such as 72 (five K steps) holds 80 columns in
+// shared memory instead of 128.  V stays in full boxes: the PV product's
+// N = 16 * KSTEPS columns (the padding column d included) are read MN-major
+// across 64-column atoms.
+template <int KSTEPS>
+struct DLayout {
+    static constexpr int TK0 = KSTEPS % 4;
+    static constexpr int NB0 = KSTEPS / 4 + (TK0 == 3 ? 1 : 0);  // full 64-column boxes
+    static constexpr int TK = TK0 == 3 ? 0 : TK0;                 // K steps in the tail box
+    static constexpr int TB = TK * 32;                            // tail box row bytes (0, 32, 64)
+    static constexpr int NBV = (KSTEPS + 3) / 4;                  // V boxes
+    static constexpr uint32_t QTile = NB0 * kQBox + 128 * TB;
+    static constexpr uint32_t KTile = NB0 * kKVBox + 64 * TB;
+    static constexpr uint32_t VTile = NBV * kKVBox;
+    static constexpr uint32_t tail_swizzle = TB == 32 ? 6u : 4u;  // descriptor layout: 32- / 64-byte swizzle
+    // 16-byte unit u of row r of the tail box, after the TMA swizzle (address
+    // bits 7.. XORed into the unit index)
+    PAB_DEV static uint32_t tail_unit(int r, int u) {
+        return TB == 32 ? (uint32_t)(u ^ ((r >> 2) & 1)) : (uint32_t)(u ^ ((r >> 1) & 3));
+    }
+};
+
+// Softmax split: SPLIT = 2 gives every query row two warps -- the two warps
+// of one TMEM lane quarter on one sub-partition -- each exponentiating 32 of
+// a 64-key tile's scores, so four softmax warps share each sub-partition and
+// hide the exponential pass's latencies (the head dims where the
+// exponentials, not the tensor cores, bound the kernel).  The two halves of
+// a row exchange their maxima through shared memory behind an mbarrier of the
+// pair (a bounded wait, like every wait here), so both take the same
+// rescaling decisions.
+#ifndef PAB_FLASH_SPLIT_KSTEPS
+#define PAB_FLASH_SPLIT_KSTEPS 0  // head dims up to 16 * this many columns split their rows
+#endif
+template <int KSTEPS>
+constexpr int flash_split() { return KSTEPS <= PAB_FLASH_SPLIT_KSTEPS ? 2 : 1; }
+template <int KSTEPS>
+constexpr int flash_threads() { return (8 * flash_split<KSTEPS>() + 4) * 32; }
+
 template <int KSTEPS, int NST, bool ONES, int GEO>
-__global__ void __launch_bounds__(kThreads, 1)
-    flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+__global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
+    flash_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_qt,
+                    const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_kt,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                    FlashTcArgs a) {
-    constexpr int NB = (KSTEPS + 3) / 4;  // 64-column boxes covering d
-    constexpr int NO = KSTEPS * 16;       // N of the PV product (d rounded up to 16)
-    constexpr uint32_t kQTile = NB * kQBox;
-    constexpr uint32_t kKVTile = NB * kKVBox;
+                    const __grid_constant__ CUtensorMap tm_ot, FlashTcArgs a) {
+    static_assert(NST >= 3 && NST <= kMaxStages, "ring depth");
+    using DL = DLayout<KSTEPS>;
+    constexpr int SPLIT = flash_split<KSTEPS>();
+    constexpr int NSW = 8 * SPLIT;           // softmax warps
+    constexpr int W_PROD = NSW, W_MMA = NSW + 1, W_ONES = NSW + 3;
+    constexpr int KC = kBN / SPLIT;          // keys of a tile per softmax warp
+    constexpr int NO = KSTEPS * 16;          // N of the PV product (d rounded up to 16)
+    constexpr int NC = NO / 16;              // 16-column chunks of O
+    constexpr bool TILED = GEO != kGeoFull;
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ Bars bars;
     const uint32_t sbase = (smem_u32(smem_raw) + 1023u) & ~1023u;
-    const uint32_t q_s = sbase;                  // [2 tiles][NB boxes]
-    const uint32_t k01_s = q_s + 2 * kQTile;     // [2][NB boxes]: K_0, K_1
-    const uint32_t v_s = k01_s + 2 * kKVTile;    // [NST][NB boxes]: V_j
-    const uint32_t k_s = v_s + NST * kKVTile;    // [NST][NB boxes]: K_{j+2}
+    const uint32_t q_s = sbase;                      // [2 buffers][2 tiles] Q tiles
+    const uint32_t k_s = q_s + 4 * DL::QTile;        // [NST] K_s
+    const uint32_t v_s = k_s + NST * DL::KTile;      // [NST] V_{s-2}
+    const uint32_t x_s = v_s + NST * DL::VTile;      // SPLIT 2: half-row maxima and sums
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
+    // [step parity][tile][half][row] maxima, [tile][half][row] row sums
+    float* xmax = reinterpret_cast<float*>(gen_base + (x_s - sbase));
+    float* xsum = xmax + 2 * 2 * 2 * 128;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int qblk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-    // tile geometries: query tile (ty, tx); window tiles [wy0, wy0 + rows) x
-    // [wx0, wx0 + wcols); the list of key tiles
-    constexpr bool TILED = GEO != kGeoFull;
-    int ty = 0, tx = 0, wy0 = 0, wx0 = 0, wcols = 1, nkv;
-    const int* klist = nullptr;
-    if constexpr (TILED) {
-        ty = qblk / a.tiles_w;
-        tx = qblk - ty * a.tiles_w;
-    }
-    if constexpr (GEO == kGeoWindow) {
-        wy0 = max(ty - a.reach_h, 0);
-        wx0 = max(tx - a.reach_w, 0);
-        const int wy1 = min(ty + a.reach_h + 1, a.tiles_h), wx1 = min(tx + a.reach_w + 1, a.tiles_w);
-        wcols = wx1 - wx0;
-        nkv = (wy1 - wy0) * wcols * 4;
-    } else if constexpr (GEO == kGeoList) {
-        klist = a.kv_list + (((long long)b * gridDim.y + h) * gridDim.x + qblk) * a.kv_count;
-        nkv = a.kv_count * 4;
-    } else {
-        nkv = (a.Lk + kBN - 1) / kBN;
-    }
-    const bool has_b = TILED || qblk * 2 * kBM + kBM < a.Lq;
-    const int ntiles = has_b ? 2 : 1;
 
-    if (threadIdx.x == 256) {
+    if (threadIdx.x == W_PROD * 32) {
         for (int x = 0; x < 2; ++x) {
-            mbar_init(smem_u32(&bars.q_full[x]), 1);
-            for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&bars.p_full[x][u]), 128);
+            for (int u = 0; u < 2; ++u) {
+                mbar_init(smem_u32(&bars.q_full[u][x]), 1);
+                mbar_init(smem_u32(&bars.q_free[u][x]), 1);
+                mbar_init(smem_u32(&bars.p_full[x][u]), 128 * SPLIT);
+            }
             mbar_init(smem_u32(&bars.o_done[x]), 1);
             mbar_init(smem_u32(&bars.mma_done[x]), 1);
         }
-        mbar_init(smem_u32(&bars.k01_full), 1);
-        for (int x = 0; x < 2; ++x) mbar_init(smem_u32(&bars.s01_done[x]), 1);
-        mbar_init(smem_u32(&bars.b_go), 128);
+        mbar_init(smem_u32(&bars.b_go), 128 * SPLIT);
+        for (int x = 0; x < 2; ++x) {
+            mbar_init(smem_u32(&bars.stage[x]), 128 * SPLIT);
+            for (int q = 0; q < 4; ++q) {
+                mbar_init(smem_u32(&bars.xsum_done[x][q]), 64);
+                for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&bars.xmax_done[x][q][u]), 64);
+            }
+        }
         for (int st = 0; st < NST; ++st) {
             mbar_init(smem_u32(&bars.slot_full[st]), 1);
             mbar_init(smem_u32(&bars.slot_ready[st]), 1);
@@ -210,8 +334,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc::prefetch_tmap(&tm_k);
         tc::prefetch_tmap(&tm_v);
         tc::prefetch_tmap(&tm_o);
+        if constexpr (DL::TK > 0) {
+            tc::prefetch_tmap(&tm_qt);
+            tc::prefetch_tmap(&tm_kt);
+            tc::prefetch_tmap(&tm_ot);
+        }
     }
-    if (warp == 9) {
+    if (warp == W_MMA) {
         tc::tmem_alloc(smem_u32(&bars.tmem_base), kTmemCols);
         tc::tmem_relinquish();
     }
@@ -219,307 +348,452 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = bars.tmem_base;
-    const int kvb = a.kv_batched ? b : 0;
-    // TMA coordinates of query tile x's box and of key block j's box
-    auto load_q = [&](uint32_t dst, int x, int bx, uint32_t bar) {
+
+    // TMA coordinates of query tile x's box at column c0 and of key block j's
+    // box at column c0
+    auto load_q = [&](uint32_t dst, const CUtensorMap* tm, const Item& m, int x, int c0, uint32_t bar) {
         if constexpr (TILED)
-            tc::tma_load_5d(dst, &tm_q, bx * 64, h, tx * 16, ty * 16 + x * 8, b, bar);
+            tc::tma_load_5d(dst, tm, c0, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b, bar);
         else
-            tc::tma_load_4d(dst, &tm_q, bx * 64, h, (qblk * 2 + x) * kBM, b, bar);
+            tc::tma_load_4d(dst, tm, c0, m.h, (m.qblk * 2 + x) * kBM, m.b, bar);
     };
-    auto load_kv = [&](uint32_t dst, const CUtensorMap* m, int j, int bx, uint32_t bar) {
+    auto load_kv = [&](uint32_t dst, const CUtensorMap* tm, const Item& m, int j, int c0, uint32_t bar) {
+        const int kvb = a.kv_batched ? m.b : 0;
         if constexpr (GEO == kGeoWindow) {
-            const int t = j >> 2, ky = wy0 + t / wcols, kx = wx0 + t % wcols;
-            tc::tma_load_5d(dst, m, bx * 64, h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
+            const int t = j >> 2, ky = m.wy0 + t / m.wcols, kx = m.wx0 + t % m.wcols;
+            tc::tma_load_5d(dst, tm, c0, m.h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
         } else if constexpr (GEO == kGeoList) {
-            int tile = __ldg(klist + (j >> 2));
+            int tile = __ldg(m.klist + (j >> 2));
             if (tile < 0 || tile >= a.tiles_h * a.tiles_w) {
                 atomicOr(&g_flash_err, kDevErrBadIndex);
                 tile = tile < 0 ? 0 : a.tiles_h * a.tiles_w - 1;
             }
             const int ky = tile / a.tiles_w, kx = tile - ky * a.tiles_w;
-            tc::tma_load_5d(dst, m, bx * 64, h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
+            tc::tma_load_5d(dst, tm, c0, m.h, kx * 16, ky * 16 + (j & 3) * 4, kvb, bar);
         } else {
-            tc::tma_load_4d(dst, m, bx * 64, h, j * kBN, kvb, bar);
+            tc::tma_load_4d(dst, tm, c0, m.h, j * kBN, kvb, bar);
         }
     };
 
-    if (warp == 8) {
+    if (warp == W_PROD) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
-            for (int x = 0; x < ntiles; ++x) {
-                mbar_arrive_expect_tx(smem_u32(&bars.q_full[x]), kQTile);
-                for (int bx = 0; bx < NB; ++bx)
-                    load_q(q_s + x * kQTile + bx * kQBox, x, bx, smem_u32(&bars.q_full[x]));
-            }
-            const int n01 = nkv < 2 ? nkv : 2;
-            if (n01 > 0) {
-                mbar_arrive_expect_tx(smem_u32(&bars.k01_full), n01 * kKVTile);
-                for (int j = 0; j < n01; ++j)
-                    for (int bx = 0; bx < NB; ++bx)
-                        load_kv(k01_s + j * kKVTile + bx * kKVBox, &tm_k, j, bx, smem_u32(&bars.k01_full));
-            }
-            int nslot = 0;  // slot loads issued
+            Cursor<GEO> ck, cv;  // the K part of ring use s (step s) and its V part (step s - 2)
+            ck.start(a);
+            cv.start(a);
+            int qloads[2] = {0, 0};  // Q loads issued per buffer
+            int s = 0;               // ring uses issued
             bool ok = true;
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j % NST;
-                for (int x = 0; x < ntiles && ok && j >= NST; ++x)
-                    ok = wait_bar(&bars, &bars.slot_done[st][x], ((j / NST) - 1) & 1);
+            for (;; ++s) {
+                const bool has_k = ck.valid(a);
+                const bool has_v = s >= 2 && cv.valid(a);
+                if (s >= 2 && !has_v) break;  // uses 0, 1 always happen (they carry no V)
+                const bool item_start = has_k && ck.j == 0;
+                const Item mq = ck.m;
+                const int kq = ck.k;
+                const int st = s % NST;
+                if (s >= NST)
+                    for (int x = 0; x < 2 && ok; ++x)
+                        ok = wait_bar(&bars, &bars.slot_done[st][x], ((s / NST) - 1) & 1);
                 if (!ok) break;
-                const bool with_k = j + 2 < nkv;
                 const uint32_t bar = smem_u32(&bars.slot_full[st]);
-                mbar_arrive_expect_tx(bar, with_k ? 2 * kKVTile : kKVTile);
-                for (int bx = 0; bx < NB; ++bx) load_kv(v_s + st * kKVTile + bx * kKVBox, &tm_v, j, bx, bar);
-                if (with_k)
-                    for (int bx = 0; bx < NB; ++bx)
-                        load_kv(k_s + st * kKVTile + bx * kKVBox, &tm_k, j + 2, bx, bar);
-                nslot = j + 1;
+                const uint32_t bytes = (has_k ? DL::KTile : 0u) + (has_v ? DL::VTile : 0u);
+                if (bytes)
+                    mbar_arrive_expect_tx(bar, bytes);
+                else
+                    mbar_arrive(bar);  // a use with nothing to carry (a one-step run)
+                if (has_k) {
+                    const uint32_t kt = k_s + st * DL::KTile;
+                    for (int bx = 0; bx < DL::NB0; ++bx) load_kv(kt + bx * kKVBox, &tm_k, ck.m, ck.j, bx * 64, bar);
+                    if constexpr (DL::TK > 0) load_kv(kt + DL::NB0 * kKVBox, &tm_kt, ck.m, ck.j, DL::NB0 * 64, bar);
+                    ck.next(a);
+                }
+                if (has_v) {
+                    for (int bx = 0; bx < DL::NBV; ++bx)
+                        load_kv(v_s + st * DL::VTile + bx * kKVBox, &tm_v, cv.m, cv.j, bx * 64, bar);
+                    cv.next(a);
+                }
+                if (item_start) {
+                    // Q of item k into buffer k & 1 once item k - 2's output staged there was
+                    // stored.  After the ring use: that output's last PV needs this use's V.
+                    const int qb = kq & 1;
+                    if (kq >= 2)
+                        for (int x = 0; x < 2 && ok; ++x)
+                            ok = wait_bar(&bars, &bars.q_free[qb][x], ((kq - 2) >> 1) & 1);
+                    if (!ok) {
+                        ++s;  // this ring use was issued
+                        break;
+                    }
+                    for (int x = 0; x < 2; ++x) {
+                        const uint32_t qbar = smem_u32(&bars.q_full[qb][x]);
+                        const uint32_t qt = q_s + (qb * 2 + x) * DL::QTile;
+                        mbar_arrive_expect_tx(qbar, DL::QTile);
+                        for (int bx = 0; bx < DL::NB0; ++bx) load_q(qt + bx * kQBox, &tm_q, mq, x, bx * 64, qbar);
+                        if constexpr (DL::TK > 0) load_q(qt + DL::NB0 * kQBox, &tm_qt, mq, x, DL::NB0 * 64, qbar);
+                    }
+                    ++qloads[qb];
+                }
             }
             if (!ok || *(volatile int*)&bars.abort) {
                 // drain: let this CTA's loads land before it exits (bounded)
                 for (int st = 0; st < NST; ++st) {
-                    const int uses = (nslot - st + NST - 1) / NST;  // loads issued into slot st
+                    const int uses = (s - st + NST - 1) / NST;  // uses of slot st issued
                     if (uses > 0)
                         mbar_wait_bounded(smem_u32(&bars.slot_full[st]), (uses - 1) & 1, &g_flash_err);
                 }
-                if (n01 > 0) mbar_wait_bounded(smem_u32(&bars.k01_full), 0, &g_flash_err);
-                for (int x = 0; x < ntiles; ++x)
-                    mbar_wait_bounded(smem_u32(&bars.q_full[x]), 0, &g_flash_err);
+                for (int qb = 0; qb < 2; ++qb)
+                    if (qloads[qb] > 0)
+                        for (int x = 0; x < 2; ++x)
+                            mbar_wait_bounded(smem_u32(&bars.q_full[qb][x]), (qloads[qb] - 1) & 1, &g_flash_err);
             }
         }
-    } else if (warp == 9 || warp == 10) {
-        // ------------------------------------------------ MMA issuers
-        // One thread per query tile: a wait of one issuer overlaps the other's
-        // MMA issue, so the tensor core queue stays fed.
-        const int x = warp - 9;
-        if (lane == 0 && x < ntiles) {
-            constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
-            constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
-            // Descriptors are built once; a K step, tile or slot only moves the
-            // start address (bits 0..13, in 16-byte units), which stays below
-            // 2^14 because shared memory is smaller than 256 KB.
-            const uint64_t dq = tc::smem_desc(q_s + x * kQTile, 16, 1024, 2);
-            const uint64_t dk01 = tc::smem_desc(k01_s, 16, 1024, 2);
-            const uint64_t dk = tc::smem_desc(k_s, 16, 1024, 2);
-            const uint64_t dv = tc::smem_desc(v_s, kKVBox, 1024, 2);
-            auto issue_s = [&](uint64_t kdesc, int j) {  // S_X(j) into buffer j & 1
-                const uint32_t d = tmem + x * 128 + (j & 1) * 64;
+    } else if (warp == W_MMA || warp == W_MMA + 1) {
+        // ------------------------------------------------ MMA issuers (warp-uniform)
+        // A wait of one issuer overlaps the other's MMA issue, so the tensor
+        // core queue stays fed.
+        const int x = warp - W_MMA;
+        constexpr uint32_t idesc_s = tc::idesc_bf16(kBM, kBN, 0, 0);
+        constexpr uint32_t idesc_o = tc::idesc_bf16(kBM, NO, 0, 1);
+        // Descriptors are built once; a K step, buffer or slot only moves the
+        // start address (bits 0..13, in 16-byte units), which stays below
+        // 2^14 because shared memory is smaller than 256 KB.
+        const uint64_t dq = tc::smem_desc(q_s + x * DL::QTile, 16, 1024, 2);
+        const uint64_t dk = tc::smem_desc(k_s, 16, 1024, 2);
+        const uint64_t dqt = tc::smem_desc(q_s + x * DL::QTile + DL::NB0 * kQBox, 16, 8 * DL::TB, DL::tail_swizzle);
+        const uint64_t dkt = tc::smem_desc(k_s + DL::NB0 * kKVBox, 16, 8 * DL::TB, DL::tail_swizzle);
+        const uint64_t dv = tc::smem_desc(v_s, kKVBox, 1024, 2);
+        // S_X(s) = Q_X(item) K_s^T into S buffer s & 1
+        auto issue_s = [&](int qb, int st, int buf) {
+            const uint32_t d = tmem + x * 128 + buf * 64;
+            const uint64_t qo = (uint64_t)((qb * 2 * DL::QTile) >> 4), ko = (uint64_t)((st * DL::KTile) >> 4);
 #pragma unroll
-                for (int ks = 0; ks < KSTEPS; ++ks) {
+            for (int ks = 0; ks < KSTEPS; ++ks) {
+                if (ks < DL::NB0 * 4) {
                     const uint32_t offa = (ks >> 2) * (kQBox >> 4) + (ks & 3) * 2;
                     const uint32_t offb = (ks >> 2) * (kKVBox >> 4) + (ks & 3) * 2;
-                    tc::mma_ss(d, dq + offa, kdesc + offb, idesc_s, ks > 0 ? 1u : 0u);
+                    tc::mma_ss_warp(d, dq + qo + offa, dk + ko + offb, idesc_s, ks > 0 ? 1u : 0u);
+                } else {  // tail box: 32 bytes per K step
+                    const uint32_t off = (ks - DL::NB0 * 4) * 2;
+                    tc::mma_ss_warp(d, dqt + qo + off, dkt + ko + off, idesc_s, ks > 0 ? 1u : 0u);
                 }
-            };
-            bool ok = wait_bar(&bars, &bars.q_full[x], 0);
-            if (ok && nkv > 0) ok = wait_bar(&bars, &bars.k01_full, 0);
-            if (ok && nkv > 0) {
-                tc::fence_after_sync();
-                issue_s(dk01, 0);
-                if (nkv > 1) issue_s(dk01 + (kKVTile >> 4), 1);
-                tc::commit(smem_u32(&bars.s01_done[x]));
             }
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j % NST;
-                ok = wait_bar(&bars, ONES ? &bars.slot_ready[st] : &bars.slot_full[st], (j / NST) & 1);
-                if (ok) ok = wait_bar(&bars, &bars.p_full[x][j & 1], (j >> 1) & 1);
-                if (!ok) break;
-                tc::fence_after_sync();
-                // O_X += P_X(j) V_j
-                const uint64_t vdesc = dv + (uint64_t)((st * kKVTile) >> 4);
-                const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128 + (j & 1) * 64;
+        };
+        Cursor<GEO> cs;  // the item and step of the next score product S(s)
+        cs.start(a);
+        bool ok = true;
+        // prologue: S(0), S(1) (ring uses 0 and 1 carry K only)
+        for (int s = 0; s < 2 && ok; ++s) {
+            ok = wait_bar(&bars, &bars.slot_full[s], 0);
+            if (ok && cs.valid(a) && cs.j == 0) ok = wait_bar(&bars, &bars.q_full[cs.k & 1][x], (cs.k >> 1) & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            if (cs.valid(a)) {
+                if (x == 0 || cs.m.has_b) issue_s(cs.k & 1, s, s & 1);
+                cs.next(a);
+            }
+            tc::commit_warp(smem_u32(&bars.slot_done[s][x]));
+        }
+        Cursor<GEO> cp;  // the item and step of P(g)
+        cp.start(a);
+        for (int g = 0; ok && cp.valid(a); ++g) {
+            const int s = g + 2, st = s % NST;
+            ok = wait_bar(&bars, &bars.p_full[x][g & 1], (g >> 1) & 1);
+            if (ok) ok = wait_bar(&bars, ONES ? &bars.slot_ready[st] : &bars.slot_full[st], (s / NST) & 1);
+            if (!ok) break;
+            tc::fence_after_sync();
+            if (x == 0 || cp.m.has_b) {
+                // O_X += P_X(g) V_g
+                const uint64_t vdesc = dv + (uint64_t)((st * DL::VTile) >> 4);
+                const uint32_t d = tmem + 256 + x * 128, pa = tmem + x * 128 + (g & 1) * 64;
 #pragma unroll
                 for (int kk = 0; kk < kBN / 16; ++kk)
-                    tc::mma_ts(d, pa + kk * 8, vdesc + kk * 128, idesc_o, (j > 0 || kk > 0) ? 1u : 0u);
-                // S_X(j+2) reuses the buffer PV_X(j) has just been queued on
-                if (j + 2 < nkv) issue_s(dk + (uint64_t)((st * kKVTile) >> 4), j + 2);
-                tc::commit(smem_u32(&bars.slot_done[st][x]));
-                if (j + 1 == nkv) tc::commit(smem_u32(&bars.o_done[x]));
+                    tc::mma_ts_warp(d, pa + kk * 8, vdesc + kk * 128, idesc_o, (cp.j > 0 || kk > 0) ? 1u : 0u);
             }
-            // all MMAs this thread issued complete before TMEM is released
-            tc::commit(smem_u32(&bars.mma_done[x]));
-            mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_flash_err);
+            // the item's output is complete once its last PV retires; committed
+            // before the next item's Q is waited for (that Q may go where this
+            // output is staged)
+            if (cp.j + 1 == cp.m.nkv) tc::commit_warp(smem_u32(&bars.o_done[x]));
+            // S_X(g+2) reuses the buffer PV_X(g) has just been queued on
+            if (cs.valid(a)) {
+                if (cs.j == 0) ok = wait_bar(&bars, &bars.q_full[cs.k & 1][x], (cs.k >> 1) & 1);
+                if (!ok) break;
+                tc::fence_after_sync();
+                if (x == 0 || cs.m.has_b) issue_s(cs.k & 1, st, s & 1);
+                cs.next(a);
+            }
+            tc::commit_warp(smem_u32(&bars.slot_done[st][x]));
+            cp.next(a);
         }
-    } else if (warp == 11) {
+        // all MMAs this warp issued complete before TMEM is released
+        tc::commit_warp(smem_u32(&bars.mma_done[x]));
+        mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_flash_err);
+    } else if (warp == W_ONES) {
         // ------------------------------------------------ V-ones warp
         if constexpr (ONES) {
             const uint32_t col = (uint32_t)a.d;
             const uint32_t ch = (col & 63) >> 3, e = col & 7;
+            Cursor<GEO> cv;  // the V part of ring use s (step s - 2)
+            cv.start(a);
             bool ok = true;
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j % NST;
-                ok = __all_sync(0xffffffffu, wait_bar(&bars, &bars.slot_full[st], (j / NST) & 1));
+            for (int s = 0; ok; ++s) {
+                const bool has_v = s >= 2 && cv.valid(a);
+                if (s >= 2 && !has_v) break;
+                const int st = s % NST;
+                ok = __all_sync(0xffffffffu, wait_bar(&bars, &bars.slot_full[st], (s / NST) & 1));
                 if (!ok) break;
-                unsigned char* vbox = gen_base + (v_s - sbase) + st * kKVTile + (col >> 6) * kKVBox;
+                if (has_v) {
+                    unsigned char* vbox = gen_base + (v_s - sbase) + st * DL::VTile + (col >> 6) * kKVBox;
 #pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int r = lane + 32 * h2;
-                    *reinterpret_cast<uint16_t*>(vbox + r * 128 + ((ch ^ (r & 7)) << 4) + e * 2) = 0x3F80u;
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int r = lane + 32 * h2;
+                        *reinterpret_cast<uint16_t*>(vbox + r * 128 + ((ch ^ (r & 7)) << 4) + e * 2) = 0x3F80u;
+                    }
+                    fence_proxy_async_smem();
+                    cv.next(a);
                 }
-                fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&bars.slot_ready[st]));
             }
         }
-    } else {
-        // ------------------------------------------------ softmax warpgroups
-        const int x = warp >> 2;  // tile
-        const int row = (warp & 3) * 32 + lane;
-        const uint32_t lane_addr = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+    } else if (warp < NSW) {
+        // ------------------------------------------------ softmax warps
+        const int lq = warp & 3;                       // TMEM lane quarter (= sub-partition)
+        const int x = (warp >> 2) & 1;                 // tile
+        const int hf = SPLIT == 2 ? (warp >> 3) : 0;   // key half of every 64-key tile
+        const int kc0 = hf * KC;                       // first key of this warp's part
+        const int row = lq * 32 + lane;
+        const uint32_t lane_addr = tmem + ((uint32_t)(lq * 32) << 16);
         const uint32_t o_col = 256 + x * 128;
-        float m_ref = -INFINITY, l = 0.f;
-        bool ok = x < ntiles;
-        if (ok && x == 1 && nkv > 0) ok = wait_bar(&bars, &bars.b_go, 0);
-        for (int j = 0; j < nkv && ok; ++j) {
-            const uint32_t s_col = x * 128 + (j & 1) * 64;
-            // S_X(j) was issued with step j-2's slot (or in the prologue)
-            if (j < 2)
-                ok = wait_bar(&bars, &bars.s01_done[x], 0);
-            else
-                ok = wait_bar(&bars, &bars.slot_done[(j - 2) % NST][x], ((j - 2) / NST) & 1);
-            if (!ok) break;
-            tc::fence_after_sync();
-            const int valid = TILED ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
-            // the row's 64 scores fit in registers: one TMEM read
-            float sv[kBN];
-            {
-                uint32_t r0[32], r1[32];
-                tc::ld_32col(lane_addr + s_col + 0, r0);
-                tc::ld_32col(lane_addr + s_col + 32, r1);
-                tc::wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    sv[i] = __uint_as_float(r0[i]);
-                    sv[32 + i] = __uint_as_float(r1[i]);
-                }
-            }
-            if (valid < kBN) {
-#pragma unroll
-                for (int i = 0; i < kBN; ++i)
-                    if (i >= valid) sv[i] = -INFINITY;
-            }
-            // row max of the raw scores (scale > 0 commutes with max): eight
-            // independent 3-input max chains over 8 scores each
-            float mt;
-            {
-                float mx[8];
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    float m = tc::max3f(sv[k], sv[k + 8], sv[k + 16]);
-                    m = tc::max3f(m, sv[k + 24], sv[k + 32]);
-                    m = tc::max3f(m, sv[k + 40], sv[k + 48]);
-                    mx[k] = fmaxf(m, sv[k + 56]);
-                }
-                mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
-                               fmaxf(mx[6], mx[7])) * a.scale_log2;
-            }
-            if (j == 0) {
-                m_ref = mt;
-                if (x == 0) mbar_arrive(smem_u32(&bars.b_go));
-            } else {
-                const bool need = mt > m_ref + kRescaleLog2;
-                if (__any_sync(0xffffffffu, need)) {
-                    // O_X must hold exactly PV_X(0..j-1): PV_X(j-1) retired
-                    // once step j-1's slot is done
-                    ok = wait_bar(&bars, &bars.slot_done[(j - 1) % NST][x], ((j - 1) / NST) & 1);
-                    if (!ok) break;
+        // O's 16-column chunks this warp rescales and stores
+        constexpr int NC0 = SPLIT == 2 ? (NC + 1) / 2 : NC;
+        const int c_lo = hf == 0 ? 0 : NC0, c_hi = hf == 0 ? NC0 : NC;
+        Cursor<GEO> c;
+        c.start(a);
+        bool ok = true;
+        if (x == 1 && c.valid(a)) ok = wait_bar(&bars, &bars.b_go, 0);
+        int g = 0;        // global step
+        int nx = 0, ns = 0;  // exchanges of maxima and of row sums with the row's other half
+        for (; ok && c.valid(a); c.next_item(a)) {
+            const Item m = c.m;
+            const int k = c.k;
+            const bool work = x == 0 || m.has_b;
+            float m_ref = -INFINITY, l = 0.f;
+            for (int j = 0; j < m.nkv; ++j, ++g) {
+                // S_X(g) was issued with ring use g
+                ok = wait_bar(&bars, &bars.slot_done[g % NST][x], (g / NST) & 1);
+                if (!ok) break;
+                if (work) {
                     tc::fence_after_sync();
-                    const float m_new = need ? mt : m_ref;
-                    const float f = ex2(m_ref - m_new);
+                    const uint32_t s_col = x * 128 + (g & 1) * 64;
+                    const int valid = TILED ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
+                    // this warp's scores of the row: one TMEM read each 32 keys
+                    float sv[KC];
+                    {
+                        uint32_t r0[32];
+                        tc::ld_32col(lane_addr + s_col + kc0, r0);
+                        if constexpr (KC == 64) {
+                            uint32_t r1[32];
+                            tc::ld_32col(lane_addr + s_col + 32, r1);
+                            tc::wait_ld();
 #pragma unroll
-                    for (int c = 0; c < NO / 16; ++c) {
-                        uint32_t r[16];
-                        tc::ld_16col(lane_addr + o_col + c * 16, r);
-                        tc::wait_ld();
+                            for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r1[i]);
+                        } else {
+                            tc::wait_ld();
+                        }
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-                        tc::st_16col(lane_addr + o_col + c * 16, r);
+                        for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r0[i]);
                     }
-                    if constexpr (!ONES) l *= f;
-                    m_ref = m_new;
-                }
-            }
-            // exponentiate, sum and write P back as bf16 over S's columns
-            const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
-            const tc::f32x2 negm2 = tc::pack2(-m_ref, -m_ref);
-            tc::f32x2 acc[4];
+                    if (kc0 + KC > valid) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = tc::pack2(0.f, 0.f);
+                        for (int i = 0; i < KC; ++i)
+                            if (kc0 + i >= valid) sv[i] = -INFINITY;
+                    }
+                    // row max of the raw scores (scale > 0 commutes with max):
+                    // eight independent 3-input max chains
+                    float mt;
+                    {
+                        float mx[8];
 #pragma unroll
-            for (int c = 0; c < kBN / 32; ++c) {
-                uint32_t r[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int idx = c * 32 + 2 * i;
-                    const tc::f32x2 t = tc::fma2(tc::pack2(sv[idx], sv[idx + 1]), scale2, negm2);
-                    float t0, t1, p0, p1;
-                    tc::unpack2(t, t0, t1);
-                    if (((idx >> 1) & 7) < kPolyPairsOf8) {
-                        tc::exp2_poly2(t0, t1, p0, p1);
+                        for (int q = 0; q < 8; ++q) {
+                            float mm = tc::max3f(sv[q], sv[q + 8], sv[q + 16]);
+                            if constexpr (KC == 64) {
+                                mm = tc::max3f(mm, sv[q + 24], sv[q + 32]);
+                                mm = tc::max3f(mm, sv[q + 40], sv[q + 48]);
+                                mx[q] = fmaxf(mm, sv[q + 56]);
+                            } else {
+                                mx[q] = fmaxf(mm, sv[q + 24]);
+                            }
+                        }
+                        mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
+                                       fmaxf(mx[6], mx[7])) * a.scale_log2;
+                    }
+                    if constexpr (SPLIT == 2) {
+                        // the two halves of the row meet (double-buffered by exchange
+                        // parity); both take max(own, other), the same value (max is
+                        // exact and order-free).  The wait also orders this half's
+                        // score reads before the other half's P writes over them.
+                        float* xm = xmax + (((nx & 1) * 2 + x) * 2) * 128;
+                        unsigned long long* xb = &bars.xmax_done[x][lq][nx & 1];
+                        xm[hf * 128 + row] = mt;
+                        tc::fence_before_sync();
+                        mbar_arrive(smem_u32(xb));
+                        ok = wait_bar(&bars, xb, (nx >> 1) & 1);
+                        if (!ok) break;
+                        tc::fence_after_sync();
+                        ++nx;
+                        const float mo = xm[(hf ^ 1) * 128 + row];
+                        mt = hf == 0 ? fmaxf(mt, mo) : fmaxf(mo, mt);
+                    }
+                    if (j == 0) {
+                        m_ref = mt;
+                        if (g == 0 && x == 0) mbar_arrive(smem_u32(&bars.b_go));
                     } else {
-                        p0 = ex2(t0);
-                        p1 = ex2(t1);
+                        const bool need = mt > m_ref + kRescaleLog2;
+                        if (__any_sync(0xffffffffu, need)) {
+                            // O_X must hold exactly PV_X(..g-1): PV_X(g-1) was
+                            // committed with ring use g + 1
+                            ok = wait_bar(&bars, &bars.slot_done[(g + 1) % NST][x], ((g + 1) / NST) & 1);
+                            if (!ok) break;
+                            tc::fence_after_sync();
+                            const float m_new = need ? mt : m_ref;
+                            const float f = ex2(m_ref - m_new);
+                            for (int cc = c_lo; cc < c_hi; ++cc) {
+                                uint32_t r[16];
+                                tc::ld_16col(lane_addr + o_col + cc * 16, r);
+                                tc::wait_ld();
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
+                                tc::st_16col(lane_addr + o_col + cc * 16, r);
+                            }
+                            if constexpr (!ONES) l *= f;
+                            m_ref = m_new;
+                        }
                     }
-                    if constexpr (!ONES) acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
-                    r[i] = pack_bf16x2(p0, p1);
+                    // exponentiate, sum and write P back as bf16 over S's columns
+                    // (keys kc0.. as pairs: columns kc0 / 2 ..)
+                    const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
+                    const tc::f32x2 negm2 = tc::pack2(-m_ref, -m_ref);
+                    tc::f32x2 acc[4];
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) acc[q] = tc::pack2(0.f, 0.f);
+#pragma unroll
+                    for (int cc = 0; cc < KC / 32; ++cc) {
+                        uint32_t r[16];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int idx = cc * 32 + 2 * i;
+                            const tc::f32x2 t = tc::fma2(tc::pack2(sv[idx], sv[idx + 1]), scale2, negm2);
+                            float t0, t1, p0, p1;
+                            tc::unpack2(t, t0, t1);
+                            if (((idx >> 1) & 7) < kPolyPairsOf8) {
+                                tc::exp2_poly2(t0, t1, p0, p1);
+                            } else {
+                                p0 = ex2(t0);
+                                p1 = ex2(t1);
+                            }
+                            if constexpr (!ONES) acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
+                            r[i] = pack_bf16x2(p0, p1);
+                        }
+                        tc::st_16col(lane_addr + s_col + kc0 / 2 + cc * 16, r);
+                    }
+                    if constexpr (!ONES) {
+                        float a0, a1;
+                        tc::unpack2(tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3])), a0, a1);
+                        l += a0 + a1;
+                    }
+                    tc::wait_st();
                 }
-                tc::st_16col(lane_addr + s_col + c * 16, r);
+                tc::fence_before_sync();
+                mbar_arrive(smem_u32(&bars.p_full[x][g & 1]));
+                if (j == 0 && k > 0 && hf == 0 && row == 0) {
+                    // the previous item's output store has read its staging: free that Q buffer
+                    bulk_wait_read<0>();
+                    mbar_arrive(smem_u32(&bars.q_free[(k - 1) & 1][x]));
+                }
             }
-            if constexpr (!ONES) {
-                float a0, a1;
-                tc::unpack2(tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3])), a0, a1);
-                l += a0 + a1;
+            if (!ok) break;
+            // ---------------- epilogue: O / l -> bf16 -> swizzled smem -> TMA store
+            ok = wait_bar(&bars, &bars.o_done[x], k & 1);
+            if (!ok) break;
+            // the item's Q buffer: every S of this item has retired
+            unsigned char* stage = gen_base + ((k & 1) * 2 + x) * DL::QTile;
+            if (work) {
+                tc::fence_after_sync();
+                if constexpr (ONES) {  // O's column d: the row sum of P
+                    uint32_t lbits;
+                    tc::ld_1col(lane_addr + o_col + (uint32_t)a.d, lbits);
+                    tc::wait_ld();
+                    l = __uint_as_float(lbits);
+                } else if constexpr (SPLIT == 2) {  // the halves' sums, added in one order
+                    float* xs = xsum + (x * 2) * 128;
+                    xs[hf * 128 + row] = l;
+                    mbar_arrive(smem_u32(&bars.xsum_done[x][lq]));
+                    ok = wait_bar(&bars, &bars.xsum_done[x][lq], ns & 1);
+                    ++ns;
+                    l = xs[row] + xs[128 + row];
+                }
+                const float inv = 1.f / l;
+                for (int cc = c_lo; cc < c_hi; ++cc) {
+                    uint32_t r[16];
+                    tc::ld_16col(lane_addr + o_col + cc * 16, r);
+                    tc::wait_ld();
+                    uint32_t w[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
+                    const int col = cc * 16;
+                    if (col < DL::NB0 * 64) {
+                        const int bx = col >> 6;
+                        const int ch = (col & 63) >> 3;
+                        unsigned char* rowp = stage + bx * kQBox + row * 128;
+                        *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
+                            make_uint4(w[4], w[5], w[6], w[7]);
+                    } else {  // tail box
+                        const int u = (col - DL::NB0 * 64) >> 3;
+                        unsigned char* rowp = stage + DL::NB0 * kQBox + row * DL::TB;
+                        *reinterpret_cast<uint4*>(rowp + (DL::tail_unit(row, u) << 4)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(rowp + (DL::tail_unit(row, u + 1) << 4)) =
+                            make_uint4(w[4], w[5], w[6], w[7]);
+                    }
+                }
+                fence_proxy_async_smem();
             }
-            tc::wait_st();
+            // Every softmax thread of the tile has staged its part once the stage
+            // barrier completes; only the storing thread waits for it (a bounded
+            // wait: no thread can be left behind at a barrier after an abort).
+            // The O columns were read: the next item's first PV, which waits for
+            // every thread's P, may overwrite them.
             tc::fence_before_sync();
-            mbar_arrive(smem_u32(&bars.p_full[x][j & 1]));
-        }
-        // ---------------- epilogue: O / l -> bf16 -> swizzled smem -> TMA store
-        if (ok && nkv > 0) ok = wait_bar(&bars, &bars.o_done[x], 0);
-        if (ok) {
-            tc::fence_after_sync();
-            if constexpr (ONES) {  // O's column d: the row sum of P
-                uint32_t lbits;
-                tc::ld_1col(lane_addr + o_col + (uint32_t)a.d, lbits);
-                tc::wait_ld();
-                l = __uint_as_float(lbits);
+            mbar_arrive(smem_u32(&bars.stage[x]));
+            if (!ok) break;
+            if (hf == 0 && row == 0) ok = wait_bar(&bars, &bars.stage[x], k & 1);
+            if (!ok) break;
+            if (work && hf == 0 && row == 0) {
+                const uint32_t src = q_s + ((k & 1) * 2 + x) * DL::QTile;
+                for (int bx = 0; bx < DL::NB0; ++bx) {
+                    if constexpr (TILED)
+                        tc::tma_store_5d(&tm_o, src + bx * kQBox, bx * 64, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b);
+                    else
+                        tc::tma_store_4d(&tm_o, src + bx * kQBox, bx * 64, m.h, (m.qblk * 2 + x) * kBM, m.b);
+                }
+                if constexpr (DL::TK > 0) {
+                    const uint32_t tsrc = src + DL::NB0 * kQBox;
+                    if constexpr (TILED)
+                        tc::tma_store_5d(&tm_ot, tsrc, DL::NB0 * 64, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b);
+                    else
+                        tc::tma_store_4d(&tm_ot, tsrc, DL::NB0 * 64, m.h, (m.qblk * 2 + x) * kBM, m.b);
+                }
+                bulk_commit();
             }
-            const float inv = 1.f / l;
-            unsigned char* stage = gen_base + x * kQTile;  // this tile's Q buffer (all S MMAs done)
-#pragma unroll
-            for (int c = 0; c < NO / 16; ++c) {
-                uint32_t r[16];
-                tc::ld_16col(lane_addr + o_col + c * 16, r);
-                tc::wait_ld();
-                uint32_t w[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i)
-                    w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                const int col = c * 16;
-                const int bx = col >> 6;
-                const int ch = (col & 63) >> 3;
-                unsigned char* rowp = stage + bx * kQBox + row * 128;
-                *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
-                    make_uint4(w[4], w[5], w[6], w[7]);
-            }
-            fence_proxy_async_smem();
         }
-        tc::named_bar_sync(1 + x, 128);
-        if (ok && row == 0) {
-            for (int bx = 0; bx < NB; ++bx) {
-                if constexpr (TILED)
-                    tc::tma_store_5d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, tx * 16, ty * 16 + x * 8, b);
-                else
-                    tc::tma_store_4d(&tm_o, q_s + x * kQTile + bx * kQBox, bx * 64, h, (qblk * 2 + x) * kBM, b);
-            }
-            bulk_commit();
-            bulk_wait<0>();
-        }
+        // shared memory stays valid until every output store has read it
+        if (hf == 0 && row == 0) bulk_wait_read<0>();
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == W_MMA) {
         __syncwarp();
         tc::fence_after_sync();
         tc::tmem_dealloc(tmem, kTmemCols);
@@ -543,74 +817,127 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
+CUtensorMapSwizzle swizzle_for(int box_cols) {
+    return box_cols >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                          : (box_cols == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
 // 4-D map over a [batches][rows][heads][d] bf16 view (row stride C elements):
-// dims (d, heads, rows, batches), box (64, 1, box_rows, 1), 128-byte swizzle.
+// dims (d, heads, rows, batches), box (box_cols, 1, box_rows, 1), swizzled
+// to the box's row bytes (64 columns: 128-byte; 32: 64-byte; 16: 32-byte).
 bool make_map(CUtensorMap* m, const void* base, int d, int heads, long long rows, long long batches,
-              long long row_stride_elems, long long batch_stride_elems, int box_rows) {
+              long long row_stride_elems, long long batch_stride_elems, int box_rows, int box_cols = 64) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)rows, (cuuint64_t)batches};
     cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)row_stride_elems * 2,
                              (cuuint64_t)(batch_stride_elems > 0 ? batch_stride_elems : rows * row_stride_elems) * 2};
-    cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+    cuuint32_t box[4] = {(cuuint32_t)box_cols, 1, (cuuint32_t)box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_cols),
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
 // 5-D map over the [frames][H][W][heads][d] bf16 spatial view: dims (d,
-// heads, W, H, frames), box (64, 1, 16, box_h, 1) -- 16 * box_h tokens of a
-// 16-wide tile, row-major, one 128-byte swizzled row each.
-bool make_map_grid(CUtensorMap* m, const void* base, int d, int heads, int H, int W, int frames, int box_h) {
+// heads, W, H, frames), box (box_cols, 1, 16, box_h, 1) -- 16 * box_h tokens
+// of a 16-wide tile, row-major, one swizzled row each.
+bool make_map_grid(CUtensorMap* m, const void* base, int d, int heads, int H, int W, int frames, int box_h,
+                   int box_cols = 64) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t C = (cuuint64_t)heads * d;
     cuuint64_t dims[5] = {(cuuint64_t)d, (cuuint64_t)heads, (cuuint64_t)W, (cuuint64_t)H, (cuuint64_t)frames};
     cuuint64_t strides[4] = {(cuuint64_t)d * 2, C * 2, (cuuint64_t)W * C * 2, (cuuint64_t)H * W * C * 2};
-    cuuint32_t box[5] = {64, 1, 16, (cuuint32_t)box_h, 1};
+    cuuint32_t box[5] = {(cuuint32_t)box_cols, 1, 16, (cuuint32_t)box_h, 1};
     cuuint32_t estr[5] = {1, 1, 1, 1, 1};
     CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle_for(box_cols),
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }
 
+// The seven tensor maps of one launch: Q, K, V, O with 64-column boxes and,
+// for head dims with a tail box, Q, K, O with tail-width boxes.
+struct FlashMaps {
+    CUtensorMap q, qt, k, kt, v, o, ot;
+};
+
+// Ring depth: the deepest ring (at most kMaxStages) that fits the 227 KB of
+// shared memory next to the double-buffered Q tiles.
+template <int KSTEPS>
+constexpr int flash_nst() {
+    using DL = DLayout<KSTEPS>;
+    constexpr long long budget = 232448 - 2048;  // static shared memory (barriers) and slack
+    constexpr long long fixed = 4LL * DL::QTile + (flash_split<KSTEPS>() == 2 ? 6144 : 0) + 1024;
+    constexpr long long n = (budget - fixed) / (DL::KTile + DL::VTile);
+    return n > kMaxStages ? kMaxStages : (int)n;
+}
+template <int KSTEPS>
+constexpr size_t flash_smem() {
+    using DL = DLayout<KSTEPS>;
+    return (size_t)4 * DL::QTile + (size_t)flash_nst<KSTEPS>() * (DL::KTile + DL::VTile) +
+           (flash_split<KSTEPS>() == 2 ? 6144 : 0) + 1024;
+}
+
 template <int KSTEPS, bool ONES, int GEO>
-cudaError_t launch_ks1(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
-                       const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
-    constexpr int NB = (KSTEPS + 3) / 4;
-    constexpr int NST = NB == 1 ? 6 : 4;  // ring slots of (V_j, K_{j+2})
-    const size_t smem = (size_t)NB * (2 * kQBox + (2 + 2 * NST) * kKVBox) + 1024;
-    const size_t smem_req = smem < 120 * 1024 ? 120 * 1024 : smem;  // one CTA per SM (TMEM: 512 columns)
-    cudaError_t e = cudaFuncSetAttribute(flash_tc_kernel<KSTEPS, NST, ONES, GEO>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_req);
+cudaError_t launch_ks1(const FlashMaps& m, const FlashTcArgs& a, cudaStream_t s) {
+    constexpr int NST = flash_nst<KSTEPS>();
+    static_assert(NST >= 3, "ring of at least three slots");
+    constexpr size_t smem = flash_smem<KSTEPS>();
+    auto kern = flash_tc_kernel<KSTEPS, NST, ONES, GEO>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    flash_tc_kernel<KSTEPS, NST, ONES, GEO><<<grid, kThreads, smem_req, s>>>(mq, mk, mv, mo, a);
+    // persistent: one CTA per SM (TMEM: 512 columns), each walking its items
+    const int grid = a.items < device_sm_count() ? a.items : device_sm_count();
+    kern<<<grid, flash_threads<KSTEPS>(), smem, s>>>(m.q, m.qt, m.k, m.kt, m.v, m.o, m.ot, a);
     return cudaGetLastError();
 }
 template <int KSTEPS, int GEO>
-cudaError_t launch_ks(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
-                      const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
+cudaError_t launch_ks(const FlashMaps& m, const FlashTcArgs& a, cudaStream_t s) {
     // a padding column inside the PV product carries the row sums when d % 16 != 0
-    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true, GEO>(mq, mk, mv, mo, a, grid, s);
-    return launch_ks1<KSTEPS, false, GEO>(mq, mk, mv, mo, a, grid, s);
+    if (PAB_FLASH_ONES && a.d % 16 != 0) return launch_ks1<KSTEPS, true, GEO>(m, a, s);
+    return launch_ks1<KSTEPS, false, GEO>(m, a, s);
 }
 template <int GEO>
-cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv, const CUtensorMap& mo,
-                     const FlashTcArgs& a, dim3 grid, cudaStream_t s) {
+cudaError_t launch_d(const FlashMaps& m, const FlashTcArgs& a, cudaStream_t s) {
     switch ((a.d + 15) / 16) {
-        case 1: return launch_ks<1, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 2: return launch_ks<2, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 3: return launch_ks<3, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 4: return launch_ks<4, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 5: return launch_ks<5, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 6: return launch_ks<6, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 7: return launch_ks<7, GEO>(mq, mk, mv, mo, a, grid, s);
-        case 8: return launch_ks<8, GEO>(mq, mk, mv, mo, a, grid, s);
+        case 1: return launch_ks<1, GEO>(m, a, s);
+        case 2: return launch_ks<2, GEO>(m, a, s);
+        case 3: return launch_ks<3, GEO>(m, a, s);
+        case 4: return launch_ks<4, GEO>(m, a, s);
+        case 5: return launch_ks<5, GEO>(m, a, s);
+        case 6: return launch_ks<6, GEO>(m, a, s);
+        case 7: return launch_ks<7, GEO>(m, a, s);
+        case 8: return launch_ks<8, GEO>(m, a, s);
         default: return cudaErrorInvalidValue;
     }
+}
+
+// Width in columns of the tail box for head dim d (0: none)
+int tail_cols(int d) {
+    const int ks = (d + 15) / 16, tk = ks % 4;
+    return tk == 3 ? 0 : tk * 16;
+}
+
+// Maps of the tile geometries: Q and O as [8][16]-token boxes, K and V as
+// [4][16]-token boxes of the [frames][H][W] grid.
+bool make_grid_maps(FlashMaps* m, const void* q, const void* k, const void* v, void* out, int d, int heads, int H,
+                    int W, int frames) {
+    if (!make_map_grid(&m->q, q, d, heads, H, W, frames, 8) || !make_map_grid(&m->k, k, d, heads, H, W, frames, 4) ||
+        !make_map_grid(&m->v, v, d, heads, H, W, frames, 4) || !make_map_grid(&m->o, out, d, heads, H, W, frames, 8))
+        return false;
+    const int tw = tail_cols(d);
+    if (!tw) {
+        m->qt = m->q;
+        m->kt = m->k;
+        m->ot = m->o;
+        return true;
+    }
+    return make_map_grid(&m->qt, q, d, heads, H, W, frames, 8, tw) &&
+           make_map_grid(&m->kt, k, d, heads, H, W, frames, 4, tw) &&
+           make_map_grid(&m->ot, out, d, heads, H, W, frames, 8, tw);
 }
 
 }  // namespace
@@ -618,28 +945,41 @@ cudaError_t launch_d(const CUtensorMap& mq, const CUtensorMap& mk, const CUtenso
 cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches, long long Lq,
                          int Lk, int heads, int d, long long q_bstride, long long kv_bstride, cudaStream_t s) {
     if (Lq == 0 || batches == 0) return cudaSuccess;
+    if (Lk < 1 || heads < 1 || batches < 0) return cudaErrorInvalidValue;
     const long long C = (long long)heads * d;
     const long long qblocks = (Lq + 2 * kBM - 1) / (2 * kBM);
-    if (qblocks > 0x7fffffffLL || batches > 65535 || heads > 65535 || Lq > 0x7fffffffLL)
-        return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv, mo;
+    if (qblocks * heads * batches > 0x7fffffffLL || Lq > 0x7fffffffLL) return cudaErrorInvalidValue;
+    FlashMaps m;
     const long long kv_batches = kv_bstride > 0 ? batches : 1;
-    if (!make_map(&mq, q, d, heads, Lq, batches, C, q_bstride, kBM) ||
-        !make_map(&mk, k, d, heads, Lk, kv_batches, C, kv_bstride, kBN) ||
-        !make_map(&mv, v, d, heads, Lk, kv_batches, C, kv_bstride, kBN) ||
-        !make_map(&mo, out, d, heads, Lq, batches, C, q_bstride, kBM))
+    const int tw = tail_cols(d);
+    if (!make_map(&m.q, q, d, heads, Lq, batches, C, q_bstride, kBM) ||
+        !make_map(&m.k, k, d, heads, Lk, kv_batches, C, kv_bstride, kBN) ||
+        !make_map(&m.v, v, d, heads, Lk, kv_batches, C, kv_bstride, kBN) ||
+        !make_map(&m.o, out, d, heads, Lq, batches, C, q_bstride, kBM))
         return cudaErrorInvalidValue;
+    if (tw) {
+        if (!make_map(&m.qt, q, d, heads, Lq, batches, C, q_bstride, kBM, tw) ||
+            !make_map(&m.kt, k, d, heads, Lk, kv_batches, C, kv_bstride, kBN, tw) ||
+            !make_map(&m.ot, out, d, heads, Lq, batches, C, q_bstride, kBM, tw))
+            return cudaErrorInvalidValue;
+    } else {
+        m.qt = m.q;
+        m.kt = m.k;
+        m.ot = m.o;
+    }
     FlashTcArgs a;
     a.Lq = (int)Lq;
     a.Lk = Lk;
     a.kv_batched = kv_bstride > 0 ? 1 : 0;
     a.d = d;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
+    a.heads = heads;
+    a.per_bh = (int)qblocks;
+    a.items = (int)(qblocks * heads * batches);
     a.tiles_h = a.tiles_w = a.reach_h = a.reach_w = 0;
     a.kv_list = nullptr;
     a.kv_count = 0;
-    dim3 grid((unsigned)qblocks, (unsigned)heads, (unsigned)batches);
-    return launch_d<kGeoFull>(mq, mk, mv, mo, a, grid, s);
+    return launch_d<kGeoFull>(m, a, s);
 }
 
 cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
@@ -649,11 +989,9 @@ cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* 
         (win_h / kStaTile) % 2 == 0 || (win_w / kStaTile) % 2 == 0)
         return cudaErrorInvalidValue;
     const long long tiles = (long long)(H / kStaTile) * (W / kStaTile);
-    if (tiles > 0x7fffffffLL || frames > 65535 || heads > 65535) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv, mo;
-    if (!make_map_grid(&mq, q, d, heads, H, W, frames, 8) || !make_map_grid(&mk, k, d, heads, H, W, frames, 4) ||
-        !make_map_grid(&mv, v, d, heads, H, W, frames, 4) || !make_map_grid(&mo, out, d, heads, H, W, frames, 8))
-        return cudaErrorInvalidValue;
+    if (tiles * heads * frames > 0x7fffffffLL || heads < 1) return cudaErrorInvalidValue;
+    FlashMaps m;
+    if (!make_grid_maps(&m, q, k, v, out, d, heads, H, W, frames)) return cudaErrorInvalidValue;
     FlashTcArgs a;
     a.Lq = H * W;
     a.Lk = H * W;
@@ -666,8 +1004,10 @@ cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* 
     a.reach_w = (win_w / kStaTile - 1) / 2;
     a.kv_list = nullptr;
     a.kv_count = 0;
-    dim3 grid((unsigned)tiles, (unsigned)heads, (unsigned)frames);
-    return launch_d<kGeoWindow>(mq, mk, mv, mo, a, grid, s);
+    a.heads = heads;
+    a.per_bh = (int)tiles;
+    a.items = (int)(tiles * heads * frames);
+    return launch_d<kGeoWindow>(m, a, s);
 }
 
 cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
@@ -675,11 +1015,9 @@ cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, 
     if (frames == 0 || H == 0 || W == 0) return cudaSuccess;
     if (H % kStaTile || W % kStaTile || kv_count < 1 || !kv_list) return cudaErrorInvalidValue;
     const long long tiles = (long long)(H / kStaTile) * (W / kStaTile);
-    if (kv_count > tiles || tiles > 0x7fffffffLL || frames > 65535 || heads > 65535) return cudaErrorInvalidValue;
-    CUtensorMap mq, mk, mv, mo;
-    if (!make_map_grid(&mq, q, d, heads, H, W, frames, 8) || !make_map_grid(&mk, k, d, heads, H, W, frames, 4) ||
-        !make_map_grid(&mv, v, d, heads, H, W, frames, 4) || !make_map_grid(&mo, out, d, heads, H, W, frames, 8))
-        return cudaErrorInvalidValue;
+    if (kv_count > tiles || tiles * heads * frames > 0x7fffffffLL || heads < 1) return cudaErrorInvalidValue;
+    FlashMaps m;
+    if (!make_grid_maps(&m, q, k, v, out, d, heads, H, W, frames)) return cudaErrorInvalidValue;
     FlashTcArgs a;
     a.Lq = H * W;
     a.Lk = H * W;
@@ -691,8 +1029,10 @@ cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, 
     a.reach_h = a.reach_w = 0;
     a.kv_list = kv_list;
     a.kv_count = kv_count;
-    dim3 grid((unsigned)tiles, (unsigned)heads, (unsigned)frames);
-    return launch_d<kGeoList>(mq, mk, mv, mo, a, grid, s);
+    a.heads = heads;
+    a.per_bh = (int)tiles;
+    a.items = (int)(tiles * heads * frames);
+    return launch_d<kGeoList>(m, a, s);
 }
 
 unsigned int flash_device_errors(bool clear) {

@@ -31,6 +31,17 @@ cudaError_t launch_swap_outer(const void* src, void* dst, int P, int Q, long lon
                               cudaStream_t s);
 unsigned int layout_device_errors(bool clear);
 
+// --- sequence-parallel exchange: multi-destination block copy --------------
+// Up to kScatterMaxTensors tensors of P * G blocks (block_rows rows of
+// row_bytes); block (p, g) (source index p*G+g for src_order 0, g*P+p for 1)
+// of tensor t goes to dst[t*G + g] + (dst_offset_rows + p*dst_stride_rows)
+// rows.  Destinations may be peer-GPU memory mapped into this process.
+constexpr int kScatterMaxTensors = 3;
+constexpr int kScatterMaxRanks = 32;
+cudaError_t launch_scatter_blocks(const void* const* src, void* const* dst, int ntensors, int G, int P,
+                                  long long block_rows, int row_bytes, int src_order, long long dst_offset_rows,
+                                  long long dst_stride_rows, cudaStream_t s);
+
 // --- temporal short-sequence attention ([N,T,C], L = T) -------------------
 // spatial_view = 1: q, k, v, out are [T, N, C] instead of [N, T, C]
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,

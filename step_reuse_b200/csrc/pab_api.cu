@@ -497,6 +497,94 @@ int pab_permute_blocks(const void* src, void* dst, int P, int Q, long long block
     PAB_GUARD_END
 }
 
+int pab_scatter_blocks(const void* const* src, void* const* dst, int ntensors, int G, int P,
+                       long long block_rows, int C, int src_order, long long dst_offset_rows,
+                       long long dst_stride_rows, int dtype, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (dtype != PAB_BF16 && dtype != PAB_FP32) return fail(PAB_ERR_ARG, "bad dtype %d", dtype);
+    if (ntensors < 1 || ntensors > pab::kScatterMaxTensors)
+        return fail(PAB_ERR_ARG, "ntensors=%d outside [1, %d]", ntensors, pab::kScatterMaxTensors);
+    if (G < 1 || G > pab::kScatterMaxRanks) return fail(PAB_ERR_ARG, "G=%d outside [1, %d]", G, pab::kScatterMaxRanks);
+    if (P < 0 || block_rows < 0 || C < 0 || dst_offset_rows < 0 || dst_stride_rows < 0)
+        return fail(PAB_ERR_ARG, "negative size");
+    if (src_order != 0 && src_order != 1) return fail(PAB_ERR_ARG, "src_order=%d must be 0 or 1", src_order);
+    if ((long long)P * G > 65535) return fail(PAB_ERR_UNSUPPORTED, "P*G=%lld blocks exceed 65535", (long long)P * G);
+    const int elem = dtype == PAB_FP32 ? 4 : 2;
+    const long long row = (long long)C * elem;
+    if ((long long)P * block_rows * C == 0) return PAB_OK;
+    if (row % 16 != 0) return fail(PAB_ERR_UNSUPPORTED, "row of %lld bytes is not a multiple of 16", row);
+    if (!src || !dst) return fail(PAB_ERR_ARG, "null pointer array");
+    if (dst_stride_rows < block_rows && P > 1)
+        return fail(PAB_ERR_ARG, "dst_stride_rows=%lld < block_rows=%lld: destination blocks overlap",
+                    dst_stride_rows, block_rows);
+    for (int t = 0; t < ntensors; ++t)
+        if (!src[t] || !aligned16(src[t])) return fail(PAB_ERR_ARG, "src[%d] null or not 16-byte aligned", t);
+    for (int i = 0; i < ntensors * G; ++i)
+        if (!dst[i] || !aligned16(dst[i])) return fail(PAB_ERR_ARG, "dst[%d] null or not 16-byte aligned", i);
+    // a destination buffer that overlaps a source of the same call
+    const long long src_bytes = (long long)P * G * block_rows * row;
+    const long long dst_bytes = ((dst_offset_rows + (long long)(P - 1) * dst_stride_rows) + block_rows) * row;
+    for (int t = 0; t < ntensors; ++t)
+        for (int i = 0; i < ntensors * G; ++i) {
+            const char* s0 = static_cast<const char*>(src[t]);
+            const char* d0 = static_cast<const char*>(dst[i]);
+            if (s0 < d0 + dst_bytes && d0 < s0 + src_bytes)
+                return fail(PAB_ERR_ARG, "src[%d] and dst[%d] overlap", t, i);
+        }
+    cudaError_t e = pab::launch_scatter_blocks(src, dst, ntensors, G, P, block_rows, (int)row, src_order,
+                                               dst_offset_rows, dst_stride_rows,
+                                               static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "block scatter launch");
+    PAB_GUARD_END
+}
+
+int pab_ipc_alloc(long long bytes, void** ptr, unsigned char handle[64]) {
+    PAB_GUARD_BEGIN
+    if (!ptr || !handle) return fail(PAB_ERR_ARG, "null output pointer");
+    *ptr = nullptr;
+    if (bytes <= 0) return fail(PAB_ERR_ARG, "bytes=%lld must be positive", bytes);
+    void* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, (size_t)bytes);
+    if (e != cudaSuccess) return cuda_fail(e, "IPC buffer allocation");
+    cudaIpcMemHandle_t h;
+    e = cudaIpcGetMemHandle(&h, p);
+    if (e != cudaSuccess) {
+        cudaFree(p);
+        return cuda_fail(e, "cudaIpcGetMemHandle");
+    }
+    static_assert(sizeof(cudaIpcMemHandle_t) == 64, "CUDA IPC handles are 64 bytes");
+    memcpy(handle, &h, 64);
+    *ptr = p;
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+int pab_ipc_free(void* ptr) {
+    if (!ptr) return PAB_OK;
+    cudaError_t e = cudaFree(ptr);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "IPC buffer free");
+}
+
+int pab_ipc_open(const unsigned char handle[64], void** ptr) {
+    PAB_GUARD_BEGIN
+    if (!ptr || !handle) return fail(PAB_ERR_ARG, "null pointer");
+    *ptr = nullptr;
+    cudaIpcMemHandle_t h;
+    memcpy(&h, handle, 64);
+    void* p = nullptr;
+    cudaError_t e = cudaIpcOpenMemHandle(&p, h, cudaIpcMemLazyEnablePeerAccess);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaIpcOpenMemHandle");
+    *ptr = p;
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
+int pab_ipc_close(void* ptr) {
+    if (!ptr) return PAB_OK;
+    cudaError_t e = cudaIpcCloseMemHandle(ptr);
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "cudaIpcCloseMemHandle");
+}
+
 int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype, double* result_dev,
                             void* cuda_stream) {
     PAB_GUARD_BEGIN

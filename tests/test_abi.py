@@ -214,3 +214,44 @@ def test_spatial_alternatives_argument_checks(pab):
             odd.set_spatial_draft(16, 2)
     finally:
         odd.close()
+
+
+def test_scatter_blocks_argument_checks(pab):
+    """The sequence-parallel exchange's argument checks run on the host before
+    any device work (fake aligned addresses: nothing is dereferenced)."""
+    lib = pab.lib
+    VP = ctypes.c_void_p
+
+    def call(nt=1, G=2, P=4, rows=8, C=64, order=0, off=0, stride=8, dtype=0, src=None, dst=None):
+        s = src if src is not None else [0x100000 * (i + 1) for i in range(nt)]
+        d = dst if dst is not None else [0x10000000 + 0x100000 * i for i in range(nt * G)]
+        sa = (VP * max(1, len(s)))(*s)
+        da = (VP * max(1, len(d)))(*d)
+        return lib.pab_scatter_blocks(sa, da, nt, G, P, rows, C, order, off, stride, dtype, None)
+
+    assert call(nt=0) == pab.PAB_ERR_ARG
+    assert call(nt=4) == pab.PAB_ERR_ARG
+    assert call(G=0) == pab.PAB_ERR_ARG
+    assert call(G=33) == pab.PAB_ERR_ARG
+    assert call(order=2) == pab.PAB_ERR_ARG
+    assert call(dtype=7) == pab.PAB_ERR_ARG
+    assert call(P=-1) == pab.PAB_ERR_ARG
+    assert call(C=60) == pab.PAB_ERR_UNSUPPORTED  # 120-byte rows
+    assert call(stride=4) == pab.PAB_ERR_ARG       # destination blocks would overlap
+    assert call(src=[0x100008]) == pab.PAB_ERR_ARG  # misaligned
+    assert call(dst=[0x10000000, 0]) == pab.PAB_ERR_ARG
+    # a destination overlapping the source
+    assert call(src=[0x100000], dst=[0x100000 + 4096, 0x20000000]) == pab.PAB_ERR_ARG
+    assert call(P=0) == pab.PAB_OK  # nothing to move
+    assert lib.pab_scatter_blocks(None, None, 1, 2, 4, 8, 64, 0, 0, 8, 0, None) == pab.PAB_ERR_ARG
+
+
+def test_ipc_argument_checks(pab):
+    lib = pab.lib
+    p = ctypes.c_void_p()
+    h = ctypes.create_string_buffer(64)
+    assert lib.pab_ipc_alloc(0, ctypes.byref(p), h) == pab.PAB_ERR_ARG
+    assert lib.pab_ipc_alloc(64, None, h) == pab.PAB_ERR_ARG
+    assert lib.pab_ipc_open(None, ctypes.byref(p)) == pab.PAB_ERR_ARG
+    assert lib.pab_ipc_free(None) == pab.PAB_OK
+    assert lib.pab_ipc_close(None) == pab.PAB_OK

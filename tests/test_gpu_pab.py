@@ -37,32 +37,36 @@ def oracle_kind(oracle_mod, kind, q, k, v, heads):
     return oracle_mod.cross_attention(q, k, v, heads)
 
 
-def sampled_check(oracle_mod, kind, w, x, out, rng, what):
+SAMPLES = (256, 512, 4096)  # spatial rows per sampled frame, temporal positions, cross rows
+
+
+def sampled_check(oracle_mod, kind, w, x, out, rng, what, sizes=SAMPLES):
     """Compare seeded samples of the output with the oracle computed on just
     those rows (each query row's result depends only on its keys).  Rows are
     gathered on the device first, so only the samples cross to the host."""
     q, k, v = x["q"], x["k"], x["v"]
     dev = q.device
+    n_rows, n_pos, n_cross = sizes
     if kind == "spatial":
         for t in rng.choice(w.T, size=min(2, w.T), replace=False):
-            rows = torch.from_numpy(np.sort(rng.choice(w.N, size=min(256, w.N), replace=False))).to(dev)
+            rows = torch.from_numpy(np.sort(rng.choice(w.N, size=min(n_rows, w.N), replace=False))).to(dev)
             t = int(t)
             # rows of frame t against all keys of frame t
             want = oracle_mod.cross_attention(to_f64(q[t].index_select(0, rows)), to_f64(k[t]),
                                               to_f64(v[t]), w.heads)
             assert_attn_close(out[t].index_select(0, rows), want, f"{what} frame {t}")
     elif kind == "temporal":
-        pos = torch.from_numpy(np.sort(rng.choice(w.N, size=min(512, w.N), replace=False))).to(dev)
+        pos = torch.from_numpy(np.sort(rng.choice(w.N, size=min(n_pos, w.N), replace=False))).to(dev)
         want = oracle_mod.temporal_attention(to_f64(q.index_select(0, pos)), to_f64(k.index_select(0, pos)),
                                              to_f64(v.index_select(0, pos)), w.heads)
         assert_attn_close(out.index_select(0, pos), want, what)
     else:
-        rows = torch.from_numpy(np.sort(rng.choice(w.T * w.N, size=min(4096, w.T * w.N), replace=False))).to(dev)
+        rows = torch.from_numpy(np.sort(rng.choice(w.T * w.N, size=min(n_cross, w.T * w.N), replace=False))).to(dev)
         want = oracle_mod.cross_attention(to_f64(q.index_select(0, rows)), to_f64(k), to_f64(v), w.heads)
         assert_attn_close(out.index_select(0, rows), want, what)
 
 
-def run_pab(pab, oracle_mod, w, ranges, check_steps, full_steps=(), mse_steps=None, seed=0):
+def run_pab(pab, oracle_mod, w, ranges, check_steps, full_steps=(), mse_steps=None, seed=0, sizes=SAMPLES):
     """Run one sampling run; returns per-kind lists of (step, computed, mse)."""
     plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, ranges,
                     dtype=w.torch_dtype)
@@ -97,7 +101,7 @@ def run_pab(pab, oracle_mod, w, ranges, check_steps, full_steps=(), mse_steps=No
                     assert_attn_close(out, want, f"{w.name} {kind} step {i} (full)")
                 elif i in check_steps:
                     bx = {n: xs[n].to(torch.bfloat16) for n in ("q", "k", "v")}
-                    sampled_check(oracle_mod, kind, w, bx, out, rng, f"{w.name} {kind} step {i}")
+                    sampled_check(oracle_mod, kind, w, bx, out, rng, f"{w.name} {kind} step {i}", sizes)
             else:
                 src = int(sched[kind][1][i])
                 s_step, s_ptr, s_clone = saved[kind]
@@ -133,16 +137,16 @@ def test_480p_run(pab, oracle_mod):
 
 @pytest.mark.parametrize("name", ["720p", "temporal_heavy"])
 def test_large_runs_sampled(pab, oracle_mod, name):
-    """Computed steps checked on seeded samples (2 frames x 256 rows spatial,
-    512 positions temporal, 4096 rows cross): every computed step of the
-    temporal-heavy run; at 720p, where one sampled host-side check costs
-    ~20 s, the first step, the first and a later middle step and the last
-    step (all three kinds compute at each), with every other step's schedule
-    and broadcast bytes still checked exactly."""
+    """Every computed step of every kind checked on seeded samples: 2 frames
+    x 256 rows spatial, 512 positions temporal and 4096 rows cross at the
+    temporal-heavy workload; at 720p (3600-token frames, 24 heads of 128,
+    where the fp64 oracle of a sample costs the most) 2 frames x 32 rows,
+    128 positions and 1024 rows, so all 49 computes stay affordable.  Every
+    broadcast step's schedule and bytes are checked exactly."""
     w = synth.WORKLOADS[name]
-    e = oracle_mod.edge_steps(w.steps)
-    steps = {0, e, e + 12, w.steps - 1} if name == "720p" else set(range(w.steps))
-    run_pab(pab, oracle_mod, w, w.ranges, check_steps=steps, mse_steps={1, w.steps - 1})
+    sizes = (32, 128, 1024) if name == "720p" else SAMPLES
+    run_pab(pab, oracle_mod, w, w.ranges, check_steps=set(range(w.steps)), mse_steps={1, w.steps - 1},
+            sizes=sizes)
 
 
 def test_plan_temporal_spatial_view(pab, oracle_mod):
