@@ -84,6 +84,9 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="the 50-step sweep (480p shapes): every range set of the sweep workload timed, "
                          "with the per-step attention difference (MSE) of the all-compute run")
+    ap.add_argument("--kernel", choices=("spatial", "temporal", "temporal_sv", "cross", "layout", "mse"),
+                    help="time one kernel alone on the workload's tensors (one input set, back-to-back "
+                         "launches): the single-kernel view used for profiling")
     ap.add_argument("--dit", action="store_true",
                     help="time the synthetic DiT block (projections, norms, MLP around the library's "
                          "attention) with the workload's PAB ranges and with ranges (1, 1, 1)")
@@ -255,9 +258,12 @@ class AttentionStack:
     fused=False: temporal attention as the three layouts + temporal-view
     kernel + layout back (every step of the hot path runs);
     fused=True: the temporal kernel reads and writes the spatial view itself
-    (pab_plan_set_temporal_view), no layout launches."""
+    (pab_plan_set_temporal_view), no layout launches.
+    mse="fused": each kind's consecutive-compute MSE is accumulated inside its
+    attention kernel (pab_plan_set_diff_mse); "separate": one MSE launch per
+    compute after the first."""
 
-    def __init__(self, pab, w, device, fused=False, window=(), draft=()):
+    def __init__(self, pab, w, device, fused=False, window=(), draft=(), mse="fused"):
         self.pab, self.w, self.dev, self.fused = pab, w, device, fused
         self.plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges,
                              dtype=torch.bfloat16)
@@ -276,6 +282,9 @@ class AttentionStack:
         self.tout = [torch.empty((T, N, C), dtype=torch.bfloat16, device=device) for _ in range(2)]
         self.tslot = 0
         self.mse = torch.zeros((3, w.steps), dtype=torch.float64, device=device)
+        self.mse_mode = mse
+        if mse == "fused":
+            self.plan.set_diff_mse(self.mse)
         self.last_ptr = {}
         self.sched = {k: [self.plan.is_compute(k, i) for i in range(w.steps)] for k in synth.KINDS}
         self.launches_per_run = self._count_launches()
@@ -287,7 +296,7 @@ class AttentionStack:
             for k in synth.KINDS:
                 if self.sched[k][i]:
                     n += 1 if (k != "temporal" or self.fused) else 5  # 3 layouts + attention + layout back
-                    if not first[k]:
+                    if not first[k] and self.mse_mode == "separate":
                         n += 1  # MSE: one launch
                     first[k] = False
         return n
@@ -339,7 +348,7 @@ class AttentionStack:
                     self.last_ptr[k] = ptr
                     shape = (T, N, C) if k == "spatial" else (T * N, C)
                     cur = pab._wrap(ptr, shape, torch.bfloat16, self.dev)
-                if k in prev:
+                if k in prev and self.mse_mode == "separate":
                     timed("mse", lambda: pab.attn_diff_mse_async(cur, prev[k], self.mse[ki, i:i + 1],
                                                                 stream=stream))
                 prev[k] = cur
@@ -469,7 +478,10 @@ def run_ours(args):
 
     n_sets = max(1, min(w.steps, args.input_sets))
     inputs = make_inputs(w, device, n_sets, seed=rank)
-    stack = AttentionStack(pab, w, device)
+    # the headline stack: temporal attention reads and writes the spatial view
+    # (each position's frames gathered with TMA), the attention-difference MSE
+    # accumulated inside the attention kernels
+    stack = AttentionStack(pab, w, device, fused=True)
     stream = torch.cuda.current_stream(device)
 
     for _ in range(args.warmup):
@@ -508,8 +520,12 @@ def run_ours(args):
             continue
         fl = flops.get(name, 0.0) if name != "layout" and name != "mse" else 0.0
         by = abytes[name]
+        if name in synth.KINDS and stack.mse_mode == "fused":
+            # every compute but a kind's first also reads the previous output once (in-kernel MSE)
+            by += (counts[name] - 1) / counts[name] * w.T * w.N * w.C * 2
         ent = {"ms": t, "launches_per_run": len(events[name][0]) // args.steps,
-               "gbs": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak}
+               "gbs": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak,
+               "bytes_per_launch": by}
         if fl:
             ent["tflops"] = fl / (t * 1e-3) / 1e12
             ent["frac_tc"] = ent["tflops"] / tc_peak
@@ -530,7 +546,10 @@ def run_ours(args):
         "config": dict(workload_config(w),
                        l2=f"inputs larger than L2 ({n_sets} drifted input sets of "
                           f"{7 * w.T * w.N * w.C * 2 / 1e6:.0f} MB each, cycled)",
-                       parallelism=f"replicas x{world} (one video per GPU)"),
+                       parallelism=f"replicas x{world} (one video per GPU)",
+                       temporal_view="spatial view: the temporal kernel gathers each position's frames with "
+                                     "TMA (the stack with explicit layout launches is reported beside)",
+                       mse="attention-difference MSE of every compute accumulated inside the attention kernels"),
         "denoising_steps_per_s": world * w.steps / (ms * 1e-3),
         "executed_tflops": world * exec_flops / (ms * 1e-3) / 1e12,
         "computes": counts,
@@ -542,7 +561,7 @@ def run_ours(args):
 
     # the same stack with every step computing (ranges 1, 1, 1): the speedup
     # the broadcast buys on this workload
-    nstack = AttentionStack(pab, dataclasses.replace(w, ranges=(1, 1, 1)), device)
+    nstack = AttentionStack(pab, dataclasses.replace(w, ranges=(1, 1, 1)), device, fused=True)
     nstack.run(inputs, stream)
     nsteps = max(3, args.steps // 10)
     barrier(device)
@@ -561,28 +580,34 @@ def run_ours(args):
     line["speedup_vs_no_broadcast"] = nms / ms
     nstack.close()
 
-    # the same stack with the temporal kernel reading / writing the spatial
-    # view itself (no layout launches): reported beside the main figure
-    fstack = AttentionStack(pab, w, device, fused=True)
+    # the same stack with explicit layout changes around temporal attention
+    # (q, k, v to the temporal view, the output back): reported beside the
+    # main figure, and the layout kernel's own timing comes from it
+    lstack = AttentionStack(pab, w, device, fused=False)
     for _ in range(args.warmup):
-        fstack.run(inputs, stream)
-    fsteps = max(3, args.steps // 4)
+        lstack.run(inputs, stream)
+    lsteps = max(3, args.steps // 4)
+    levents = {}
     barrier(device)
     torch.cuda.synchronize(device)
     f0 = torch.cuda.Event(enable_timing=True)
     f1 = torch.cuda.Event(enable_timing=True)
     f0.record(stream)
-    for _ in range(fsteps):
-        fstack.run(inputs, stream)
+    for _ in range(lsteps):
+        lstack.run(inputs, stream, levents)
     f1.record(stream)
     torch.cuda.synchronize(device)
-    fms = max_over_ranks(f0.elapsed_time(f1) / fsteps, device)
-    line["fused_temporal_view"] = {
-        "value": world * dense_flops / (fms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": fms, "steps": fsteps,
-        "denoising_steps_per_s": world * w.steps / (fms * 1e-3),
-        "gpu_launches": fstack.launches_per_run * fsteps,
-        "note": "temporal attention reads/writes the spatial view via TMA; no layout launches"}
-    fstack.close()
+    lms = max_over_ranks(f0.elapsed_time(f1) / lsteps, device)
+    lay = mean_ms(levents["layout"])
+    kernels["layout"] = {"ms": lay, "launches_per_run": len(levents["layout"][0]) // lsteps,
+                         "gbs": abytes["layout"] / (lay * 1e-3) / 1e9,
+                         "frac_hbm": abytes["layout"] / (lay * 1e-3) / 1e9 / hbm_peak}
+    line["layout_path"] = {
+        "value": world * dense_flops / (lms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": lms, "steps": lsteps,
+        "denoising_steps_per_s": world * w.steps / (lms * 1e-3),
+        "gpu_launches": lstack.launches_per_run * lsteps,
+        "note": "temporal attention on the temporal view, three layout launches before it and one after"}
+    lstack.close()
 
     if not args.no_e2e:
         line["e2e"] = run_e2e(pab, w, stack, device, stream, args)
@@ -639,7 +664,9 @@ def run_e2e(pab, w, stack, device, stream, args):
         sp = pab._wrap(stack.last_ptr["spatial"], (w.T, w.N, w.C), torch.bfloat16, device)
         cr = pab._wrap(stack.last_ptr["cross"], (w.T * w.N, w.C), torch.bfloat16, device)
         outs_host["spatial"].copy_(sp, non_blocking=True)
-        outs_host["temporal"].copy_(stack.tout[stack.tslot], non_blocking=True)
+        tmp = (pab._wrap(stack.last_ptr["temporal"], (w.T, w.N, w.C), torch.bfloat16, device) if stack.fused
+               else stack.tout[stack.tslot])
+        outs_host["temporal"].copy_(tmp, non_blocking=True)
         outs_host["cross"].copy_(cr, non_blocking=True)
         mse_host.copy_(stack.mse, non_blocking=True)
 
@@ -1120,10 +1147,82 @@ def run_dsp(args):
     return 0
 
 
+def run_kernel(args):
+    """One kernel alone: the workload's tensors for that kernel only (q, k, v
+    and the output, or the layout / MSE operands), `warmup` untimed launches,
+    then `steps` launches timed with CUDA events; one JSON line with the
+    kernel's time and its roofline fraction."""
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (no CPU fallback)")
+    device = torch.device("cuda", 0)
+    torch.cuda.set_device(device)
+    import step_reuse_b200 as pab
+
+    w = synth.WORKLOADS[args.workload]
+    T, N, C, L = w.T, w.N, w.C, w.text_len
+    g = torch.Generator(device=device).manual_seed(0)
+    rnd = lambda *shape: torch.randn(shape, generator=g, device=device).to(torch.bfloat16)
+    flops, abytes = w.flops(), algorithmic_bytes(w)
+    kind = args.kernel
+    if kind == "spatial":
+        q, k, v = rnd(T, N, C), rnd(T, N, C), rnd(T, N, C)
+        out = torch.empty_like(q)
+        fn = lambda: pab.spatial_attention(q, k, v, w.heads, out=out)
+    elif kind in ("temporal", "temporal_sv"):
+        q, k, v = rnd(T, N, C), rnd(T, N, C), rnd(T, N, C)  # either view holds T*N rows
+        out = torch.empty_like(q)
+        f = pab.temporal_attention_sv if kind == "temporal_sv" else pab.temporal_attention
+        if kind == "temporal":
+            q, k, v, out = (t.view(N, T, C) for t in (q, k, v, out))
+        fn = lambda: f(q, k, v, w.heads, out=out)
+    elif kind == "cross":
+        q, kt, vt = rnd(T * N, C), rnd(L, C), rnd(L, C)
+        out = torch.empty_like(q)
+        fn = lambda: pab.cross_attention(q, kt, vt, w.heads, out=out)
+    elif kind == "layout":
+        src = rnd(T, N, C)
+        dst = torch.empty((N, T, C), dtype=torch.bfloat16, device=device)
+        fn = lambda: pab.layout(src, True, out=dst)
+    else:
+        a, b = rnd(T * N * C), rnd(T * N * C)
+        res = torch.zeros(1, dtype=torch.float64, device=device)
+        fn = lambda: pab.attn_diff_mse_async(a, b, res)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize(device)
+    clocks = ClockSampler(0)
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark_start()
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize(device)
+    clocks.mark_end()
+    clk = clocks.stop()
+    assert pab.device_errors() == 0
+    ms = e0.elapsed_time(e1) / args.steps
+    peaks = load_peaks()
+    base = kind.replace("_sv", "")
+    by = abytes[base]
+    line = {"metric": f"{kind} kernel alone", "workload": w.name, "ms_per_launch": ms, "launches": args.steps,
+            "warmup": args.warmup, "gbs": by / (ms * 1e-3) / 1e9, "frac_hbm": by / (ms * 1e-3) / 1e9 / peaks["hbm"],
+            "bytes_per_launch": by, "clocks": clk}
+    if base in flops:
+        tf = flops[base] / (ms * 1e-3) / 1e12
+        line.update(tflops=tf, frac_tc=tf / peaks["tc"], flops_per_launch=flops[base])
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
+    if args.kernel:
+        return run_kernel(args)
     if args.sta:
         return run_sta(args)
     if args.draft:

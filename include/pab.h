@@ -223,6 +223,39 @@ int pab_ipc_open(const unsigned char handle[64], void** ptr);
 int pab_ipc_close(void* ptr);
 
 /* ---------------------------------------------------------------------- */
+/* Dense parts of a video DiT block around the attention kinds (PAB report, */
+/* "Implementation": PAB broadcasts the outputs of attention modules that   */
+/* sit in DiT blocks between layer norms, projections and an MLP; a kind    */
+/* that broadcasts also skips its norm and projections).                    */
+/* ---------------------------------------------------------------------- */
+
+/* D = epilogue(A B) on the tensor cores (bf16 inputs, fp32 accumulation):
+ * A [M, K] and B [K, N] bf16 row-major (B holds weights as [in, out]); K a
+ * positive multiple of 8, N a multiple of 32.
+ *   epilogue 0: bf16(A B) into out[0..N/split-1], output i taking columns
+ *               [i*split, (i+1)*split) as an [M, split] row-major matrix
+ *               (split 0: one output of N columns; split a multiple of 32
+ *               dividing N into at most 3 outputs -- one projection for
+ *               q, k and v);
+ *   epilogue 1: bf16(GELU(A B)) into out[0], GELU the tanh form
+ *               0.5 z (1 + tanh(sqrt(2/pi) (z + 0.044715 z^3)));
+ *   epilogue 2: X [M, N] fp32 += A B (the residual stream, read and written),
+ *               and Y [M, N] bf16 = bf16(A B) when Y is not NULL.
+ * out is a HOST array of device pointers; all device pointers 16-byte
+ * aligned.  Outputs must not overlap the inputs. */
+int pab_block_gemm(const void* A, const void* B, int M, int N, int K, int epilogue, void* const* out, int split,
+                   float* X, void* Y, void* cuda_stream);
+
+/* x += ys[0] + ... + ys[ny-1] (each [rows, C] bf16, added in that order;
+ * x [rows, C] fp32 written back) -- the cached outputs of broadcasting
+ * modules added to the residual stream -- then, when h is not NULL,
+ * h [rows, C] bf16 = LayerNorm(x) over each row (no affine parameters, eps
+ * 1e-6; mean and variance in fp32).  ys is a HOST array of ny (0..3) device
+ * pointers.  C a multiple of 8, at most 3072. */
+int pab_block_layer_norm(float* x, const void* const* ys, int ny, void* h, long long rows, int C,
+                         void* cuda_stream);
+
+/* ---------------------------------------------------------------------- */
 /* Attention-difference diagnostic (PAB report, Fig. 1: the difference      */
 /* between consecutive diffusion steps' attention outputs, as MSE).        */
 /* ---------------------------------------------------------------------- */
@@ -318,6 +351,25 @@ int pab_plan_set_spatial_window(pab_plan* plan, int tile, int win_h, int win_w);
  * attention.  A spatial window (pab_plan_set_spatial_window) and a draft
  * setting replace each other.  Same argument rules as pab_draft_select. */
 int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep);
+
+/* Attention-difference diagnostic inside the plan (PAB report, Fig. 1: the
+ * difference between consecutive diffusion steps' attention outputs, as MSE).
+ * With results_dev set -- a DEVICE array of 3 * steps doubles, kind-major,
+ * 8-byte aligned, owned by the caller -- every compute of a kind after the
+ * kind's first compute of the run also writes
+ *   results_dev[kind * steps + step] = mean over T*N*C of (out - prev)^2,
+ * prev being the kind's previous computed output (the plan's other slot).
+ * For PAB_BF16 plans the kind's attention kernel accumulates it in its
+ * epilogue while the new output tile is on chip, so each previous-output
+ * element is read once and no extra kernel runs; per thread the squared
+ * differences of each 8-element vector are summed in fp32 and added in fp64,
+ * CTAs reduce in a fixed order and the last CTA adds the per-CTA sums in CTA
+ * order (bitwise reproducible for a given device).  PAB_FP32 plans run the
+ * MSE kernel after the compute.  Nothing is written for broadcast steps (the
+ * output is the source step's, bit for bit) or for a kind's first compute.
+ * NULL disables.  The first call with a non-NULL array allocates the plan's
+ * reduction scratch on the current device (the plan's device). */
+int pab_plan_set_diff_mse(pab_plan* plan, double* results_dev);
 
 /* Allocate the cache (2 output slots per kind, plus bf16 staging for
  * PAB_FP32 plans) on the current device now instead of at each kind's first

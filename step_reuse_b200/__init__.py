@@ -36,10 +36,10 @@ EXPORTS = (
     "pab_temporal_attention_sv", "pab_plan_set_temporal_view", "pab_sta_attention",
     "pab_plan_set_spatial_window", "pab_draft_workspace_bytes", "pab_draft_select",
     "pab_region_sparse_attention", "pab_plan_set_spatial_draft", "pab_permute_blocks",
-    "pab_scatter_blocks", "pab_ipc_alloc", "pab_ipc_free", "pab_ipc_open", "pab_ipc_close",
+    "pab_scatter_blocks", "pab_block_gemm", "pab_block_layer_norm", "pab_ipc_alloc", "pab_ipc_free", "pab_ipc_open", "pab_ipc_close",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
-    "pab_plan_prepare", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
+    "pab_plan_prepare", "pab_plan_set_diff_mse", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
     "pab_attention",
 )
 
@@ -77,6 +77,8 @@ def _load() -> ctypes.CDLL:
         "pab_layout": ([i, vp, vp, i, i, i, i, vp], i),
         "pab_permute_blocks": ([vp, vp, i, i, ll, i, i, vp], i),
         "pab_scatter_blocks": ([ctypes.POINTER(vp), ctypes.POINTER(vp), i, i, i, ll, i, i, ll, ll, i, vp], i),
+        "pab_block_gemm": ([vp, vp, i, i, i, i, ctypes.POINTER(vp), i, vp, vp, vp], i),
+        "pab_block_layer_norm": ([vp, ctypes.POINTER(vp), i, vp, ll, i, vp], i),
         "pab_ipc_alloc": ([ll, ctypes.POINTER(vp), ctypes.c_char_p], i),
         "pab_ipc_free": ([vp], i),
         "pab_ipc_open": ([ctypes.c_char_p, ctypes.POINTER(vp)], i),
@@ -89,6 +91,7 @@ def _load() -> ctypes.CDLL:
         "pab_plan_destroy": ([vp], i),
         "pab_plan_reset": ([vp], i),
         "pab_plan_prepare": ([vp], i),
+        "pab_plan_set_diff_mse": ([vp, vp], i),
         "pab_schedule_query": ([vp, i, i, ctypes.POINTER(i)], i),
         "pab_schedule_source": ([vp, i, i, ctypes.POINTER(i)], i),
         "pab_schedule_count": ([vp, i, ctypes.POINTER(i)], i),
@@ -277,6 +280,44 @@ def scatter_blocks(srcs, dsts, G: int, P: int, block_rows: int, src_order: int, 
                                   dst_stride_rows, _dtype_code(srcs[0]), _stream(stream)))
 
 
+GEMM_STORE, GEMM_GELU, GEMM_RESID = 0, 1, 2
+
+
+def block_gemm(A, B, epilogue=GEMM_STORE, outs=None, X=None, Y=None, stream=None):
+    """A [M, K] @ B [K, N] (bf16 CUDA tensors) on the tensor cores with an
+    epilogue: GEMM_STORE writes bf16 column blocks into `outs` (1..3 tensors
+    of N / len(outs) columns each; new tensors when None), GEMM_GELU writes
+    bf16 GELU(A B) into outs[0], GEMM_RESID adds A B into the fp32 tensor X
+    (and writes bf16 A B into Y when given).  Returns the outputs."""
+    M, K = A.shape
+    N = B.shape[1]
+    if epilogue == GEMM_RESID:
+        if X is None or X.dtype != torch.float32:
+            raise ValueError("GEMM_RESID needs an fp32 X")
+        arr = (ctypes.c_void_p * 1)(None)
+        _check(lib.pab_block_gemm(_ptr(A), _ptr(B), M, N, K, epilogue, arr, 0, _ptr(X), _ptr(Y), _stream(stream)))
+        return X
+    if outs is None:
+        outs = [torch.empty((M, N), dtype=torch.bfloat16, device=A.device)]
+    split = N // len(outs)
+    arr = (ctypes.c_void_p * len(outs))(*[o.data_ptr() for o in outs])
+    _check(lib.pab_block_gemm(_ptr(A), _ptr(B), M, N, K, epilogue, arr, split if len(outs) > 1 else 0, None, None,
+                              _stream(stream)))
+    return outs
+
+
+def block_layer_norm(x, h=None, ys=(), norm=True, stream=None):
+    """x += sum of the bf16 tensors in `ys` (written back into the fp32 x),
+    then h = bf16(LayerNorm(x)) over the last dim when `norm`."""
+    C = x.shape[-1]
+    if norm and h is None:
+        h = torch.empty(x.shape, dtype=torch.bfloat16, device=x.device)
+    arr = (ctypes.c_void_p * max(1, len(ys)))(*[y.data_ptr() for y in ys])
+    _check(lib.pab_block_layer_norm(_ptr(x), arr, len(ys), _ptr(h) if norm else None, x.numel() // C, C,
+                                    _stream(stream)))
+    return h
+
+
 def ipc_alloc(nbytes: int):
     """(device address, 64-byte handle) of a new buffer that other processes
     of this node can map with ipc_open; release it with ipc_free."""
@@ -407,6 +448,20 @@ class Plan:
 
     def prepare(self):
         _check(lib.pab_plan_prepare(self._h))
+
+    def set_diff_mse(self, results=None):
+        """results: a float64 CUDA tensor of 3 * steps elements ([3, steps]);
+        every compute after a kind's first writes MSE(out, previous compute)
+        at [kind, step] (computed inside the attention kernels for bf16
+        plans).  None disables."""
+        if results is not None:
+            if results.dtype != torch.float64 or results.numel() != 3 * self.steps or not results.is_contiguous():
+                raise ValueError(f"need a contiguous float64 tensor of 3 * {self.steps} elements")
+            self._mse_results = results  # keep the memory alive while the plan writes to it
+            _check(lib.pab_plan_set_diff_mse(self._h, ctypes.c_void_p(results.data_ptr())))
+        else:
+            _check(lib.pab_plan_set_diff_mse(self._h, None))
+            self._mse_results = None
 
     def is_compute(self, kind, step: int) -> bool:
         kind = KIND.get(kind, kind)

@@ -8,6 +8,19 @@
 
 namespace pab {
 
+// The attention-difference MSE (mean of (out - prev)^2 over n elements)
+// fused into an attention launch's epilogue; prev == nullptr: off.  The
+// scratch (one double per CTA plus the completion ticket, zero before the
+// launch and returned to zero by it) is the caller's.
+struct FusedMse {
+    const void* prev;            // the previous output (bf16), same layout as the launch's output
+    double* partials;            // one per CTA of the launch
+    unsigned long long* ticket;  // completion ticket
+    double* result;              // device scalar: the mean
+    double n;                    // elements compared
+};
+constexpr int kFusedMseMaxCtas = 4096;  // partials a fused-MSE scratch holds
+
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
@@ -45,7 +58,7 @@ cudaError_t launch_scatter_blocks(const void* const* src, void* const* dst, int 
 // --- temporal short-sequence attention ([N,T,C], L = T) -------------------
 // spatial_view = 1: q, k, v, out are [T, N, C] instead of [N, T, C]
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
-                            int heads, int d, int spatial_view, cudaStream_t s);
+                            int heads, int d, int spatial_view, cudaStream_t s, const FusedMse* mse = nullptr);
 unsigned int temporal_device_errors(bool clear);
 
 // --- flash attention for spatial (per frame) and cross (shared text K/V) --
@@ -53,20 +66,22 @@ unsigned int temporal_device_errors(bool clear);
 // k/v with kv_bstride (0 = shared K/V).  out has q's layout.
 cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches,
                          long long Lq, int Lk, int heads, int d, long long q_bstride,
-                         long long kv_bstride, cudaStream_t s);
+                         long long kv_bstride, cudaStream_t s, const FusedMse* mse = nullptr);
 // Sliding tile attention within each frame of a [frames][H*W][heads*d] bf16
 // spatial view: 16 x 16-token tiles, a window of win_h x win_w tokens (odd
 // tile counts) centred on the query's tile and clipped at the frame edge.
 // H, W, win_h, win_w must be multiples of 16 (cudaErrorInvalidValue else).
 cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
-                             int heads, int d, int win_h, int win_w, cudaStream_t s);
+                             int heads, int d, int win_h, int win_w, cudaStream_t s,
+                             const FusedMse* mse = nullptr);
 
 // Attention of every 16 x 16 query tile of each frame over the 16 x 16 key
 // tiles kv_list names for it: [frames][heads][tiles][kv_count] tile indices
 // (ty * (W/16) + tx) of the same frame.  An index outside the frame raises
 // kDevErrBadIndex in the flash status word and is clamped.
 cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
-                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s);
+                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s,
+                                   const FusedMse* mse = nullptr);
 
 unsigned int flash_device_errors(bool clear);
 
@@ -80,8 +95,22 @@ cudaError_t launch_draft_select(const void* q, const void* k, int T, int H, int 
 
 // --- cross attention (text_len <= 128: persistent cross_tc; longer: flash) --
 cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,
-                         int d, cudaStream_t s);
+                         int d, cudaStream_t s, const FusedMse* mse = nullptr);
 unsigned int cross_device_errors(bool clear);
+
+// --- dense parts of a DiT block around the attention kinds ----------------
+// D = epilogue(A B): A [M, K] bf16 row-major, B [K, N] bf16 row-major, K a
+// multiple of 8, N of 32.  epi 0: bf16 outputs out[0..2] of `split` columns
+// each (split 0: one output of N columns); 1: bf16(GELU_tanh(.)) into out[0];
+// 2: X [M, N] fp32 += A B, and Y [M, N] bf16 = A B when Y is not null.
+cudaError_t launch_gemm(const void* A, const void* B, int M, int N, int K, int epi, void* const* out, int split,
+                        float* X, void* Y, cudaStream_t s);
+// x += ys[0] + ... + ys[ny-1] (bf16, in that order; x fp32 written back),
+// then h [rows, C] bf16 = LayerNorm(x) (no affine) when h is not null.
+// C % 4 == 0, C <= 3072, ny <= 3.
+cudaError_t launch_ln_rows(float* x, const void* const* ys, int ny, void* h, long long rows, int C, float eps,
+                           cudaStream_t s);
+unsigned int block_device_errors(bool clear);
 
 // --- dtype conversion for fp32 plans --------------------------------------
 cudaError_t launch_f32_to_bf16(const float* src, void* dst, long long n, cudaStream_t s);

@@ -101,10 +101,10 @@ int check_ptrs(const char* names, const void* a, const void* b, const void* c, c
 }
 
 int run_spatial(const void* q, const void* k, const void* v, void* out, int T, int N, int heads,
-                int d, cudaStream_t s) {
+                int d, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
     const long long C = (long long)heads * d;
     cudaError_t e = pab::launch_flash(q, k, v, out, T, N, N, heads, d, (long long)N * C,
-                                      (long long)N * C, s);
+                                      (long long)N * C, s, mse);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "spatial attention launch");
 }
 
@@ -119,8 +119,8 @@ int check_sta(int H, int W, int tile, int win_h, int win_w) {
 }
 
 int run_sta(const void* q, const void* k, const void* v, void* out, int T, int H, int W, int heads, int d,
-            int win_h, int win_w, cudaStream_t s) {
-    cudaError_t e = pab::launch_flash_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, s);
+            int win_h, int win_w, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
+    cudaError_t e = pab::launch_flash_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, s, mse);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "sliding tile attention launch");
 }
 
@@ -134,22 +134,22 @@ int check_draft(int H, int W, int region, int keep) {
 }
 
 int run_draft(const void* q, const void* k, const void* v, void* out, int T, int H, int W, int heads, int d,
-              int keep, int* sel, void* sketch, cudaStream_t s) {
+              int keep, int* sel, void* sketch, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
     cudaError_t e = pab::launch_draft_select(q, k, T, H, W, heads, d, keep, sel, sketch, s);
     if (e != cudaSuccess) return cuda_fail(e, "draft selection launch");
-    e = pab::launch_flash_tile_list(q, k, v, out, T, H, W, heads, d, sel, keep, s);
+    e = pab::launch_flash_tile_list(q, k, v, out, T, H, W, heads, d, sel, keep, s, mse);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "region-sparse attention launch");
 }
 
 int run_temporal(const void* q, const void* k, const void* v, void* out, int N, int T, int heads,
-                 int d, int spatial_view, cudaStream_t s) {
-    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s);
+                 int d, int spatial_view, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
+    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s, mse);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "temporal attention launch");
 }
 
 int run_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lt,
-              int heads, int d, cudaStream_t s) {
-    cudaError_t e = pab::launch_cross(q, kt, vt, out, R, Lt, heads, d, s);
+              int heads, int d, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
+    cudaError_t e = pab::launch_cross(q, kt, vt, out, R, Lt, heads, d, s, mse);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "cross attention launch");
 }
 
@@ -199,6 +199,10 @@ struct pab_plan {
     int cur[3];          // slot holding the latest computed output, -1 = none
     int cached_step[3];  // step of that compute
     int last_step[3];    // last step seen (order check)
+    // attention-difference MSE of consecutive computes, written to the
+    // caller's device array [3][steps]; fp64 scratch: ticket + partials
+    double* mse_results;
+    double* mse_scratch;
     // bf16 staging for fp32 plans
     void* stage_in[3];
     void* stage_out;
@@ -230,6 +234,8 @@ void plan_free_device(pab_plan* p) {
     p->stage_out = nullptr;
     if (p->draft_sel) cudaFree(p->draft_sel);
     if (p->draft_sketch) cudaFree(p->draft_sketch);
+    if (p->mse_scratch) cudaFree(p->mse_scratch);
+    p->mse_scratch = nullptr;
     p->draft_sel = nullptr;
     p->draft_sketch = nullptr;
     p->device = -1;
@@ -272,7 +278,7 @@ int plan_alloc_kind(pab_plan* p, int kind) {
 }
 
 int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void* v, void* out,
-                 cudaStream_t s) {
+                 cudaStream_t s, const void* prev, double* mse_result) {
     const long long qn = (long long)p->T * p->N * p->C;
     const long long kvn = (kind == PAB_CROSS) ? (long long)p->text_len * p->C : qn;
     const void *qq = q, *kk = k, *vv = v;
@@ -290,22 +296,32 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
         vv = p->stage_in[2];
         oo = p->stage_out;
     }
+    // bf16 plans: the kind's kernel accumulates the difference to the previous
+    // output in its epilogue; fp32 plans: the MSE kernel runs after the compute
+    pab::FusedMse fm{prev, p->mse_scratch + 1, reinterpret_cast<unsigned long long*>(p->mse_scratch),
+                     mse_result, (double)qn};
+    const pab::FusedMse* mse = (prev && p->dtype == PAB_BF16) ? &fm : nullptr;
     int rc;
     if (kind == PAB_SPATIAL && p->draft_keep > 0)
         rc = run_draft(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->draft_keep, p->draft_sel,
-                       p->draft_sketch, s);
+                       p->draft_sketch, s, mse);
     else if (kind == PAB_SPATIAL && p->sta_win_h > 0)
-        rc = run_sta(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->sta_win_h, p->sta_win_w, s);
+        rc = run_sta(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->sta_win_h, p->sta_win_w, s, mse);
     else if (kind == PAB_SPATIAL)
-        rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s);
+        rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s, mse);
     else if (kind == PAB_TEMPORAL)
-        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, p->temporal_sv, s);
+        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, p->temporal_sv, s, mse);
     else
-        rc = run_cross(qq, kk, vv, oo, (long long)p->T * p->N, p->text_len, p->heads, p->d, s);
+        rc = run_cross(qq, kk, vv, oo, (long long)p->T * p->N, p->text_len, p->heads, p->d, s, mse);
     if (rc) return rc;
     if (p->dtype == PAB_FP32) {
         cudaError_t e = pab::launch_bf16_to_f32(p->stage_out, static_cast<float*>(out), qn, s);
         if (e != cudaSuccess) return cuda_fail(e, "bf16 -> fp32 conversion");
+        if (prev) {
+            const int parts = pab::mse_num_partials(qn, 4);
+            e = pab::launch_mse(out, prev, qn, PAB_FP32, p->mse_scratch, parts, mse_result, s);
+            if (e != cudaSuccess) return cuda_fail(e, "attention-difference MSE launch");
+        }
     }
     return PAB_OK;
 }
@@ -585,6 +601,47 @@ int pab_ipc_close(void* ptr) {
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "cudaIpcCloseMemHandle");
 }
 
+int pab_block_gemm(const void* A, const void* B, int M, int N, int K, int epilogue, void* const* out, int split,
+                   float* X, void* Y, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (M < 0 || N < 0 || K < 0) return fail(PAB_ERR_ARG, "negative size");
+    if (epilogue < 0 || epilogue > 2) return fail(PAB_ERR_ARG, "bad epilogue %d", epilogue);
+    if ((long long)M * N == 0) return PAB_OK;
+    if (K == 0 || K % 8) return fail(PAB_ERR_UNSUPPORTED, "K=%d must be a positive multiple of 8", K);
+    if (N % 32) return fail(PAB_ERR_UNSUPPORTED, "N=%d must be a multiple of 32", N);
+    if (!A || !B || !aligned16(A) || !aligned16(B)) return fail(PAB_ERR_ARG, "A/B null or not 16-byte aligned");
+    if (epilogue == 2) {
+        if (!X || !aligned16(X)) return fail(PAB_ERR_ARG, "X null or not 16-byte aligned");
+        if (Y && !aligned16(Y)) return fail(PAB_ERR_ARG, "Y not 16-byte aligned");
+    } else {
+        const int sp = split > 0 ? split : N;
+        if (sp % 32 || N % sp || N / sp > 3)
+            return fail(PAB_ERR_ARG, "split=%d must divide N=%d into at most 3 outputs of a multiple of 32", split, N);
+        if (epilogue == 1 && sp != N) return fail(PAB_ERR_ARG, "the GELU epilogue has one output");
+        if (!out) return fail(PAB_ERR_ARG, "null output array");
+        for (int i = 0; i < N / sp; ++i)
+            if (!out[i] || !aligned16(out[i])) return fail(PAB_ERR_ARG, "out[%d] null or not 16-byte aligned", i);
+    }
+    cudaError_t e = pab::launch_gemm(A, B, M, N, K, epilogue, out, split, X, Y, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "block GEMM launch");
+    PAB_GUARD_END
+}
+
+int pab_block_layer_norm(float* x, const void* const* ys, int ny, void* h, long long rows, int C,
+                         void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (rows < 0 || C <= 0) return fail(PAB_ERR_ARG, "rows=%lld, C=%d", rows, C);
+    if (ny < 0 || ny > 3 || (ny > 0 && !ys)) return fail(PAB_ERR_ARG, "ny=%d outside [0, 3] or null array", ny);
+    if (rows == 0) return PAB_OK;
+    if (C % 8 || C > 3072) return fail(PAB_ERR_UNSUPPORTED, "C=%d must be a multiple of 8, at most 3072", C);
+    if (!x || !aligned16(x) || (h && !aligned16(h))) return fail(PAB_ERR_ARG, "null or misaligned pointer");
+    for (int j = 0; j < ny; ++j)
+        if (!ys[j] || !aligned16(ys[j])) return fail(PAB_ERR_ARG, "ys[%d] null or not 16-byte aligned", j);
+    cudaError_t e = pab::launch_ln_rows(x, ys, ny, h, rows, C, 1e-6f, static_cast<cudaStream_t>(cuda_stream));
+    return e == cudaSuccess ? PAB_OK : cuda_fail(e, "layer norm launch");
+    PAB_GUARD_END
+}
+
 int pab_attn_diff_mse_async(const void* a, const void* b, long long n, int dtype, double* result_dev,
                             void* cuda_stream) {
     PAB_GUARD_BEGIN
@@ -633,8 +690,9 @@ int pab_attn_diff_mse(const void* a, const void* b, long long n, int dtype, doub
 int pab_device_errors(int clear, unsigned int* flags) {
     PAB_GUARD_BEGIN
     if (!flags) return fail(PAB_ERR_ARG, "null flags pointer");
-    const unsigned int words[4] = {pab::layout_device_errors(clear != 0), pab::flash_device_errors(clear != 0),
-                                   pab::temporal_device_errors(clear != 0), pab::cross_device_errors(clear != 0)};
+    const unsigned int words[5] = {pab::layout_device_errors(clear != 0), pab::flash_device_errors(clear != 0),
+                                   pab::temporal_device_errors(clear != 0), pab::cross_device_errors(clear != 0),
+                                   pab::block_device_errors(clear != 0)};
     unsigned int v = 0;
     for (unsigned int w : words) {
         if (w == 0xffffffffu) return fail(PAB_ERR_CUDA, "could not read the device status words");
@@ -761,6 +819,26 @@ int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep) {
     PAB_GUARD_END
 }
 
+int pab_plan_set_diff_mse(pab_plan* plan, double* results_dev) {
+    PAB_GUARD_BEGIN
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    if (results_dev && (reinterpret_cast<uintptr_t>(results_dev) & 7u))
+        return fail(PAB_ERR_ARG, "results_dev not 8-byte aligned");
+    if (results_dev && !plan->mse_scratch) {
+        const int need = pab::kFusedMseMaxCtas + 1;
+        cudaError_t e = cudaMalloc(&plan->mse_scratch, sizeof(double) * need);
+        if (e != cudaSuccess) {
+            plan->mse_scratch = nullptr;
+            return cuda_fail(e, "MSE scratch allocation");
+        }
+        e = cudaMemset(plan->mse_scratch, 0, sizeof(unsigned long long));  // the completion ticket
+        if (e != cudaSuccess) return cuda_fail(e, "MSE scratch clear");
+    }
+    plan->mse_results = results_dev;
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
 int pab_plan_prepare(pab_plan* plan) {
     PAB_GUARD_BEGIN
     if (!plan) return fail(PAB_ERR_ARG, "null plan");
@@ -819,7 +897,15 @@ int pab_attention(pab_plan* plan, int kind, int step, const void* q, const void*
     rc = plan_alloc_kind(plan, kind);
     if (rc) return rc;
     const int slot = plan->cur[kind] < 0 ? 0 : 1 - plan->cur[kind];
-    rc = plan_compute(plan, kind, q, k, v, plan->slot[kind][slot], static_cast<cudaStream_t>(cuda_stream));
+    // the attention-difference MSE against the kind's previous compute of this run
+    const void* prev = nullptr;
+    double* mse_result = nullptr;
+    if (plan->mse_results && plan->cur[kind] >= 0) {
+        prev = plan->slot[kind][plan->cur[kind]];
+        mse_result = plan->mse_results + (long long)kind * plan->steps + step;
+    }
+    rc = plan_compute(plan, kind, q, k, v, plan->slot[kind][slot], static_cast<cudaStream_t>(cuda_stream), prev,
+                      mse_result);
     if (rc) return rc;
     plan->cur[kind] = slot;
     plan->cached_step[kind] = step;

@@ -4,8 +4,7 @@ The PAB report ("Implementation") places the three attention kinds inside
 the DiT blocks of a video diffusion model and broadcasts each kind's
 attention output to the following steps of its range; the speedups it
 quotes (up to 35% from broadcast alone) are for whole models.  This block
-measures that effect on one GPU with random weights, around the library's
-own kernels:
+measures that effect on one GPU with random weights:
 
     x <- x + A_spatial(LN(x))            A_kind(h) = Attn_kind(h Wq, h Wk, h Wv) Wo
     x <- x + A_temporal(LN(x))           (cross: keys and values from the text)
@@ -13,17 +12,24 @@ own kernels:
     x <- x + GELU(LN(x) W1) W2
 
 LN is a layer norm over C without affine parameters (eps 1e-6), GELU the
-tanh form.  The attention runs through the C ABI (pab_attention; temporal
-attention on the spatial view, no layout change).  Projections, norms and
-the MLP are plain library operations (cuBLAS GEMMs in bf16 with fp32
-accumulation, PyTorch's layer norm and GELU); the residual stream is fp32.
+tanh form; the residual stream x is fp32, everything the tensor cores read
+is bf16.  Every operation runs in the library's kernels (C ABI):
+  * LN -- pab_block_layer_norm, which also adds the cached outputs of the
+    kinds that broadcast since the previous norm (up to three) into x;
+  * the q, k, v projections -- one pab_block_gemm with Wq | Wk | Wv
+    concatenated, its epilogue writing q, k and v as three tensors (cross:
+    q from the video tokens, k | v from the text);
+  * the attention -- pab_attention (temporal attention on the spatial view);
+  * the output projection -- pab_block_gemm whose epilogue adds A_kind into
+    x in fp32 and keeps bf16(A_kind) for the broadcast steps;
+  * the MLP -- pab_block_gemm with GELU in the epilogue of W1 and the
+    residual add in the epilogue of W2.
 A kind that broadcasts at a step adds the module output it computed at its
 latest computing step: its norm, projections and attention are all skipped.
 """
 from __future__ import annotations
 
 import torch
-import torch.nn.functional as F
 
 KINDS = ("spatial", "temporal", "cross")
 LN_EPS = 1e-6
@@ -48,10 +54,23 @@ class DiTBlock:
     def __init__(self, pab, T, H, W, heads, d, text_len, steps, ranges, weights, device="cuda"):
         self.pab = pab
         self.T, self.N, self.C, self.heads, self.d = T, H * W, heads * d, heads, d
+        R, C = T * H * W, heads * d
         self.w = weights
+        # the projections of each kind as one [C, 3C] (cross: q [C, C] and the
+        # text's k | v [C, 2C]) matrix
+        cat = lambda *ms: torch.cat([weights[m] for m in ms], dim=1).contiguous()
+        self.wqkv = {k: cat(f"{k}.wq", f"{k}.wk", f"{k}.wv") for k in ("spatial", "temporal")}
+        self.wq_cross = weights["cross.wq"]
+        self.wkv_cross = cat("cross.wk", "cross.wv")
         self.plan = pab.Plan(T, H, W, heads, d, text_len, steps, ranges, dtype=torch.bfloat16)
         self.plan.set_temporal_view(True)
         self.plan.prepare()
+        bf = dict(dtype=torch.bfloat16, device=device)
+        self.h = torch.empty((R, C), **bf)
+        self.q, self.k, self.v = (torch.empty((R, C), **bf) for _ in range(3))
+        self.kt, self.vt = (torch.empty((text_len, C), **bf) for _ in range(2))
+        self.hid = torch.empty((R, 4 * C), **bf)
+        self.mods = {kind: torch.empty((T, H * W, C), **bf) for kind in KINDS}
         self.cache = {}
         self.device = device
 
@@ -63,31 +82,33 @@ class DiTBlock:
         self.plan.reset()
         self.cache = {}
 
-    def _ln(self, x):
-        return F.layer_norm(x, (self.C,), eps=LN_EPS).to(torch.bfloat16)
-
-    def _module(self, kind, step, x, text, stream):
-        T, N, C, w = self.T, self.N, self.C, self.w
-        h = self._ln(x).view(T * N, C)
-        q = (h @ w[f"{kind}.wq"]).view(T, N, C)
-        if kind == "cross":
-            k, v = text @ w["cross.wk"], text @ w["cross.wv"]
-            q = q.view(T * N, C)
-        else:
-            k = (h @ w[f"{kind}.wk"]).view(T, N, C)
-            v = (h @ w[f"{kind}.wv"]).view(T, N, C)
-        a = self.plan.attention(kind, step, q, k, v, stream)
-        return (a.reshape(T * N, C) @ w[f"{kind}.wo"]).view(T, N, C)
-
     def step(self, step: int, x: torch.Tensor, text: torch.Tensor, stream=None) -> torch.Tensor:
         """Block output at diffusion step `step` for x [T, N, C] (fp32) and the
         text [text_len, C] (bf16); returns a new fp32 tensor."""
+        pab, T, N, C = self.pab, self.T, self.N, self.C
+        R = T * N
         x = x.float().clone()
+        xr = x.view(R, C)
+        pending = []  # broadcast module outputs not yet added to x
         for kind in KINDS:
-            if self.plan.is_compute(kind, step):
-                self.cache[kind] = self._module(kind, step, x, text, stream)
-            x += self.cache[kind].float()
-        h = self._ln(x).view(self.T * self.N, self.C)
-        y = F.gelu((h @ self.w["mlp.w1"]).float(), approximate="tanh").to(torch.bfloat16) @ self.w["mlp.w2"]
-        x += y.view(self.T, self.N, self.C).float()
+            if not self.plan.is_compute(kind, step):
+                pending.append(self.cache[kind].view(R, C))
+                continue
+            pab.block_layer_norm(xr, self.h, ys=pending, stream=stream)
+            pending = []
+            if kind == "cross":
+                pab.block_gemm(self.h, self.wq_cross, outs=[self.q], stream=stream)
+                pab.block_gemm(text, self.wkv_cross, outs=[self.kt, self.vt], stream=stream)
+                a = self.plan.attention(kind, step, self.q, self.kt, self.vt, stream)
+            else:
+                pab.block_gemm(self.h, self.wqkv[kind], outs=[self.q, self.k, self.v], stream=stream)
+                a = self.plan.attention(kind, step, self.q.view(T, N, C), self.k.view(T, N, C),
+                                        self.v.view(T, N, C), stream)
+            # x += A_kind in fp32; bf16(A_kind) kept for the broadcast steps
+            pab.block_gemm(a.reshape(R, C), self.w[f"{kind}.wo"], pab.GEMM_RESID, X=xr,
+                           Y=self.mods[kind].view(R, C), stream=stream)
+            self.cache[kind] = self.mods[kind]
+        pab.block_layer_norm(xr, self.h, ys=pending, stream=stream)
+        pab.block_gemm(self.h, self.w["mlp.w1"], pab.GEMM_GELU, outs=[self.hid], stream=stream)
+        pab.block_gemm(self.hid, self.w["mlp.w2"], pab.GEMM_RESID, X=xr, stream=stream)
         return x
