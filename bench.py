@@ -259,11 +259,10 @@ class AttentionStack:
     kernel + layout back (every step of the hot path runs);
     fused=True: the temporal kernel reads and writes the spatial view itself
     (pab_plan_set_temporal_view), no layout launches.
-    mse="fused": each kind's consecutive-compute MSE is accumulated inside its
-    attention kernel (pab_plan_set_diff_mse); "separate": one MSE launch per
-    compute after the first."""
+    Every compute of a kind after its first is followed by one MSE launch
+    against the kind's previous output (the attention-difference diagnostic)."""
 
-    def __init__(self, pab, w, device, fused=False, window=(), draft=(), mse="fused"):
+    def __init__(self, pab, w, device, fused=False, window=(), draft=()):
         self.pab, self.w, self.dev, self.fused = pab, w, device, fused
         self.plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges,
                              dtype=torch.bfloat16)
@@ -282,9 +281,6 @@ class AttentionStack:
         self.tout = [torch.empty((T, N, C), dtype=torch.bfloat16, device=device) for _ in range(2)]
         self.tslot = 0
         self.mse = torch.zeros((3, w.steps), dtype=torch.float64, device=device)
-        self.mse_mode = mse
-        if mse == "fused":
-            self.plan.set_diff_mse(self.mse)
         self.last_ptr = {}
         self.sched = {k: [self.plan.is_compute(k, i) for i in range(w.steps)] for k in synth.KINDS}
         self.launches_per_run = self._count_launches()
@@ -296,7 +292,7 @@ class AttentionStack:
             for k in synth.KINDS:
                 if self.sched[k][i]:
                     n += 1 if (k != "temporal" or self.fused) else 5  # 3 layouts + attention + layout back
-                    if not first[k] and self.mse_mode == "separate":
+                    if not first[k]:
                         n += 1  # MSE: one launch
                     first[k] = False
         return n
@@ -348,7 +344,7 @@ class AttentionStack:
                     self.last_ptr[k] = ptr
                     shape = (T, N, C) if k == "spatial" else (T * N, C)
                     cur = pab._wrap(ptr, shape, torch.bfloat16, self.dev)
-                if k in prev and self.mse_mode == "separate":
+                if k in prev:
                     timed("mse", lambda: pab.attn_diff_mse_async(cur, prev[k], self.mse[ki, i:i + 1],
                                                                 stream=stream))
                 prev[k] = cur
@@ -479,8 +475,8 @@ def run_ours(args):
     n_sets = max(1, min(w.steps, args.input_sets))
     inputs = make_inputs(w, device, n_sets, seed=rank)
     # the headline stack: temporal attention reads and writes the spatial view
-    # (each position's frames gathered with TMA), the attention-difference MSE
-    # accumulated inside the attention kernels
+    # (each position's frames gathered with TMA); one MSE launch per compute
+    # after a kind's first
     stack = AttentionStack(pab, w, device, fused=True)
     stream = torch.cuda.current_stream(device)
 
@@ -520,9 +516,6 @@ def run_ours(args):
             continue
         fl = flops.get(name, 0.0) if name != "layout" and name != "mse" else 0.0
         by = abytes[name]
-        if name in synth.KINDS and stack.mse_mode == "fused":
-            # every compute but a kind's first also reads the previous output once (in-kernel MSE)
-            by += (counts[name] - 1) / counts[name] * w.T * w.N * w.C * 2
         ent = {"ms": t, "launches_per_run": len(events[name][0]) // args.steps,
                "gbs": by / (t * 1e-3) / 1e9, "frac_hbm": by / (t * 1e-3) / 1e9 / hbm_peak,
                "bytes_per_launch": by}
@@ -549,7 +542,7 @@ def run_ours(args):
                        parallelism=f"replicas x{world} (one video per GPU)",
                        temporal_view="spatial view: the temporal kernel gathers each position's frames with "
                                      "TMA (the stack with explicit layout launches is reported beside)",
-                       mse="attention-difference MSE of every compute accumulated inside the attention kernels"),
+                       mse="attention-difference MSE of every compute after a kind's first, one launch each"),
         "denoising_steps_per_s": world * w.steps / (ms * 1e-3),
         "executed_tflops": world * exec_flops / (ms * 1e-3) / 1e12,
         "computes": counts,

@@ -359,14 +359,11 @@ int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep);
  * kind's first compute of the run also writes
  *   results_dev[kind * steps + step] = mean over T*N*C of (out - prev)^2,
  * prev being the kind's previous computed output (the plan's other slot).
- * For PAB_BF16 plans the kind's attention kernel accumulates it in its
- * epilogue while the new output tile is on chip, so each previous-output
- * element is read once and no extra kernel runs; per thread the squared
- * differences of each 8-element vector are summed in fp32 and added in fp64,
- * CTAs reduce in a fixed order and the last CTA adds the per-CTA sums in CTA
- * order (bitwise reproducible for a given device).  PAB_FP32 plans run the
- * MSE kernel after the compute.  Nothing is written for broadcast steps (the
- * output is the source step's, bit for bit) or for a kind's first compute.
+ * The MSE kernel (the reduction of pab_attn_diff_mse_async) runs on the
+ * same stream right after the kind's attention kernel, so the value is
+ * ready when the output is, with no host synchronisation.  Nothing is
+ * written for broadcast steps (the output is the source step's, bit for
+ * bit) or for a kind's first compute.
  * NULL disables.  The first call with a non-NULL array allocates the plan's
  * reduction scratch on the current device (the plan's device). */
 int pab_plan_set_diff_mse(pab_plan* plan, double* results_dev);

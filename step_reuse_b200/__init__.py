@@ -452,8 +452,8 @@ class Plan:
     def set_diff_mse(self, results=None):
         """results: a float64 CUDA tensor of 3 * steps elements ([3, steps]);
         every compute after a kind's first writes MSE(out, previous compute)
-        at [kind, step] (computed inside the attention kernels for bf16
-        plans).  None disables."""
+        at [kind, step] (the MSE kernel runs on the attention's stream right
+        after it).  None disables."""
         if results is not None:
             if results.dtype != torch.float64 or results.numel() != 3 * self.steps or not results.is_contiguous():
                 raise ValueError(f"need a contiguous float64 tensor of 3 * {self.steps} elements")

@@ -7,8 +7,6 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "kernels.h"
-
 #define PAB_DEV __device__ __forceinline__
 
 namespace pab {
@@ -169,55 +167,6 @@ PAB_DEV float quad_sum(float x) {
     x += __shfl_xor_sync(0xffffffffu, x, 1);
     x += __shfl_xor_sync(0xffffffffu, x, 2);
     return x;
-}
-
-}  // namespace pab
-
-namespace pab {
-
-// ---------------------------------------------------------------- fused MSE
-// The attention-difference diagnostic (mean of (out - prev)^2, PAB report,
-// Fig. 1) accumulated inside an attention kernel's epilogue, where the new
-// output is already in registers or shared memory: each element of the
-// previous output is read once and no separate launch runs.  Each thread
-// sums in a fixed order, each CTA reduces its threads in a fixed order, and
-// the CTA that takes the last completion ticket adds the per-CTA partials in
-// CTA order -- the result is bitwise reproducible for a given launch shape.
-// Sum of squared differences of 8 bf16 values (one 16-byte vector each):
-// differences and squares in fp32 (differences of bf16 values are exact
-// unless the exponents differ by more than 16), the vector's sum in fp32.
-PAB_DEV float sq_diff_bf16x8(const uint4& a, const uint4& b) {
-    const uint32_t* pa = reinterpret_cast<const uint32_t*>(&a);
-    const uint32_t* pb = reinterpret_cast<const uint32_t*>(&b);
-    float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float d0 = __uint_as_float(pa[i] << 16) - __uint_as_float(pb[i] << 16);
-        const float d1 = __uint_as_float(pa[i] & 0xffff0000u) - __uint_as_float(pb[i] & 0xffff0000u);
-        acc0 = fmaf(d0, d0, acc0);
-        acc1 = fmaf(d1, d1, acc1);
-    }
-    return acc0 + acc1;
-}
-
-PAB_DEV double warp_sum_f64(double x) {
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    return x;
-}
-
-// Called by ONE thread per CTA with the CTA's total: publishes it, and the
-// CTA that finishes last sums every CTA's partial in CTA order.
-PAB_DEV void fused_mse_finish(const FusedMse& m, double cta_total) {
-    m.partials[blockIdx.x] = cta_total;
-    __threadfence();  // the partial is visible before the ticket is taken
-    if (atomicAdd(m.ticket, 1ull) == (unsigned long long)gridDim.x - 1) {
-        __threadfence();
-        double s = 0.0;
-        for (unsigned int i = 0; i < gridDim.x; ++i) s += __ldcg(m.partials + i);
-        *m.result = m.n > 0 ? s / m.n : 0.0;
-        *m.ticket = 0ull;
-    }
 }
 
 }  // namespace pab

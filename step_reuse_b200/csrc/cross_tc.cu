@@ -60,9 +60,6 @@ struct CrossArgs {
     int nqt;           // query tiles per head
     long long tiles;   // heads * nqt
     float scale_log2;  // log2(e) / sqrt(d)
-    long long R;       // query rows
-    int C;             // heads * d
-    FusedMse mse;      // attention-difference MSE against the previous output (off when mse.prev is null)
 };
 
 constexpr int kQBufs = 3;
@@ -118,9 +115,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ double mse_warp[4];
-    double mse_acc = 0.0;  // epilogue threads: squared differences to the previous output
-    const __nv_bfloat16* mse_prev = static_cast<const __nv_bfloat16*>(a.mse.prev);
     // this CTA's contiguous run of work items
     // (work-item indices fit 32 bits: heads * query tiles < 2^31, checked on the host)
     const int tiles = (int)a.tiles;
@@ -380,28 +374,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < n; ++i) {
             const int x = i & 1;
             const uint32_t o_col = 256 + x * 128;
-            unsigned char* stage = gen_base + (o_s - sbase) + x * kTile;
-            // the staging unit of 8 output columns starting at col (128-byte swizzle)
-            auto unit_ptr = [&](int col) -> unsigned char* {
-                const int ch = (col & 63) >> 3;
-                return stage + (col >> 6) * kBox + row * 128 + ((ch ^ (row & 7)) << 4);
-            };
-            // the slot's staging buffer: the store of tile i-2 must have read it
-            if (row == 0) bulk_wait_read<1>();
-            tc::named_bar_sync(1, 128);
-            // Fused MSE: this row of the previous output is copied (cp.async, no
-            // registers held) into the staging units its new values will take,
-            // while the tile's O is still being computed; each thread reads back
-            // only the units it copied.  d % 8 == 0.
-            const int t = t_begin + i;
-            const int h = t / a.nqt, qt = t - h * a.nqt;
-            const long long qr = (long long)qt * kBM + row;
-            const bool row_in = mse_prev && qr < a.R;
-            if (row_in) {
-                const __nv_bfloat16* prow = mse_prev + qr * a.C + (long long)h * a.d;
-                for (int col = 0; col < a.d; col += 8) cp_async16(smem_u32(unit_ptr(col)), prow + col, 16);
-                cp_async_commit();
-            }
             if (ok) ok = wait_bar(&bars, &bars.o_full[x], (i >> 1) & 1);
             uint32_t ov[NC][16];
             float inv = 0.f;
@@ -416,8 +388,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(smem_u32(&bars.o_free[x]));  // O_X has been read out
                 inv = 1.f / __uint_as_float(lbits);
             }
-            if (row_in) cp_async_wait<0>();
+            // the slot's staging buffer: the store of tile i-2 must have read it
+            if (row == 0) bulk_wait_read<1>();
+            tc::named_bar_sync(1, 128);
             if (ok) {
+                unsigned char* stage = gen_base + (o_s - sbase) + x * kTile;
 #pragma unroll
                 for (int c = 0; c < NC; ++c) {
                     uint32_t w[8];
@@ -426,38 +401,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                         w[e] = pack_bf16x2(__uint_as_float(ov[c][2 * e]) * inv,
                                            __uint_as_float(ov[c][2 * e + 1]) * inv);
                     const int col = c * 16;
-                    uint4* u0 = reinterpret_cast<uint4*>(unit_ptr(col));
-                    uint4* u1 = reinterpret_cast<uint4*>(unit_ptr(col + 8));
-                    const uint4 n0 = make_uint4(w[0], w[1], w[2], w[3]), n1 = make_uint4(w[4], w[5], w[6], w[7]);
-                    if (row_in) {
-                        if (col < a.d) mse_acc += (double)sq_diff_bf16x8(n0, *u0);
-                        if (col + 8 < a.d) mse_acc += (double)sq_diff_bf16x8(n1, *u1);
-                    }
-                    *u0 = n0;
-                    *u1 = n1;
+                    const int bx = col >> 6;
+                    const int ch = (col & 63) >> 3;
+                    unsigned char* rowp = stage + bx * kBox + row * 128;
+                    *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
+                        make_uint4(w[4], w[5], w[6], w[7]);
                 }
                 fence_proxy_async_smem();
             }
             tc::named_bar_sync(1, 128);
             if (ok && row == 0) {
+                const int t = t_begin + i;
+                const int h = t / a.nqt, qt = t - h * a.nqt;
                 for (int bx = 0; bx < NB; ++bx)
                     tc::tma_store_4d(&tm_o, o_s + x * kTile + bx * kBox, bx * 64, h, qt * kBM, 0);
                 bulk_commit();
             }
         }
         if (row == 0) bulk_wait<0>();
-        if (mse_prev) {
-            const double ws = warp_sum_f64(mse_acc);
-            if (lane == 0) mse_warp[warp - 8] = ws;
-        }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (mse_prev && threadIdx.x == 0) {  // the CTA's rows in warp order, then the launch's CTAs
-        double t = 0.0;
-        for (int w = 0; w < 4; ++w) t += mse_warp[w];
-        fused_mse_finish(a.mse, t);
-    }
     if (warp == 13) {
         __syncwarp();
         tc::fence_after_sync();
@@ -512,11 +477,11 @@ cudaError_t launch_ks(const CUtensorMap* m, const CrossArgs& a, cudaStream_t s) 
 }  // namespace
 
 cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,
-                         int d, cudaStream_t s, const FusedMse* mse) {
+                         int d, cudaStream_t s) {
     if (R == 0) return cudaSuccess;
     // longer texts, and head dims whose P Vt product leaves no columns for the
     // row sums and the maxima exchange, take the general flash kernel
-    if (Lk > kBN || d > 96) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s, mse);
+    if (Lk > kBN || d > 96) return launch_flash(q, kt, vt, out, 1, R, Lk, heads, d, 0, 0, s);
     CrossArgs a;
     a.Lk = Lk;
     a.d = d;
@@ -525,9 +490,6 @@ cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* ou
     a.nqt = (int)nqt;
     a.tiles = (long long)heads * a.nqt;
     a.scale_log2 = 1.4426950408889634f / sqrtf((float)d);
-    a.R = R;
-    a.C = heads * d;
-    a.mse = mse ? *mse : FusedMse{nullptr, nullptr, nullptr, nullptr, 0.0};
     CUtensorMap m[4];
     if (!make_map(&m[0], q, d, heads, R) || !make_map(&m[1], kt, d, heads, Lk) ||
         !make_map(&m[2], vt, d, heads, Lk) || !make_map(&m[3], out, d, heads, R))

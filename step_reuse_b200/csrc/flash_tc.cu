@@ -93,9 +93,6 @@ constexpr int kPolyPairsOf8 = PAB_POLY_PAIRS_OF_8;
 #ifndef PAB_FLASH_ONES
 #define PAB_FLASH_ONES 1
 #endif
-#ifndef PAB_FLASH_HALVES
-#define PAB_FLASH_HALVES 0
-#endif
 
 __device__ unsigned int g_flash_err = 0;
 
@@ -115,12 +112,6 @@ struct FlashTcArgs {
     int tiles_h, tiles_w, reach_h, reach_w;
     const int* kv_list;
     int kv_count;
-    // fused attention-difference MSE against the previous output (off when
-    // mse.prev is null): output element (b, row, h, col) is at
-    // b * q_bstride + row * C + h * d + col; W is the frame width (tiles)
-    FusedMse mse;
-    long long q_bstride;
-    int C, W;
 };
 
 // Key geometries of the flash kernel: every key of the (frame, head) row
@@ -300,7 +291,6 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
     constexpr int NO = KSTEPS * 16;          // N of the PV product (d rounded up to 16)
     constexpr int NC = NO / 16;              // 16-column chunks of O
     constexpr bool TILED = GEO != kGeoFull;
-    constexpr bool HALVES = PAB_FLASH_HALVES && SPLIT == 1;  // the softmax step in two pipelined halves
 
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     __shared__ Bars bars;
@@ -315,9 +305,6 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
     float* xsum = xmax + 2 * 2 * 2 * 128;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    __shared__ double mse_warp[NSW];
-    double mse_acc = 0.0;  // softmax threads: this row's squared differences to the previous output
-    const __nv_bfloat16* mse_prev = static_cast<const __nv_bfloat16*>(a.mse.prev);
 
     if (threadIdx.x == W_PROD * 32) {
         for (int x = 0; x < 2; ++x) {
@@ -600,125 +587,6 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                     tc::fence_after_sync();
                     const uint32_t s_col = x * 128 + (g & 1) * 64;
                     const int valid = TILED ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
-                  if constexpr (HALVES) {
-                    // Two 32-key halves, software-pipelined: the second half's
-                    // TMEM load is in flight while the first half is
-                    // exponentiated.  The lazy-rescale test uses the first
-                    // half's maximum; if the second half then exceeds the
-                    // reference by more than 2^8, the first half's P (already in
-                    // TMEM) and O are rescaled (rare).
-                    const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
-                    float acc_l = 0.f;
-                    auto exp_half = [&](const float (&sv)[32], int half) {
-                        const tc::f32x2 negm2 = tc::pack2(-m_ref, -m_ref);
-                        tc::f32x2 acc[2] = {tc::pack2(0.f, 0.f), tc::pack2(0.f, 0.f)};
-                        uint32_t r[16];
-#pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const tc::f32x2 t = tc::fma2(tc::pack2(sv[2 * i], sv[2 * i + 1]), scale2, negm2);
-                            float t0, t1, p0, p1;
-                            tc::unpack2(t, t0, t1);
-                            if ((i & 7) < kPolyPairsOf8) {
-                                tc::exp2_poly2(t0, t1, p0, p1);
-                            } else {
-                                p0 = ex2(t0);
-                                p1 = ex2(t1);
-                            }
-                            if constexpr (!ONES) acc[i & 1] = tc::add2(acc[i & 1], tc::pack2(p0, p1));
-                            r[i] = pack_bf16x2(p0, p1);
-                        }
-                        tc::st_16col(lane_addr + s_col + half * 16, r);
-                        if constexpr (!ONES) {
-                            float a0, a1;
-                            tc::unpack2(tc::add2(acc[0], acc[1]), a0, a1);
-                            acc_l += a0 + a1;
-                        }
-                    };
-                    auto row_max = [&](float (&sv)[32], int k0) {
-                        if (k0 + 32 > valid) {
-#pragma unroll
-                            for (int i = 0; i < 32; ++i)
-                                if (k0 + i >= valid) sv[i] = -INFINITY;
-                        }
-                        float mx[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) mx[q] = fmaxf(tc::max3f(sv[q], sv[q + 8], sv[q + 16]), sv[q + 24]);
-                        return tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
-                                         fmaxf(mx[6], mx[7])) * a.scale_log2;
-                    };
-                    // O_X must hold exactly PV_X(..g-1) before it is rescaled
-                    auto rescale_o = [&](float f) -> bool {
-                        if (j == 0) return true;  // this item's O is not accumulated yet
-                        if (!wait_bar(&bars, &bars.slot_done[(g + 1) % NST][x], ((g + 1) / NST) & 1)) return false;
-                        tc::fence_after_sync();
-                        for (int cc = 0; cc < NO / 16; ++cc) {
-                            uint32_t r[16];
-                            tc::ld_16col(lane_addr + o_col + cc * 16, r);
-                            tc::wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
-                            tc::st_16col(lane_addr + o_col + cc * 16, r);
-                        }
-                        return true;
-                    };
-                    float sa[32];
-                    {
-                        uint32_t r0[32];
-                        tc::ld_32col(lane_addr + s_col, r0);
-                        tc::wait_ld();
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sa[i] = __uint_as_float(r0[i]);
-                    }
-                    uint32_t r1[32];
-                    tc::ld_32col(lane_addr + s_col + 32, r1);  // waited for after the first half
-                    const float mt0 = row_max(sa, 0);
-                    if (j == 0) {
-                        m_ref = mt0;
-                        if (g == 0 && x == 0) mbar_arrive(smem_u32(&bars.b_go));
-                    } else {
-                        const bool need = mt0 > m_ref + kRescaleLog2;
-                        if (__any_sync(0xffffffffu, need)) {
-                            const float m_new = need ? mt0 : m_ref;
-                            const float f = ex2(m_ref - m_new);
-                            ok = rescale_o(f);
-                            if constexpr (!ONES) l *= f;
-                            m_ref = m_new;
-                        }
-                    }
-                    if (ok) exp_half(sa, 0);
-                    tc::wait_ld();
-                    if (!ok) break;
-                    float sb[32];
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) sb[i] = __uint_as_float(r1[i]);
-                    const float mt1 = row_max(sb, 32);
-                    {
-                        const bool need = mt1 > m_ref + kRescaleLog2;
-                        if (__any_sync(0xffffffffu, need)) {  // rare: rescale O and the first half's P
-                            const float m_new = need ? mt1 : m_ref;
-                            const float f = ex2(m_ref - m_new);
-                            if (!rescale_o(f)) {
-                                ok = false;
-                                break;
-                            }
-                            tc::wait_st();
-                            uint32_t r[16];
-                            tc::ld_16col(lane_addr + s_col, r);
-                            tc::wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                r[i] = pack_bf16x2(__uint_as_float(r[i] << 16) * f, __uint_as_float(r[i] & 0xffff0000u) * f);
-                            tc::st_16col(lane_addr + s_col, r);
-                            if constexpr (!ONES) {
-                                l *= f;
-                                acc_l *= f;
-                            }
-                            m_ref = m_new;
-                        }
-                    }
-                    exp_half(sb, 1);
-                    if constexpr (!ONES) l += acc_l;
-                  } else {
                     // this warp's scores of the row: one TMEM read each 32 keys
                     float sv[KC];
                     {
@@ -834,7 +702,6 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                         tc::unpack2(tc::add2(tc::add2(acc[0], acc[1]), tc::add2(acc[2], acc[3])), a0, a1);
                         l += a0 + a1;
                     }
-                  }
                     tc::wait_st();
                 }
                 tc::fence_before_sync();
@@ -847,48 +714,10 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
             }
             if (!ok) break;
             // ---------------- epilogue: O / l -> bf16 -> swizzled smem -> TMA store
+            ok = wait_bar(&bars, &bars.o_done[x], k & 1);
+            if (!ok) break;
             // the item's Q buffer: every S of this item has retired
             unsigned char* stage = gen_base + ((k & 1) * 2 + x) * DL::QTile;
-            // the staging address of 16-byte unit u (8 columns) of chunk cc of this row
-            auto unit_ptr = [&](int cc, int u) -> unsigned char* {
-                const int col = cc * 16;
-                if (col < DL::NB0 * 64) {
-                    const int ch = (col & 63) >> 3;
-                    return stage + (col >> 6) * kQBox + row * 128 + (((ch + u) ^ (row & 7)) << 4);
-                }
-                const int tu = (col - DL::NB0 * 64) >> 3;
-                return stage + DL::NB0 * kQBox + row * DL::TB + (DL::tail_unit(row, tu + u) << 4);
-            };
-            // Fused MSE: this row of the previous output is copied (cp.async, no
-            // registers held) into the staging units its new values will take,
-            // during the wait for the item's last PV; each thread later reads
-            // back only the units it copied.  d % 8 == 0: each 8-column unit lies
-            // wholly inside or past d.
-            bool row_in = false;
-            if (mse_prev && work) {
-                long long row_off;
-                if constexpr (TILED) {
-                    const int tok = (m.ty * 16 + x * 8 + (row >> 4)) * a.W + m.tx * 16 + (row & 15);
-                    row_off = m.b * a.q_bstride + (long long)tok * a.C + m.h * a.d;
-                    row_in = true;
-                } else {
-                    const int qr = (m.qblk * 2 + x) * kBM + row;
-                    row_off = m.b * a.q_bstride + (long long)qr * a.C + m.h * a.d;
-                    row_in = qr < a.Lq;
-                }
-                if (row_in) {
-                    const __nv_bfloat16* prow = mse_prev + row_off;
-                    for (int cc = c_lo; cc < c_hi; ++cc)
-                        for (int u = 0; u < 2; ++u)
-                            if (cc * 16 + u * 8 < a.d) cp_async16(smem_u32(unit_ptr(cc, u)), prow + cc * 16 + u * 8, 16);
-                    cp_async_commit();
-                }
-            }
-            ok = wait_bar(&bars, &bars.o_done[x], k & 1);
-            if (!ok) {
-                cp_async_wait<0>();  // no copy lands in shared memory after the CTA exits
-                break;
-            }
             if (work) {
                 tc::fence_after_sync();
                 if constexpr (ONES) {  // O's column d: the row sum of P
@@ -905,7 +734,6 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                     l = xs[row] + xs[128 + row];
                 }
                 const float inv = 1.f / l;
-                if (row_in) cp_async_wait<0>();
                 for (int cc = c_lo; cc < c_hi; ++cc) {
                     uint32_t r[16];
                     tc::ld_16col(lane_addr + o_col + cc * 16, r);
@@ -914,15 +742,22 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
 #pragma unroll
                     for (int i = 0; i < 8; ++i)
                         w[i] = pack_bf16x2(__uint_as_float(r[2 * i]) * inv, __uint_as_float(r[2 * i + 1]) * inv);
-                    uint4* u0 = reinterpret_cast<uint4*>(unit_ptr(cc, 0));
-                    uint4* u1 = reinterpret_cast<uint4*>(unit_ptr(cc, 1));
-                    const uint4 n0 = make_uint4(w[0], w[1], w[2], w[3]), n1 = make_uint4(w[4], w[5], w[6], w[7]);
-                    if (row_in) {
-                        if (cc * 16 < a.d) mse_acc += (double)sq_diff_bf16x8(n0, *u0);
-                        if (cc * 16 + 8 < a.d) mse_acc += (double)sq_diff_bf16x8(n1, *u1);
+                    const int col = cc * 16;
+                    if (col < DL::NB0 * 64) {
+                        const int bx = col >> 6;
+                        const int ch = (col & 63) >> 3;
+                        unsigned char* rowp = stage + bx * kQBox + row * 128;
+                        *reinterpret_cast<uint4*>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(rowp + (((ch + 1) ^ (row & 7)) << 4)) =
+                            make_uint4(w[4], w[5], w[6], w[7]);
+                    } else {  // tail box
+                        const int u = (col - DL::NB0 * 64) >> 3;
+                        unsigned char* rowp = stage + DL::NB0 * kQBox + row * DL::TB;
+                        *reinterpret_cast<uint4*>(rowp + (DL::tail_unit(row, u) << 4)) =
+                            make_uint4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<uint4*>(rowp + (DL::tail_unit(row, u + 1) << 4)) =
+                            make_uint4(w[4], w[5], w[6], w[7]);
                     }
-                    *u0 = n0;
-                    *u1 = n1;
                 }
                 fence_proxy_async_smem();
             }
@@ -956,18 +791,9 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
         }
         // shared memory stays valid until every output store has read it
         if (hf == 0 && row == 0) bulk_wait_read<0>();
-        if (mse_prev) {
-            const double ws = warp_sum_f64(mse_acc);
-            if (lane == 0) mse_warp[warp] = ws;
-        }
     }
     tc::fence_before_sync();
     __syncthreads();
-    if (mse_prev && threadIdx.x == 0) {  // the CTA's rows in warp order, then the launch's CTAs
-        double t = 0.0;
-        for (int w = 0; w < NSW; ++w) t += mse_warp[w];
-        fused_mse_finish(a.mse, t);
-    }
     if (warp == W_MMA) {
         __syncwarp();
         tc::fence_after_sync();
@@ -1090,13 +916,6 @@ cudaError_t launch_d(const FlashMaps& m, const FlashTcArgs& a, cudaStream_t s) {
     }
 }
 
-void set_mse(FlashTcArgs* a, const FusedMse* mse, long long q_bstride, int C, int W) {
-    a->mse = mse ? *mse : FusedMse{nullptr, nullptr, nullptr, nullptr, 0.0};
-    a->q_bstride = q_bstride;
-    a->C = C;
-    a->W = W;
-}
-
 // Width in columns of the tail box for head dim d (0: none)
 int tail_cols(int d) {
     const int ks = (d + 15) / 16, tk = ks % 4;
@@ -1125,8 +944,7 @@ bool make_grid_maps(FlashMaps* m, const void* q, const void* k, const void* v, v
 }  // namespace
 
 cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches, long long Lq,
-                         int Lk, int heads, int d, long long q_bstride, long long kv_bstride, cudaStream_t s,
-                         const FusedMse* mse) {
+                         int Lk, int heads, int d, long long q_bstride, long long kv_bstride, cudaStream_t s) {
     if (Lq == 0 || batches == 0) return cudaSuccess;
     if (Lk < 1 || heads < 1 || batches < 0) return cudaErrorInvalidValue;
     const long long C = (long long)heads * d;
@@ -1159,7 +977,6 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
     a.heads = heads;
     a.per_bh = (int)qblocks;
     a.items = (int)(qblocks * heads * batches);
-    set_mse(&a, mse, q_bstride > 0 ? q_bstride : Lq * C, (int)C, 0);
     a.tiles_h = a.tiles_w = a.reach_h = a.reach_w = 0;
     a.kv_list = nullptr;
     a.kv_count = 0;
@@ -1167,7 +984,7 @@ cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out,
 }
 
 cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
-                             int heads, int d, int win_h, int win_w, cudaStream_t s, const FusedMse* mse) {
+                             int heads, int d, int win_h, int win_w, cudaStream_t s) {
     if (frames == 0 || H == 0 || W == 0) return cudaSuccess;
     if (H % kStaTile || W % kStaTile || win_h % kStaTile || win_w % kStaTile || win_h <= 0 || win_w <= 0 ||
         (win_h / kStaTile) % 2 == 0 || (win_w / kStaTile) % 2 == 0)
@@ -1191,13 +1008,11 @@ cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* 
     a.heads = heads;
     a.per_bh = (int)tiles;
     a.items = (int)(tiles * heads * frames);
-    set_mse(&a, mse, (long long)H * W * heads * d, heads * d, W);
     return launch_d<kGeoWindow>(m, a, s);
 }
 
 cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
-                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s,
-                                   const FusedMse* mse) {
+                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s) {
     if (frames == 0 || H == 0 || W == 0) return cudaSuccess;
     if (H % kStaTile || W % kStaTile || kv_count < 1 || !kv_list) return cudaErrorInvalidValue;
     const long long tiles = (long long)(H / kStaTile) * (W / kStaTile);
@@ -1218,7 +1033,6 @@ cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, 
     a.heads = heads;
     a.per_bh = (int)tiles;
     a.items = (int)(tiles * heads * frames);
-    set_mse(&a, mse, (long long)H * W * heads * d, heads * d, W);
     return launch_d<kGeoList>(m, a, s);
 }
 

@@ -8,19 +8,6 @@
 
 namespace pab {
 
-// The attention-difference MSE (mean of (out - prev)^2 over n elements)
-// fused into an attention launch's epilogue; prev == nullptr: off.  The
-// scratch (one double per CTA plus the completion ticket, zero before the
-// launch and returned to zero by it) is the caller's.
-struct FusedMse {
-    const void* prev;            // the previous output (bf16), same layout as the launch's output
-    double* partials;            // one per CTA of the launch
-    unsigned long long* ticket;  // completion ticket
-    double* result;              // device scalar: the mean
-    double n;                    // elements compared
-};
-constexpr int kFusedMseMaxCtas = 4096;  // partials a fused-MSE scratch holds
-
 // Streaming multiprocessors of the current device (cached per device).
 int device_sm_count();
 
@@ -58,7 +45,7 @@ cudaError_t launch_scatter_blocks(const void* const* src, void* const* dst, int 
 // --- temporal short-sequence attention ([N,T,C], L = T) -------------------
 // spatial_view = 1: q, k, v, out are [T, N, C] instead of [N, T, C]
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
-                            int heads, int d, int spatial_view, cudaStream_t s, const FusedMse* mse = nullptr);
+                            int heads, int d, int spatial_view, cudaStream_t s);
 unsigned int temporal_device_errors(bool clear);
 
 // --- flash attention for spatial (per frame) and cross (shared text K/V) --
@@ -66,22 +53,20 @@ unsigned int temporal_device_errors(bool clear);
 // k/v with kv_bstride (0 = shared K/V).  out has q's layout.
 cudaError_t launch_flash(const void* q, const void* k, const void* v, void* out, int batches,
                          long long Lq, int Lk, int heads, int d, long long q_bstride,
-                         long long kv_bstride, cudaStream_t s, const FusedMse* mse = nullptr);
+                         long long kv_bstride, cudaStream_t s);
 // Sliding tile attention within each frame of a [frames][H*W][heads*d] bf16
 // spatial view: 16 x 16-token tiles, a window of win_h x win_w tokens (odd
 // tile counts) centred on the query's tile and clipped at the frame edge.
 // H, W, win_h, win_w must be multiples of 16 (cudaErrorInvalidValue else).
 cudaError_t launch_flash_sta(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
-                             int heads, int d, int win_h, int win_w, cudaStream_t s,
-                             const FusedMse* mse = nullptr);
+                             int heads, int d, int win_h, int win_w, cudaStream_t s);
 
 // Attention of every 16 x 16 query tile of each frame over the 16 x 16 key
 // tiles kv_list names for it: [frames][heads][tiles][kv_count] tile indices
 // (ty * (W/16) + tx) of the same frame.  An index outside the frame raises
 // kDevErrBadIndex in the flash status word and is clamped.
 cudaError_t launch_flash_tile_list(const void* q, const void* k, const void* v, void* out, int frames, int H, int W,
-                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s,
-                                   const FusedMse* mse = nullptr);
+                                   int heads, int d, const int* kv_list, int kv_count, cudaStream_t s);
 
 unsigned int flash_device_errors(bool clear);
 
@@ -95,7 +80,7 @@ cudaError_t launch_draft_select(const void* q, const void* k, int T, int H, int 
 
 // --- cross attention (text_len <= 128: persistent cross_tc; longer: flash) --
 cudaError_t launch_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lk, int heads,
-                         int d, cudaStream_t s, const FusedMse* mse = nullptr);
+                         int d, cudaStream_t s);
 unsigned int cross_device_errors(bool clear);
 
 // --- dense parts of a DiT block around the attention kinds ----------------

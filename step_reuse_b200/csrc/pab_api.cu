@@ -101,10 +101,10 @@ int check_ptrs(const char* names, const void* a, const void* b, const void* c, c
 }
 
 int run_spatial(const void* q, const void* k, const void* v, void* out, int T, int N, int heads,
-                int d, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
+                int d, cudaStream_t s) {
     const long long C = (long long)heads * d;
     cudaError_t e = pab::launch_flash(q, k, v, out, T, N, N, heads, d, (long long)N * C,
-                                      (long long)N * C, s, mse);
+                                      (long long)N * C, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "spatial attention launch");
 }
 
@@ -119,8 +119,8 @@ int check_sta(int H, int W, int tile, int win_h, int win_w) {
 }
 
 int run_sta(const void* q, const void* k, const void* v, void* out, int T, int H, int W, int heads, int d,
-            int win_h, int win_w, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
-    cudaError_t e = pab::launch_flash_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, s, mse);
+            int win_h, int win_w, cudaStream_t s) {
+    cudaError_t e = pab::launch_flash_sta(q, k, v, out, T, H, W, heads, d, win_h, win_w, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "sliding tile attention launch");
 }
 
@@ -134,22 +134,22 @@ int check_draft(int H, int W, int region, int keep) {
 }
 
 int run_draft(const void* q, const void* k, const void* v, void* out, int T, int H, int W, int heads, int d,
-              int keep, int* sel, void* sketch, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
+              int keep, int* sel, void* sketch, cudaStream_t s) {
     cudaError_t e = pab::launch_draft_select(q, k, T, H, W, heads, d, keep, sel, sketch, s);
     if (e != cudaSuccess) return cuda_fail(e, "draft selection launch");
-    e = pab::launch_flash_tile_list(q, k, v, out, T, H, W, heads, d, sel, keep, s, mse);
+    e = pab::launch_flash_tile_list(q, k, v, out, T, H, W, heads, d, sel, keep, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "region-sparse attention launch");
 }
 
 int run_temporal(const void* q, const void* k, const void* v, void* out, int N, int T, int heads,
-                 int d, int spatial_view, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
-    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s, mse);
+                 int d, int spatial_view, cudaStream_t s) {
+    cudaError_t e = pab::launch_temporal(q, k, v, out, N, T, heads, d, spatial_view, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "temporal attention launch");
 }
 
 int run_cross(const void* q, const void* kt, const void* vt, void* out, long long R, int Lt,
-              int heads, int d, cudaStream_t s, const pab::FusedMse* mse = nullptr) {
-    cudaError_t e = pab::launch_cross(q, kt, vt, out, R, Lt, heads, d, s, mse);
+              int heads, int d, cudaStream_t s) {
+    cudaError_t e = pab::launch_cross(q, kt, vt, out, R, Lt, heads, d, s);
     return e == cudaSuccess ? PAB_OK : cuda_fail(e, "cross attention launch");
 }
 
@@ -296,32 +296,30 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
         vv = p->stage_in[2];
         oo = p->stage_out;
     }
-    // bf16 plans: the kind's kernel accumulates the difference to the previous
-    // output in its epilogue; fp32 plans: the MSE kernel runs after the compute
-    pab::FusedMse fm{prev, p->mse_scratch + 1, reinterpret_cast<unsigned long long*>(p->mse_scratch),
-                     mse_result, (double)qn};
-    const pab::FusedMse* mse = (prev && p->dtype == PAB_BF16) ? &fm : nullptr;
     int rc;
     if (kind == PAB_SPATIAL && p->draft_keep > 0)
         rc = run_draft(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->draft_keep, p->draft_sel,
-                       p->draft_sketch, s, mse);
+                       p->draft_sketch, s);
     else if (kind == PAB_SPATIAL && p->sta_win_h > 0)
-        rc = run_sta(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->sta_win_h, p->sta_win_w, s, mse);
+        rc = run_sta(qq, kk, vv, oo, p->T, p->H, p->W, p->heads, p->d, p->sta_win_h, p->sta_win_w, s);
     else if (kind == PAB_SPATIAL)
-        rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s, mse);
+        rc = run_spatial(qq, kk, vv, oo, p->T, p->N, p->heads, p->d, s);
     else if (kind == PAB_TEMPORAL)
-        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, p->temporal_sv, s, mse);
+        rc = run_temporal(qq, kk, vv, oo, p->N, p->T, p->heads, p->d, p->temporal_sv, s);
     else
-        rc = run_cross(qq, kk, vv, oo, (long long)p->T * p->N, p->text_len, p->heads, p->d, s, mse);
+        rc = run_cross(qq, kk, vv, oo, (long long)p->T * p->N, p->text_len, p->heads, p->d, s);
     if (rc) return rc;
     if (p->dtype == PAB_FP32) {
         cudaError_t e = pab::launch_bf16_to_f32(p->stage_out, static_cast<float*>(out), qn, s);
         if (e != cudaSuccess) return cuda_fail(e, "bf16 -> fp32 conversion");
-        if (prev) {
-            const int parts = pab::mse_num_partials(qn, 4);
-            e = pab::launch_mse(out, prev, qn, PAB_FP32, p->mse_scratch, parts, mse_result, s);
-            if (e != cudaSuccess) return cuda_fail(e, "attention-difference MSE launch");
-        }
+    }
+    if (prev) {
+        // the difference to the kind's previous output, read back from HBM by
+        // the MSE kernel on the same stream
+        const int elem = p->dtype == PAB_FP32 ? 4 : 2;
+        const int parts = pab::mse_num_partials(qn, elem);
+        cudaError_t e = pab::launch_mse(out, prev, qn, p->dtype, p->mse_scratch, parts, mse_result, s);
+        if (e != cudaSuccess) return cuda_fail(e, "attention-difference MSE launch");
     }
     return PAB_OK;
 }
@@ -825,13 +823,14 @@ int pab_plan_set_diff_mse(pab_plan* plan, double* results_dev) {
     if (results_dev && (reinterpret_cast<uintptr_t>(results_dev) & 7u))
         return fail(PAB_ERR_ARG, "results_dev not 8-byte aligned");
     if (results_dev && !plan->mse_scratch) {
-        const int need = pab::kFusedMseMaxCtas + 1;
+        // the completion ticket and the most partial sums one MSE launch takes
+        const int need = pab::mse_num_partials(1LL << 40, 2) + 1;
         cudaError_t e = cudaMalloc(&plan->mse_scratch, sizeof(double) * need);
         if (e != cudaSuccess) {
             plan->mse_scratch = nullptr;
             return cuda_fail(e, "MSE scratch allocation");
         }
-        e = cudaMemset(plan->mse_scratch, 0, sizeof(unsigned long long));  // the completion ticket
+        e = cudaMemset(plan->mse_scratch, 0, sizeof(unsigned long long));  // the ticket starts at zero
         if (e != cudaSuccess) return cuda_fail(e, "MSE scratch clear");
     }
     plan->mse_results = results_dev;

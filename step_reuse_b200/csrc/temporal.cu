@@ -51,12 +51,11 @@ struct TemporalArgs {
     int RT;      // rows per head block in smem (T rounded up to 16)
     long long units;
     float scale_log2;  // log2(e) / sqrt(d)
-    FusedMse mse;      // attention-difference MSE against the previous output (off when mse.prev is null)
 };
 
 // smem layout of one stage: [3 tensors][G heads][RT rows][P cols] bf16
 template <int DN>
-__global__ void __launch_bounds__(kThreads, DN <= 9 ? 2 : 1) temporal_kernel(const __grid_constant__ CUtensorMap tm_q,
+__global__ void __launch_bounds__(kThreads) temporal_kernel(const __grid_constant__ CUtensorMap tm_q,
                                                             const __grid_constant__ CUtensorMap tm_k,
                                                             const __grid_constant__ CUtensorMap tm_v,
                                                             const __grid_constant__ CUtensorMap tm_o,
@@ -65,9 +64,6 @@ __global__ void __launch_bounds__(kThreads, DN <= 9 ? 2 : 1) temporal_kernel(con
     __shared__ __align__(8) unsigned long long full_bar[2];
     __shared__ __align__(8) unsigned long long done_bar[2];  // every compute warp finished the stage's unit
     __shared__ int abort_flag;
-    __shared__ double mse_warp[kWarps];
-    double mse_acc = 0.0;  // compute threads: squared differences to the previous output
-    const __nv_bfloat16* mse_prev = static_cast<const __nv_bfloat16*>(p.mse.prev);
     constexpr int DK = (DN + 1) / 2;  // 16-wide k chunks covering d
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = p.G, P = p.P, RT = p.RT, T = p.T;
@@ -187,31 +183,6 @@ __global__ void __launch_bounds__(kThreads, DN <= 9 ? 2 : 1) temporal_kernel(con
                 qa[DK - 1][2] = 0u;
                 qa[DK - 1][3] = 0u;
             }
-            if (mse_prev) {
-                // Fused MSE: the task's rows of the previous output (this head,
-                // frames t < T) are copied (cp.async) over the q rows, which the q
-                // fragments no longer need, and read back where the output goes.
-                // Consuming the fragments first makes their shared-memory reads
-                // complete before any copy can land.
-                uint32_t dep = 0;
-#pragma unroll
-                for (int kc = 0; kc < DK; ++kc) dep ^= qa[kc][0] ^ qa[kc][1] ^ qa[kc][2] ^ qa[kc][3];
-                asm volatile("" :: "r"(dep) : "memory");
-                __syncwarp();
-                const int un = (int)(u / hg_count);
-                const int uh = (int)(u - (long long)un * hg_count) * G + g;
-                const long long C = (long long)p.heads * p.d;
-                const int nv = p.d / 8;
-                for (int idx = lane; idx < 16 * nv; idx += 32) {
-                    const int rr = idx / nv, vc = idx - rr * nv;
-                    const int t = mt * 16 + rr;
-                    if (t < T) {
-                        const long long prow = p.spatial_view ? (long long)t * p.N + un : (long long)un * T + t;
-                        cp_async16(smem_u32(qs + rr * P + vc * 8), mse_prev + prow * C + (long long)uh * p.d + vc * 8, 16);
-                    }
-                }
-                cp_async_commit();
-            }
             float o[DN][4];
 #pragma unroll
             for (int j = 0; j < DN; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.f;
@@ -290,55 +261,20 @@ __global__ void __launch_bounds__(kThreads, DN <= 9 ? 2 : 1) temporal_kernel(con
             l0 = quad_sum(l0);
             l1 = quad_sum(l1);
             const float inv0 = 1.f / l0, inv1 = 1.f / l1;
-            // stage O (bf16) over this warp's own q rows (after reading the
-            // previous output staged at the same positions, fused MSE)
+            // stage O (bf16) over this warp's own q rows
             const int r0 = lane >> 2, cq = 2 * (lane & 3);
-            if (mse_prev) {
-                cp_async_wait<0>();
-                __syncwarp();  // every lane's copies are visible
-            }
-            const bool in0 = mse_prev && mt * 16 + r0 < T, in1 = mse_prev && mt * 16 + r0 + 8 < T;
-            float sq = 0.f;
 #pragma unroll
             for (int j = 0; j < DN; ++j) {
-                uint32_t* d0 = reinterpret_cast<uint32_t*>(qs + r0 * P + j * 8 + cq);
-                uint32_t* d1 = reinterpret_cast<uint32_t*>(qs + (r0 + 8) * P + j * 8 + cq);
-                const uint32_t n0 = pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
-                const uint32_t n1 = pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
-                if (in0) {
-                    const uint32_t pv = *d0;
-                    const float a0 = __uint_as_float(n0 << 16) - __uint_as_float(pv << 16);
-                    const float a1 = __uint_as_float(n0 & 0xffff0000u) - __uint_as_float(pv & 0xffff0000u);
-                    sq = fmaf(a0, a0, fmaf(a1, a1, sq));
-                }
-                if (in1) {
-                    const uint32_t pv = *d1;
-                    const float a0 = __uint_as_float(n1 << 16) - __uint_as_float(pv << 16);
-                    const float a1 = __uint_as_float(n1 & 0xffff0000u) - __uint_as_float(pv & 0xffff0000u);
-                    sq = fmaf(a0, a0, fmaf(a1, a1, sq));
-                }
-                *d0 = n0;
-                *d1 = n1;
+                *reinterpret_cast<uint32_t*>(qs + r0 * P + j * 8 + cq) = pack_bf16x2(o[j][0] * inv0, o[j][1] * inv0);
+                *reinterpret_cast<uint32_t*>(qs + (r0 + 8) * P + j * 8 + cq) =
+                    pack_bf16x2(o[j][2] * inv1, o[j][3] * inv1);
             }
-            if (mse_prev) mse_acc += (double)sq;
         }
             // the outputs are written over this warp's own q rows: visible to the
             // TMA store (async proxy) once the producer sees every warp's arrival
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_u32(&done_bar[stage]));
-        }
-        if (mse_prev) {
-            const double ws = warp_sum_f64(mse_acc);
-            if (lane == 0) mse_warp[warp] = ws;
-        }
-    }
-    if (mse_prev) {
-        __syncthreads();
-        if (threadIdx.x == 0) {  // the CTA's warps in order, then the launch's CTAs
-            double t = 0.0;
-            for (int w = 0; w < kWarps; ++w) t += mse_warp[w];
-            fused_mse_finish(p.mse, t);
         }
     }
 }
@@ -397,9 +333,8 @@ cudaError_t launch_dn(const CUtensorMap* maps, const TemporalArgs& p, size_t sme
 }  // namespace
 
 cudaError_t launch_temporal(const void* q, const void* k, const void* v, void* out, int N, int T,
-                            int heads, int d, int spatial_view, cudaStream_t s, const FusedMse* mse) {
+                            int heads, int d, int spatial_view, cudaStream_t s) {
     TemporalArgs p;
-    p.mse = mse ? *mse : FusedMse{nullptr, nullptr, nullptr, nullptr, 0.0};
     p.spatial_view = spatial_view;
     p.N = N;
     p.T = T;

@@ -194,8 +194,8 @@ def test_sweep_u_shape_and_counts(pab, oracle_mod):
                 assert edge_mse > 5 * mid_mse, (kind, edge_mse, mid_mse)
 
 
-def _run_fused_mse(pab, w, ranges, setup=None, seed=0):
-    """One run with the plan's in-kernel MSE on: (mse table, outputs of every compute)."""
+def _run_plan_mse(pab, w, ranges, setup=None, seed=0):
+    """One run with the plan's MSE table on: (mse table, outputs of every compute)."""
     plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, ranges, dtype=w.torch_dtype)
     if setup:
         setup(plan)
@@ -229,21 +229,19 @@ def _edge(w):
 
 
 @pytest.mark.parametrize("name,view", [("tiny", False), ("480p", False), ("480p", True), ("720p", False)])
-def test_fused_diff_mse(pab, oracle_mod, name, view):
-    """The plan's attention-difference MSE (PAB report, Fig. 1) computed inside
-    the attention kernels' epilogues (bf16 plans; the fp32 tiny plan runs the
-    MSE kernel after each compute): every compute after a kind's first writes
-    the MSE of its output against the kind's previous compute -- equal to the
-    oracle's to 1e-5 relative (checked on every pair at the tiny size, on the
-    first and last pair of each kind at the large ones, where the host oracle
-    of a pair reads two whole outputs) and to the stand-alone MSE call on
-    every pair to 1e-7 (both add fp64 sums of fp32 partial sums; the partial
-    sums group the elements differently) -- and nothing else is written; a
-    second run writes bit-identical values."""
+def test_plan_diff_mse(pab, oracle_mod, name, view):
+    """The plan's attention-difference MSE (PAB report, Fig. 1): every compute
+    after a kind's first writes the MSE of its output against the kind's
+    previous compute -- equal to the oracle's to 1e-5 relative (checked on
+    every pair at the tiny size, on the first and last pair of each kind at
+    the large ones, where the host oracle of a pair reads two whole outputs)
+    and bit-identical to the stand-alone MSE call on every pair (the same
+    reduction over the same data) -- and nothing else is written; a second
+    run writes bit-identical values."""
     w = synth.WORKLOADS[name]
     setup = (lambda p: p.set_temporal_view(True)) if view else None
-    t1, outs = _run_fused_mse(pab, w, w.ranges, setup)
-    t2, _ = _run_fused_mse(pab, w, w.ranges, setup)
+    t1, outs = _run_plan_mse(pab, w, w.ranges, setup)
+    t2, _ = _run_plan_mse(pab, w, w.ranges, setup)
     assert np.array_equal(t1, t2)  # bitwise reproducible
     for ki, kind in enumerate(synth.KINDS):
         comps = outs[kind]
@@ -251,22 +249,22 @@ def test_fused_diff_mse(pab, oracle_mod, name, view):
         assert written == {i for i, _ in comps[1:]}, (kind, written)
         for n, ((i, o), (_, prev)) in enumerate(zip(comps[1:], comps[:-1])):
             alone = pab.attn_diff_mse(o, prev)
-            assert abs(t1[ki, i] - alone) <= 1e-7 * alone, (kind, i, t1[ki, i], alone)
+            assert t1[ki, i] == alone, (kind, i, t1[ki, i], alone)
             if name == "tiny" or n in (0, len(comps) - 2):
                 want = oracle_mod.mse(to_f64(o), to_f64(prev))
                 assert abs(t1[ki, i] - want) <= MSE_REL * want, (kind, i, t1[ki, i], want)
 
 
 @pytest.mark.parametrize("mode", ["window", "draft"])
-def test_fused_diff_mse_spatial_alternatives(pab, oracle_mod, mode):
+def test_plan_diff_mse_spatial_alternatives(pab, oracle_mod, mode):
     """The same diagnostic through the sliding-tile (window) and draft-attention
     (region list) forms of the spatial kind."""
     w = synth.Workload(name="tiles", T=2, H=32, W=48, heads=2, d=64, text_len=16, steps=10, ranges=(2, 3, 4),
                        sigma=0.05, dtype="bf16")
     setup = (lambda p: p.set_spatial_window(16, 48, 48)) if mode == "window" else \
         (lambda p: p.set_spatial_draft(16, 3))
-    t1, outs = _run_fused_mse(pab, w, w.ranges, setup)
-    t2, _ = _run_fused_mse(pab, w, w.ranges, setup)
+    t1, outs = _run_plan_mse(pab, w, w.ranges, setup)
+    t2, _ = _run_plan_mse(pab, w, w.ranges, setup)
     assert np.array_equal(t1, t2)
     comps = outs["spatial"]
     assert len(comps) > 2
