@@ -368,6 +368,23 @@ int pab_plan_set_spatial_draft(pab_plan* plan, int region, int keep);
  * reduction scratch on the current device (the plan's device). */
 int pab_plan_set_diff_mse(pab_plan* plan, double* results_dev);
 
+/* Where the plan's MSE launches run (pab_plan_set_diff_mse).  enable = 1:
+ * on cuda_stream (a side stream; NULL is the legacy default stream), so the
+ * HBM-bound MSE overlaps the next attention computes: after each compute the
+ * compute stream records an event the side stream waits on before the MSE
+ * launch, and the kind's next compute -- which overwrites the slot that MSE
+ * reads -- waits on the compute stream for an event recorded behind it.  The
+ * table entries are then complete once cuda_stream has drained (synchronise
+ * it, or the device, before reading them); the values are bit-identical to
+ * the in-line ones (the same kernel and reduction).  enable = 0 (the
+ * default): in line on the compute stream, after the compute; a pending
+ * side-stream MSE is waited for first (the launches share the plan's
+ * scratch).  cuda_stream must belong to the plan's device and outlive the
+ * plan's use of it; pab_plan_destroy waits for every pending side-stream MSE.
+ * The first enable creates the plan's events on the current device.
+ * Errors: PAB_ERR_ARG (null plan, enable not 0 or 1), PAB_ERR_CUDA. */
+int pab_plan_set_diff_mse_stream(pab_plan* plan, int enable, void* cuda_stream);
+
 /* Allocate the cache (2 output slots per kind, plus bf16 staging for
  * PAB_FP32 plans) on the current device now instead of at each kind's first
  * compute.  Idempotent. */

@@ -39,7 +39,7 @@ EXPORTS = (
     "pab_scatter_blocks", "pab_block_gemm", "pab_block_layer_norm", "pab_ipc_alloc", "pab_ipc_free", "pab_ipc_open", "pab_ipc_close",
     "pab_cross_attention", "pab_layout", "pab_attn_diff_mse", "pab_attn_diff_mse_async", "pab_attn_diff_mse_noalloc",
     "pab_device_errors", "pab_plan_create", "pab_plan_destroy", "pab_plan_reset",
-    "pab_plan_prepare", "pab_plan_set_diff_mse", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
+    "pab_plan_prepare", "pab_plan_set_diff_mse", "pab_plan_set_diff_mse_stream", "pab_schedule_query", "pab_schedule_source", "pab_schedule_count",
     "pab_attention",
 )
 
@@ -92,6 +92,7 @@ def _load() -> ctypes.CDLL:
         "pab_plan_reset": ([vp], i),
         "pab_plan_prepare": ([vp], i),
         "pab_plan_set_diff_mse": ([vp, vp], i),
+        "pab_plan_set_diff_mse_stream": ([vp, i, vp], i),
         "pab_schedule_query": ([vp, i, i, ctypes.POINTER(i)], i),
         "pab_schedule_source": ([vp, i, i, ctypes.POINTER(i)], i),
         "pab_schedule_count": ([vp, i, ctypes.POINTER(i)], i),
@@ -462,6 +463,17 @@ class Plan:
         else:
             _check(lib.pab_plan_set_diff_mse(self._h, None))
             self._mse_results = None
+
+    def set_diff_mse_stream(self, stream=None):
+        """Run the plan's MSE launches on `stream` (a torch.cuda.Stream), where
+        they overlap the following attention computes; the table is complete
+        once that stream has drained.  None: in line on the compute stream."""
+        if stream is None:
+            _check(lib.pab_plan_set_diff_mse_stream(self._h, 0, None))
+            self._mse_stream = None
+        else:
+            self._mse_stream = stream  # keep the stream alive while the plan launches on it
+            _check(lib.pab_plan_set_diff_mse_stream(self._h, 1, _stream(stream)))
 
     def is_compute(self, kind, step: int) -> bool:
         kind = KIND.get(kind, kind)

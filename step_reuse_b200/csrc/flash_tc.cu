@@ -31,10 +31,10 @@
 //                          accumulates the row sums of P with the same bf16 P
 //                          as the numerator (the softmax keeps no running sum);
 //   softmax warps         per tile X one warp per TMEM lane quarter (for
-//                          head dims up to 96 two, each taking 32 of every 64
-//                          keys): the thread of query row i (TMEM lane i)
-//                          reads its scores of S with
-//                          tcgen05.ld, keeps the running max in registers,
+//                          head dims up to 16 * PAB_FLASH_SPLIT_KSTEPS two,
+//                          taking the 64-key steps in turns): the thread of
+//                          query row i (TMEM lane i) reads its scores of S
+//                          with tcgen05.ld, keeps the running max,
 //                          writes P as bf16 over S's columns and rescales O in
 //                          TMEM only when the running max grew by more than
 //                          2^8 (the final O / l is exact either way);
@@ -81,6 +81,9 @@ constexpr int kBN = 64;           // keys per K/V tile
 constexpr int kQBox = 128 * 128;  // bytes of one [128 rows][64 cols] bf16 box (Q, O)
 constexpr int kKVBox = 64 * 128;  // bytes of one [64 rows][64 cols] bf16 box (K, V)
 constexpr uint32_t kTmemCols = 512;
+// SPLIT 2 register split (setmaxnreg): softmax warpgroups / the other warpgroup
+constexpr int kSplitRegsSoftmax = 104;
+constexpr int kSplitRegsOther = 64;
 constexpr float kRescaleLog2 = 8.0f;
 // Exponentials: of every 8 consecutive pairs of a row's scores, this many go
 // to tc::exp2_poly2 on the FMA pipes and the rest to the MUFU ex2 unit,
@@ -193,8 +196,8 @@ struct Cursor {
 //   slot_full/ready/done[s]     once per ring use s (use u of slot s: u / NST)
 //   p_full[X][b]                once per global step g with g & 1 == b
 //   o_done[X], stage[X]         once per item
-//   xmax_done[X][q][b]          once per exchange of maxima with b == its count & 1
-//   xsum_done[X][q]             once per exchange of row sums
+//   mref_full[X][q][b]          once per global step g with g & 1 == b (SPLIT 2)
+//   xsum_done[X][q]             once per item with work for tile X (SPLIT 2 without the ones column)
 struct Bars {
     unsigned long long q_full[2][2];              // [Q buffer][tile]: Q landed
     unsigned long long q_free[2][2];              // [Q buffer][tile]: the output staged there was stored
@@ -205,8 +208,8 @@ struct Bars {
     unsigned long long p_full[2][2];              // [tile][S buffer]: P written
     unsigned long long o_done[2];                 // [tile]: the item's last PV retired
     unsigned long long stage[2];                  // [tile]: the item's output is staged
-    unsigned long long xmax_done[2][4][2];        // [tile][lane quarter][buffer]: both halves' maxima written
-    unsigned long long xsum_done[2][4];           // [tile][lane quarter]: both halves' row sums written
+    unsigned long long mref_full[2][4][2];        // [tile][lane quarter][step parity]: the step's maxima written
+    unsigned long long xsum_done[2][4];           // [tile][lane quarter]: both warps' row sums written
     unsigned long long mma_done[2];
     uint32_t tmem_base;
     int abort;
@@ -261,13 +264,17 @@ struct DLayout {
 };
 
 // Softmax split: SPLIT = 2 gives every query row two warps -- the two warps
-// of one TMEM lane quarter on one sub-partition -- each exponentiating 32 of
-// a 64-key tile's scores, so four softmax warps share each sub-partition and
-// hide the exponential pass's latencies (the head dims where the
-// exponentials, not the tensor cores, bound the kernel).  The two halves of
-// a row exchange their maxima through shared memory behind an mbarrier of the
-// pair (a bounded wait, like every wait here), so both take the same
-// rescaling decisions.
+// of one TMEM lane quarter on one sub-partition -- that take the row's 64-key
+// steps in turns (warp par takes the global steps g with g & 1 == par, i.e.
+// the S buffer par), so four softmax warps share each sub-partition and the
+// turns keep them out of phase: one warp's TMEM load and row maximum run
+// while the other exponentiates.  The row's running maximum passes from step
+// to step through shared memory behind an mbarrier per (tile, lane quarter,
+// step parity) (a bounded wait, like every wait here), published as soon as
+// the step has decided it, before its exponentials; the rescaling of O then
+// follows the one sequence of maxima, and without the ones column each warp
+// keeps its own row sum in the units of the maximum of its latest step
+// (brought to the final one in the epilogue).
 #ifndef PAB_FLASH_SPLIT_KSTEPS
 #define PAB_FLASH_SPLIT_KSTEPS 0  // head dims up to 16 * this many columns split their rows
 #endif
@@ -287,7 +294,6 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
     constexpr int SPLIT = flash_split<KSTEPS>();
     constexpr int NSW = 8 * SPLIT;           // softmax warps
     constexpr int W_PROD = NSW, W_MMA = NSW + 1, W_ONES = NSW + 3;
-    constexpr int KC = kBN / SPLIT;          // keys of a tile per softmax warp
     constexpr int NO = KSTEPS * 16;          // N of the PV product (d rounded up to 16)
     constexpr int NC = NO / 16;              // 16-column chunks of O
     constexpr bool TILED = GEO != kGeoFull;
@@ -298,11 +304,12 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
     const uint32_t q_s = sbase;                      // [2 buffers][2 tiles] Q tiles
     const uint32_t k_s = q_s + 4 * DL::QTile;        // [NST] K_s
     const uint32_t v_s = k_s + NST * DL::KTile;      // [NST] V_{s-2}
-    const uint32_t x_s = v_s + NST * DL::VTile;      // SPLIT 2: half-row maxima and sums
+    const uint32_t x_s = v_s + NST * DL::VTile;      // SPLIT 2: row maxima and sums
     unsigned char* gen_base = smem_raw + (sbase - smem_u32(smem_raw));
-    // [step parity][tile][half][row] maxima, [tile][half][row] row sums
-    float* xmax = reinterpret_cast<float*>(gen_base + (x_s - sbase));
-    float* xsum = xmax + 2 * 2 * 2 * 128;
+    // [tile][step parity][row] maxima, [item parity][tile][sum of warp 0, 1;
+    // maximum of warp 0, 1][row] row sums
+    float* mref = reinterpret_cast<float*>(gen_base + (x_s - sbase));
+    float* xsum = mref + 2 * 2 * 128;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -311,17 +318,17 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
             for (int u = 0; u < 2; ++u) {
                 mbar_init(smem_u32(&bars.q_full[u][x]), 1);
                 mbar_init(smem_u32(&bars.q_free[u][x]), 1);
-                mbar_init(smem_u32(&bars.p_full[x][u]), 128 * SPLIT);
+                mbar_init(smem_u32(&bars.p_full[x][u]), 128);
             }
             mbar_init(smem_u32(&bars.o_done[x]), 1);
             mbar_init(smem_u32(&bars.mma_done[x]), 1);
         }
-        mbar_init(smem_u32(&bars.b_go), 128 * SPLIT);
+        mbar_init(smem_u32(&bars.b_go), 128);
         for (int x = 0; x < 2; ++x) {
             mbar_init(smem_u32(&bars.stage[x]), 128 * SPLIT);
             for (int q = 0; q < 4; ++q) {
                 mbar_init(smem_u32(&bars.xsum_done[x][q]), 64);
-                for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&bars.xmax_done[x][q][u]), 64);
+                for (int u = 0; u < 2; ++u) mbar_init(smem_u32(&bars.mref_full[x][q][u]), 32);
             }
         }
         for (int st = 0; st < NST; ++st) {
@@ -349,6 +356,12 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = bars.tmem_base;
+    // SPLIT 2: 640 threads launch with 96 registers each; the softmax
+    // warpgroups take 104, the producer / MMA / ones warpgroup keeps 64
+    // (4 x 128 x 104 + 128 x 64 = 640 x 96), each at the top of its role
+    auto regs_other = [&]() {
+        if constexpr (SPLIT == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(kSplitRegsOther) : "memory");
+    };
 
     // TMA coordinates of query tile x's box at column c0 and of key block j's
     // box at column c0
@@ -378,6 +391,7 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
 
     if (warp == W_PROD) {
         // ------------------------------------------------ TMA producer
+        regs_other();
         if (lane == 0) {
             Cursor<GEO> ck, cv;  // the K part of ring use s (step s) and its V part (step s - 2)
             ck.start(a);
@@ -450,6 +464,7 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
         }
     } else if (warp == W_MMA || warp == W_MMA + 1) {
         // ------------------------------------------------ MMA issuers (warp-uniform)
+        regs_other();
         // A wait of one issuer overlaps the other's MMA issue, so the tensor
         // core queue stays fed.
         const int x = warp - W_MMA;
@@ -530,6 +545,7 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
         mbar_wait_bounded(smem_u32(&bars.mma_done[x]), 0, &g_flash_err);
     } else if (warp == W_ONES) {
         // ------------------------------------------------ V-ones warp
+        regs_other();
         if constexpr (ONES) {
             const uint32_t col = (uint32_t)a.d;
             const uint32_t ch = (col & 63) >> 3, e = col & 7;
@@ -558,107 +574,76 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
         }
     } else if (warp < NSW) {
         // ------------------------------------------------ softmax warps
-        const int lq = warp & 3;                       // TMEM lane quarter (= sub-partition)
-        const int x = (warp >> 2) & 1;                 // tile
-        const int hf = SPLIT == 2 ? (warp >> 3) : 0;   // key half of every 64-key tile
-        const int kc0 = hf * KC;                       // first key of this warp's part
+        if constexpr (SPLIT == 2)
+            asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(kSplitRegsSoftmax) : "memory");
+        const int lq = warp & 3;                      // TMEM lane quarter (= sub-partition)
+        const int x = (warp >> 2) & 1;                // tile
+        const int par = SPLIT == 2 ? (warp >> 3) : 0; // SPLIT 2: the parity of the global steps taken
         const int row = lq * 32 + lane;
         const uint32_t lane_addr = tmem + ((uint32_t)(lq * 32) << 16);
         const uint32_t o_col = 256 + x * 128;
-        // O's 16-column chunks this warp rescales and stores
+        // O's 16-column chunks this warp normalises and stages in the epilogue
         constexpr int NC0 = SPLIT == 2 ? (NC + 1) / 2 : NC;
-        const int c_lo = hf == 0 ? 0 : NC0, c_hi = hf == 0 ? NC0 : NC;
+        const int c_lo = par == 0 ? 0 : NC0, c_hi = par == 0 ? NC0 : NC;
+        const bool store_thread = par == 0 && row == 0;
         Cursor<GEO> c;
         c.start(a);
         bool ok = true;
         if (x == 1 && c.valid(a)) ok = wait_bar(&bars, &bars.b_go, 0);
-        int g = 0;        // global step
-        int nx = 0, ns = 0;  // exchanges of maxima and of row sums with the row's other half
+        int g = 0;              // global step
+        bool owe_free = false;  // store thread: the previous item's Q buffer is still to be freed
+        int ns = 0;             // row-sum exchanges (SPLIT 2 without the ones column)
         for (; ok && c.valid(a); c.next_item(a)) {
             const Item m = c.m;
             const int k = c.k;
             const bool work = x == 0 || m.has_b;
+            // m_ref: the maximum P was taken against at this warp's latest step
+            // of the item (SPLIT 1: every step); l: the row sum in its units
             float m_ref = -INFINITY, l = 0.f;
+            if (SPLIT == 2 && owe_free && m.nkv == 1 && (g & 1) != par) {
+                // no step of this item here: free the previous item's Q buffer now
+                bulk_wait_read<0>();
+                mbar_arrive(smem_u32(&bars.q_free[(k - 1) & 1][x]));
+                owe_free = false;
+            }
             for (int j = 0; j < m.nkv; ++j, ++g) {
+                if (SPLIT == 2 && (g & 1) != par) continue;  // the other warp's step
                 // S_X(g) was issued with ring use g
                 ok = wait_bar(&bars, &bars.slot_done[g % NST][x], (g / NST) & 1);
                 if (!ok) break;
-                if (work) {
-                    tc::fence_after_sync();
-                    const uint32_t s_col = x * 128 + (g & 1) * 64;
-                    const int valid = TILED ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
-                    // this warp's scores of the row: one TMEM read each 32 keys
-                    float sv[KC];
-                    {
-                        uint32_t r0[32];
-                        tc::ld_32col(lane_addr + s_col + kc0, r0);
-                        if constexpr (KC == 64) {
-                            uint32_t r1[32];
-                            tc::ld_32col(lane_addr + s_col + 32, r1);
-                            tc::wait_ld();
-#pragma unroll
-                            for (int i = 0; i < 32; ++i) sv[32 + i] = __uint_as_float(r1[i]);
-                        } else {
-                            tc::wait_ld();
-                        }
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) sv[i] = __uint_as_float(r0[i]);
-                    }
-                    if (kc0 + KC > valid) {
-#pragma unroll
-                        for (int i = 0; i < KC; ++i)
-                            if (kc0 + i >= valid) sv[i] = -INFINITY;
-                    }
-                    // row max of the raw scores (scale > 0 commutes with max):
-                    // eight independent 3-input max chains
-                    float mt;
-                    {
-                        float mx[8];
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) {
-                            float mm = tc::max3f(sv[q], sv[q + 8], sv[q + 16]);
-                            if constexpr (KC == 64) {
-                                mm = tc::max3f(mm, sv[q + 24], sv[q + 32]);
-                                mm = tc::max3f(mm, sv[q + 40], sv[q + 48]);
-                                mx[q] = fmaxf(mm, sv[q + 56]);
-                            } else {
-                                mx[q] = fmaxf(mm, sv[q + 24]);
-                            }
-                        }
-                        mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
-                                       fmaxf(mx[6], mx[7])) * a.scale_log2;
-                    }
+                const uint32_t s_col = x * 128 + (g & 1) * 64;
+                // The row's maximum for this step from mt, the row max of its
+                // scaled scores: against the maximum so far -- this warp's own
+                // (SPLIT 1) or the one the other warp took at step g - 1 (SPLIT
+                // 2, read behind the barrier of that step's parity; waited for at
+                // every step, so that the slot is not written again before it
+                // was read) -- with O rescaled when it grows by more than 2^8.
+                // Returns false on an abort.
+                auto decide = [&](float mt, float& m_use) -> bool {
+                    float m_in = m_ref;
                     if constexpr (SPLIT == 2) {
-                        // the two halves of the row meet (double-buffered by exchange
-                        // parity); both take max(own, other), the same value (max is
-                        // exact and order-free).  The wait also orders this half's
-                        // score reads before the other half's P writes over them.
-                        float* xm = xmax + (((nx & 1) * 2 + x) * 2) * 128;
-                        unsigned long long* xb = &bars.xmax_done[x][lq][nx & 1];
-                        xm[hf * 128 + row] = mt;
-                        tc::fence_before_sync();
-                        mbar_arrive(smem_u32(xb));
-                        ok = wait_bar(&bars, xb, (nx >> 1) & 1);
-                        if (!ok) break;
-                        tc::fence_after_sync();
-                        ++nx;
-                        const float mo = xm[(hf ^ 1) * 128 + row];
-                        mt = hf == 0 ? fmaxf(mt, mo) : fmaxf(mo, mt);
+                        if (g > 0) {
+                            const int pg = (g - 1) & 1;
+                            if (!wait_bar(&bars, &bars.mref_full[x][lq][pg], ((g - 1) >> 1) & 1)) return false;
+                            m_in = mref[(x * 2 + pg) * 128 + row];
+                        }
                     }
                     if (j == 0) {
-                        m_ref = mt;
+                        m_use = mt;
                         if (g == 0 && x == 0) mbar_arrive(smem_u32(&bars.b_go));
                     } else {
-                        const bool need = mt > m_ref + kRescaleLog2;
+                        m_use = m_in;
+                        const bool need = mt > m_in + kRescaleLog2;
                         if (__any_sync(0xffffffffu, need)) {
                             // O_X must hold exactly PV_X(..g-1): PV_X(g-1) was
                             // committed with ring use g + 1
-                            ok = wait_bar(&bars, &bars.slot_done[(g + 1) % NST][x], ((g + 1) / NST) & 1);
-                            if (!ok) break;
+                            if (!wait_bar(&bars, &bars.slot_done[(g + 1) % NST][x], ((g + 1) / NST) & 1))
+                                return false;
                             tc::fence_after_sync();
-                            const float m_new = need ? mt : m_ref;
-                            const float f = ex2(m_ref - m_new);
-                            for (int cc = c_lo; cc < c_hi; ++cc) {
+                            if (need) m_use = mt;
+                            const float f = ex2(m_in - m_use);
+#pragma unroll 1
+                            for (int cc = 0; cc < NC; ++cc) {
                                 uint32_t r[16];
                                 tc::ld_16col(lane_addr + o_col + cc * 16, r);
                                 tc::wait_ld();
@@ -666,19 +651,62 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                                 for (int i = 0; i < 16; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * f);
                                 tc::st_16col(lane_addr + o_col + cc * 16, r);
                             }
-                            if constexpr (!ONES) l *= f;
-                            m_ref = m_new;
                         }
                     }
+                    if constexpr (SPLIT == 2) {
+                        // publish this step's maximum before the exponentials
+                        mref[(x * 2 + (g & 1)) * 128 + row] = m_use;
+                        mbar_arrive(smem_u32(&bars.mref_full[x][lq][g & 1]));
+                    }
+                    // this warp's running sum follows the row's maximum
+                    if constexpr (!ONES)
+                        if (l != 0.f && m_use != m_ref) l *= ex2(m_ref - m_use);
+                    m_ref = m_use;
+                    return true;
+                };
+                if (work) {
+                    tc::fence_after_sync();
+                    const int valid = TILED ? kBN : a.Lk - j * kBN;  // keys of this tile that exist
+                    float sv[kBN];
+                    {
+                        uint32_t r0[32], r1[32];
+                        tc::ld_32col(lane_addr + s_col, r0);
+                        tc::ld_32col(lane_addr + s_col + 32, r1);
+                        tc::wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) {
+                            sv[i] = __uint_as_float(r0[i]);
+                            sv[32 + i] = __uint_as_float(r1[i]);
+                        }
+                    }
+                    if (valid < kBN) {
+#pragma unroll
+                        for (int i = 0; i < kBN; ++i)
+                            if (i >= valid) sv[i] = -INFINITY;
+                    }
+                    // row max of the raw scores (scale > 0 commutes with max):
+                    // eight independent 3-input max chains
+                    float mx[8];
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float mm = tc::max3f(sv[q], sv[q + 8], sv[q + 16]);
+                        mm = tc::max3f(mm, sv[q + 24], sv[q + 32]);
+                        mm = tc::max3f(mm, sv[q + 40], sv[q + 48]);
+                        mx[q] = fmaxf(mm, sv[q + 56]);
+                    }
+                    const float mt = tc::max3f(tc::max3f(mx[0], mx[1], mx[2]), tc::max3f(mx[3], mx[4], mx[5]),
+                                               fmaxf(mx[6], mx[7])) * a.scale_log2;
+                    float m_use;
+                    ok = decide(mt, m_use);
+                    if (!ok) break;
                     // exponentiate, sum and write P back as bf16 over S's columns
-                    // (keys kc0.. as pairs: columns kc0 / 2 ..)
                     const tc::f32x2 scale2 = tc::pack2(a.scale_log2, a.scale_log2);
-                    const tc::f32x2 negm2 = tc::pack2(-m_ref, -m_ref);
+                    const tc::f32x2 negm2 = tc::pack2(-m_use, -m_use);
                     tc::f32x2 acc[4];
 #pragma unroll
                     for (int q = 0; q < 4; ++q) acc[q] = tc::pack2(0.f, 0.f);
 #pragma unroll
-                    for (int cc = 0; cc < KC / 32; ++cc) {
+                    for (int cc = 0; cc < kBN / 32; ++cc) {
                         uint32_t r[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
@@ -695,7 +723,7 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                             if constexpr (!ONES) acc[i & 3] = tc::add2(acc[i & 3], tc::pack2(p0, p1));
                             r[i] = pack_bf16x2(p0, p1);
                         }
-                        tc::st_16col(lane_addr + s_col + kc0 / 2 + cc * 16, r);
+                        tc::st_16col(lane_addr + s_col + cc * 16, r);
                     }
                     if constexpr (!ONES) {
                         float a0, a1;
@@ -703,13 +731,24 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                         l += a0 + a1;
                     }
                     tc::wait_st();
+                } else {
+                    float m_use;
+                    ok = decide(-INFINITY, m_use);
+                    if (!ok) break;
+                }
+                if (SPLIT == 2 && j == 0 && k > 0) {
+                    // the item's first PV overwrites O: both warps of the tile
+                    // have read the previous item's O (its stage barrier)
+                    ok = wait_bar(&bars, &bars.stage[x], (k - 1) & 1);
+                    if (!ok) break;
                 }
                 tc::fence_before_sync();
                 mbar_arrive(smem_u32(&bars.p_full[x][g & 1]));
-                if (j == 0 && k > 0 && hf == 0 && row == 0) {
+                if (owe_free) {
                     // the previous item's output store has read its staging: free that Q buffer
                     bulk_wait_read<0>();
                     mbar_arrive(smem_u32(&bars.q_free[(k - 1) & 1][x]));
+                    owe_free = false;
                 }
             }
             if (!ok) break;
@@ -725,13 +764,22 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                     tc::ld_1col(lane_addr + o_col + (uint32_t)a.d, lbits);
                     tc::wait_ld();
                     l = __uint_as_float(lbits);
-                } else if constexpr (SPLIT == 2) {  // the halves' sums, added in one order
-                    float* xs = xsum + (x * 2) * 128;
-                    xs[hf * 128 + row] = l;
+                } else if constexpr (SPLIT == 2) {
+                    // the two warps' sums, each in the units of its latest
+                    // maximum, brought to the later (larger) one and added in
+                    // one order (double-buffered by exchange parity; both warps
+                    // of the tile skip the exchange together when the tile is idle)
+                    float* xs = xsum + ((ns & 1) * 2 + x) * 4 * 128;
+                    xs[par * 128 + row] = l;
+                    xs[(2 + par) * 128 + row] = m_ref;
                     mbar_arrive(smem_u32(&bars.xsum_done[x][lq]));
                     ok = wait_bar(&bars, &bars.xsum_done[x][lq], ns & 1);
                     ++ns;
-                    l = xs[row] + xs[128 + row];
+                    if (!ok) break;
+                    const float l0 = xs[row], l1 = xs[128 + row];
+                    const float m0 = xs[256 + row], m1 = xs[384 + row];
+                    const float mf = fmaxf(m0, m1);
+                    l = (l0 != 0.f ? l0 * ex2(m0 - mf) : 0.f) + (l1 != 0.f ? l1 * ex2(m1 - mf) : 0.f);
                 }
                 const float inv = 1.f / l;
                 for (int cc = c_lo; cc < c_hi; ++cc) {
@@ -762,35 +810,38 @@ __global__ void __launch_bounds__(flash_threads<KSTEPS>(), 1)
                 fence_proxy_async_smem();
             }
             // Every softmax thread of the tile has staged its part once the stage
-            // barrier completes; only the storing thread waits for it (a bounded
-            // wait: no thread can be left behind at a barrier after an abort).
-            // The O columns were read: the next item's first PV, which waits for
-            // every thread's P, may overwrite them.
+            // barrier completes; only the storing thread waits for it here (a
+            // bounded wait: no thread can be left behind at a barrier after an
+            // abort).  The O columns were read: the next item's first PV, which
+            // waits for every thread's P (SPLIT 2: and for this barrier), may
+            // overwrite them.
             tc::fence_before_sync();
             mbar_arrive(smem_u32(&bars.stage[x]));
+            if (store_thread) ok = wait_bar(&bars, &bars.stage[x], k & 1);
             if (!ok) break;
-            if (hf == 0 && row == 0) ok = wait_bar(&bars, &bars.stage[x], k & 1);
-            if (!ok) break;
-            if (work && hf == 0 && row == 0) {
-                const uint32_t src = q_s + ((k & 1) * 2 + x) * DL::QTile;
-                for (int bx = 0; bx < DL::NB0; ++bx) {
-                    if constexpr (TILED)
-                        tc::tma_store_5d(&tm_o, src + bx * kQBox, bx * 64, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b);
-                    else
-                        tc::tma_store_4d(&tm_o, src + bx * kQBox, bx * 64, m.h, (m.qblk * 2 + x) * kBM, m.b);
+            if (store_thread) {
+                if (work) {
+                    const uint32_t src = q_s + ((k & 1) * 2 + x) * DL::QTile;
+                    for (int bx = 0; bx < DL::NB0; ++bx) {
+                        if constexpr (TILED)
+                            tc::tma_store_5d(&tm_o, src + bx * kQBox, bx * 64, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b);
+                        else
+                            tc::tma_store_4d(&tm_o, src + bx * kQBox, bx * 64, m.h, (m.qblk * 2 + x) * kBM, m.b);
+                    }
+                    if constexpr (DL::TK > 0) {
+                        const uint32_t tsrc = src + DL::NB0 * kQBox;
+                        if constexpr (TILED)
+                            tc::tma_store_5d(&tm_ot, tsrc, DL::NB0 * 64, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b);
+                        else
+                            tc::tma_store_4d(&tm_ot, tsrc, DL::NB0 * 64, m.h, (m.qblk * 2 + x) * kBM, m.b);
+                    }
+                    bulk_commit();
                 }
-                if constexpr (DL::TK > 0) {
-                    const uint32_t tsrc = src + DL::NB0 * kQBox;
-                    if constexpr (TILED)
-                        tc::tma_store_5d(&tm_ot, tsrc, DL::NB0 * 64, m.h, m.tx * 16, m.ty * 16 + x * 8, m.b);
-                    else
-                        tc::tma_store_4d(&tm_ot, tsrc, DL::NB0 * 64, m.h, (m.qblk * 2 + x) * kBM, m.b);
-                }
-                bulk_commit();
+                owe_free = true;
             }
         }
         // shared memory stays valid until every output store has read it
-        if (hf == 0 && row == 0) bulk_wait_read<0>();
+        if (store_thread) bulk_wait_read<0>();
     }
     tc::fence_before_sync();
     __syncthreads();
@@ -865,13 +916,16 @@ struct FlashMaps {
     CUtensorMap q, qt, k, kt, v, o, ot;
 };
 
+// SPLIT 2 exchange arrays: maxima [2][2][128] and row sums [2][2][4][128] floats
+constexpr int kSplitSmem = (2 * 2 * 128 + 2 * 2 * 4 * 128) * 4;
+
 // Ring depth: the deepest ring (at most kMaxStages) that fits the 227 KB of
 // shared memory next to the double-buffered Q tiles.
 template <int KSTEPS>
 constexpr int flash_nst() {
     using DL = DLayout<KSTEPS>;
     constexpr long long budget = 232448 - 2048;  // static shared memory (barriers) and slack
-    constexpr long long fixed = 4LL * DL::QTile + (flash_split<KSTEPS>() == 2 ? 6144 : 0) + 1024;
+    constexpr long long fixed = 4LL * DL::QTile + (flash_split<KSTEPS>() == 2 ? kSplitSmem : 0) + 1024;
     constexpr long long n = (budget - fixed) / (DL::KTile + DL::VTile);
     return n > kMaxStages ? kMaxStages : (int)n;
 }
@@ -879,7 +933,7 @@ template <int KSTEPS>
 constexpr size_t flash_smem() {
     using DL = DLayout<KSTEPS>;
     return (size_t)4 * DL::QTile + (size_t)flash_nst<KSTEPS>() * (DL::KTile + DL::VTile) +
-           (flash_split<KSTEPS>() == 2 ? 6144 : 0) + 1024;
+           (flash_split<KSTEPS>() == 2 ? kSplitSmem : 0) + 1024;
 }
 
 template <int KSTEPS, bool ONES, int GEO>
@@ -890,6 +944,19 @@ cudaError_t launch_ks1(const FlashMaps& m, const FlashTcArgs& a, cudaStream_t s)
     auto kern = flash_tc_kernel<KSTEPS, NST, ONES, GEO>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
+    if constexpr (flash_split<KSTEPS>() == 2) {
+        // the softmax warpgroups' setmaxnreg.inc is served by the registers the
+        // launch holds: refuse a build whose launch holds fewer than the split takes
+        static int regs = -1;
+        if (regs < 0) {
+            cudaFuncAttributes fa;
+            e = cudaFuncGetAttributes(&fa, kern);
+            if (e != cudaSuccess) return e;
+            regs = fa.numRegs;
+        }
+        if (regs * flash_threads<KSTEPS>() < kSplitRegsSoftmax * 512 + kSplitRegsOther * 128)
+            return cudaErrorInvalidConfiguration;
+    }
     // persistent: one CTA per SM (TMEM: 512 columns), each walking its items
     const int grid = a.items < device_sm_count() ? a.items : device_sm_count();
     kern<<<grid, flash_threads<KSTEPS>(), smem, s>>>(m.q, m.qt, m.k, m.kt, m.v, m.o, m.ot, a);

@@ -4,15 +4,18 @@
 // quantified by MSE).
 //
 // HBM-bound: each element is read once from each tensor (2 x size bytes).
-// One launch: a grid of (SM count x 4) blocks streams 16-byte vectors with a
-// grid-stride loop, accumulates (a - b)^2 in fp64 per thread, reduces each
+// One launch: a grid of (SM count x 8) blocks of 256 threads streams 16-byte
+// vectors with a grid-stride loop, accumulates (a - b)^2 in fp64 per thread, reduces each
 // warp with shuffles and each block through shared memory, and writes one
 // fp64 partial per block.  The block that finishes last (a completion
 // ticket counted with an atomic add) sums the partials in a fixed order,
 // divides by n and returns the ticket to zero for the next call.  The split
 // depends only on n and the SM count, and the final sum's order does not
 // depend on which block finishes last, so the result is bitwise reproducible
-// on a given device.
+// on a given device.  A block holds at most 48 registers a thread (12 K a
+// block), so when the MSE runs on a side stream its blocks fit on an SM next
+// to a flash attention CTA (384 threads of at most 136 registers, under
+// 230 KB of shared memory) and stream their bytes while the tensor cores work.
 #include "../../include/pab.h"
 #include "common.cuh"
 #include "kernels.h"
@@ -20,7 +23,8 @@
 namespace pab {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 256;
+constexpr int kMinBlocks = 5;  // 65536 / (256 * 5): at most 48 registers a thread
 constexpr int kUnroll = 4;
 
 template <typename T>
@@ -93,10 +97,9 @@ PAB_DEV double block_sum(double x, double* red) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) mse_kernel(const T* __restrict__ a, const T* __restrict__ b,
-                                                       long long n, unsigned long long* __restrict__ ticket,
-                                                       double* __restrict__ partials,
-                                                       double* __restrict__ result) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks)
+    mse_kernel(const T* __restrict__ a, const T* __restrict__ b, long long n, unsigned long long* __restrict__ ticket,
+               double* __restrict__ partials, double* __restrict__ result) {
     __shared__ double red[kThreads / 32];
     __shared__ bool last;
     constexpr int E = Vec<T>::kElems;
@@ -148,7 +151,7 @@ int mse_num_partials(long long n, int elem_size) {
     const long long nvec = n * elem_size / 16;
     const long long per_block = (long long)kThreads * kUnroll;
     long long blocks = (nvec + per_block - 1) / per_block;
-    const long long cap = (long long)device_sm_count() * 4;
+    const long long cap = (long long)device_sm_count() * 8;
     if (blocks > cap) blocks = cap;
     if (blocks < 1) blocks = 1;
     return (int)blocks;

@@ -203,6 +203,15 @@ struct pab_plan {
     // caller's device array [3][steps]; fp64 scratch: ticket + partials
     double* mse_results;
     double* mse_scratch;
+    // optional side stream for those MSE launches: the compute stream records
+    // ev_done for the side stream to wait on; ev_mse[kind] marks the kind's
+    // latest MSE, which the kind's next compute (it overwrites the slot the
+    // MSE reads) waits for while mse_pending[kind] is set
+    int mse_on_stream;
+    cudaStream_t mse_stream;
+    cudaEvent_t ev_done;
+    cudaEvent_t ev_mse[3];
+    int mse_pending[3];
     // bf16 staging for fp32 plans
     void* stage_in[3];
     void* stage_out;
@@ -218,6 +227,18 @@ bool sched_compute(const pab_plan* p, int kind, int i) {
 int sched_source(const pab_plan* p, int kind, int i) {
     if (sched_compute(p, kind, i)) return i;
     return p->lo + ((i - p->lo) / p->range[kind]) * p->range[kind];
+}
+
+// Let every side-stream MSE finish (it reads the slots) and release the events.
+void plan_free_events(pab_plan* p) {
+    for (int k = 0; k < 3; ++k) {
+        if (p->mse_pending[k] && p->ev_mse[k]) cudaEventSynchronize(p->ev_mse[k]);
+        p->mse_pending[k] = 0;
+        if (p->ev_mse[k]) cudaEventDestroy(p->ev_mse[k]);
+        p->ev_mse[k] = nullptr;
+    }
+    if (p->ev_done) cudaEventDestroy(p->ev_done);
+    p->ev_done = nullptr;
 }
 
 void plan_free_device(pab_plan* p) {
@@ -278,7 +299,7 @@ int plan_alloc_kind(pab_plan* p, int kind) {
 }
 
 int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void* v, void* out,
-                 cudaStream_t s, const void* prev, double* mse_result) {
+                 cudaStream_t s) {
     const long long qn = (long long)p->T * p->N * p->C;
     const long long kvn = (kind == PAB_CROSS) ? (long long)p->text_len * p->C : qn;
     const void *qq = q, *kk = k, *vv = v;
@@ -312,14 +333,6 @@ int plan_compute(pab_plan* p, int kind, const void* q, const void* k, const void
     if (p->dtype == PAB_FP32) {
         cudaError_t e = pab::launch_bf16_to_f32(p->stage_out, static_cast<float*>(out), qn, s);
         if (e != cudaSuccess) return cuda_fail(e, "bf16 -> fp32 conversion");
-    }
-    if (prev) {
-        // the difference to the kind's previous output, read back from HBM by
-        // the MSE kernel on the same stream
-        const int elem = p->dtype == PAB_FP32 ? 4 : 2;
-        const int parts = pab::mse_num_partials(qn, elem);
-        cudaError_t e = pab::launch_mse(out, prev, qn, p->dtype, p->mse_scratch, parts, mse_result, s);
-        if (e != cudaSuccess) return cuda_fail(e, "attention-difference MSE launch");
     }
     return PAB_OK;
 }
@@ -758,6 +771,7 @@ int pab_plan_create(int T, int H, int W, int heads, int d, int text_len, int ste
 
 int pab_plan_destroy(pab_plan* plan) {
     if (!plan) return PAB_OK;
+    plan_free_events(plan);
     plan_free_device(plan);
     delete plan;
     return PAB_OK;
@@ -838,6 +852,27 @@ int pab_plan_set_diff_mse(pab_plan* plan, double* results_dev) {
     PAB_GUARD_END
 }
 
+int pab_plan_set_diff_mse_stream(pab_plan* plan, int enable, void* cuda_stream) {
+    PAB_GUARD_BEGIN
+    if (!plan) return fail(PAB_ERR_ARG, "null plan");
+    if (enable != 0 && enable != 1) return fail(PAB_ERR_ARG, "enable must be 0 or 1");
+    if (enable) {
+        for (int k = 0; k < 4; ++k) {
+            cudaEvent_t* ev = k < 3 ? &plan->ev_mse[k] : &plan->ev_done;
+            if (*ev) continue;
+            cudaError_t e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming);
+            if (e != cudaSuccess) {
+                *ev = nullptr;
+                return cuda_fail(e, "MSE stream events");
+            }
+        }
+        plan->mse_stream = static_cast<cudaStream_t>(cuda_stream);
+    }
+    plan->mse_on_stream = enable;
+    return PAB_OK;
+    PAB_GUARD_END
+}
+
 int pab_plan_prepare(pab_plan* plan) {
     PAB_GUARD_BEGIN
     if (!plan) return fail(PAB_ERR_ARG, "null plan");
@@ -903,9 +938,46 @@ int pab_attention(pab_plan* plan, int kind, int step, const void* q, const void*
         prev = plan->slot[kind][plan->cur[kind]];
         mse_result = plan->mse_results + (long long)kind * plan->steps + step;
     }
-    rc = plan_compute(plan, kind, q, k, v, plan->slot[kind][slot], static_cast<cudaStream_t>(cuda_stream), prev,
-                      mse_result);
+    cudaStream_t s = static_cast<cudaStream_t>(cuda_stream);
+    // the slot about to be written may still be read by this kind's latest
+    // side-stream MSE
+    if (plan->mse_pending[kind]) {
+        cudaError_t e = cudaStreamWaitEvent(s, plan->ev_mse[kind], 0);
+        if (e != cudaSuccess) return cuda_fail(e, "wait for the side-stream MSE");
+        plan->mse_pending[kind] = 0;
+    }
+    rc = plan_compute(plan, kind, q, k, v, plan->slot[kind][slot], s);
     if (rc) return rc;
+    if (prev) {
+        // the difference to the kind's previous output, read back from HBM by
+        // the MSE kernel: on the compute stream, or on the side stream once the
+        // compute is done there (an inline launch first waits for every
+        // side-stream MSE still pending: they share the plan's scratch)
+        cudaStream_t ms = s;
+        cudaError_t e = cudaSuccess;
+        if (plan->mse_on_stream) {
+            ms = plan->mse_stream;
+            e = cudaEventRecord(plan->ev_done, s);
+            if (e == cudaSuccess) e = cudaStreamWaitEvent(ms, plan->ev_done, 0);
+        } else {
+            for (int j = 0; j < 3 && e == cudaSuccess; ++j)
+                if (plan->mse_pending[j]) {
+                    e = cudaStreamWaitEvent(s, plan->ev_mse[j], 0);
+                    plan->mse_pending[j] = 0;
+                }
+        }
+        if (e != cudaSuccess) return cuda_fail(e, "MSE stream ordering");
+        const long long qn = (long long)plan->T * plan->N * plan->C;
+        const int parts = pab::mse_num_partials(qn, plan->dtype == PAB_FP32 ? 4 : 2);
+        e = pab::launch_mse(plan->slot[kind][slot], prev, qn, plan->dtype, plan->mse_scratch, parts, mse_result,
+                            ms);
+        if (e != cudaSuccess) return cuda_fail(e, "attention-difference MSE launch");
+        if (plan->mse_on_stream) {
+            e = cudaEventRecord(plan->ev_mse[kind], ms);
+            if (e != cudaSuccess) return cuda_fail(e, "side-stream MSE event");
+            plan->mse_pending[kind] = 1;
+        }
+    }
     plan->cur[kind] = slot;
     plan->cached_step[kind] = step;
     plan->last_step[kind] = step;

@@ -165,6 +165,12 @@ def test_stateless_argument_checks(pab):
     assert lib.pab_attn_diff_mse(None, None, 10, 0, ctypes.byref(res), None) == pab.PAB_ERR_ARG
     assert lib.pab_attn_diff_mse(None, None, 10, 7, ctypes.byref(res), None) == pab.PAB_ERR_ARG
     assert lib.pab_attn_diff_mse(None, None, 10, 0, None, None) == pab.PAB_ERR_ARG
+    # side-stream MSE option: null plan, bad flag; disabling needs no device
+    assert lib.pab_plan_set_diff_mse_stream(None, 1, None) == pab.PAB_ERR_ARG
+    plan = pab.Plan(4, 8, 8, 2, 32, 16, 10, (2, 3, 4))
+    assert lib.pab_plan_set_diff_mse_stream(plan._h, 2, None) == pab.PAB_ERR_ARG
+    assert lib.pab_plan_set_diff_mse_stream(plan._h, 0, None) == pab.PAB_OK
+    plan.close()
 
 
 def test_spatial_alternatives_argument_checks(pab):

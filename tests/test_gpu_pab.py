@@ -194,13 +194,16 @@ def test_sweep_u_shape_and_counts(pab, oracle_mod):
                 assert edge_mse > 5 * mid_mse, (kind, edge_mse, mid_mse)
 
 
-def _run_plan_mse(pab, w, ranges, setup=None, seed=0):
-    """One run with the plan's MSE table on: (mse table, outputs of every compute)."""
+def _run_plan_mse(pab, w, ranges, setup=None, seed=0, side=None):
+    """One run with the plan's MSE table on (its launches on the stream
+    `side` when given): (mse table, outputs of every compute)."""
     plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, ranges, dtype=w.torch_dtype)
     if setup:
         setup(plan)
     table = torch.full((3, w.steps), -1.0, dtype=torch.float64, device="cuda")
     plan.set_diff_mse(table)
+    if side is not None:
+        plan.set_diff_mse_stream(side)
     x = synth.initial_inputs(w, device="cuda", seed=seed)
     g = synth.generator(seed + 1, "cuda")
     edge = _edge(w)
@@ -253,6 +256,47 @@ def test_plan_diff_mse(pab, oracle_mod, name, view):
             if name == "tiny" or n in (0, len(comps) - 2):
                 want = oracle_mod.mse(to_f64(o), to_f64(prev))
                 assert abs(t1[ki, i] - want) <= MSE_REL * want, (kind, i, t1[ki, i], want)
+
+
+@pytest.mark.parametrize("name", ["tiny", "480p"])
+def test_plan_diff_mse_side_stream(pab, name):
+    """The plan's MSE launches on a side stream (pab_plan_set_diff_mse_stream):
+    the table is bit-identical to the in-line one and every computed output
+    is unchanged -- the kind's next compute waits for the MSE reading the
+    slot it overwrites."""
+    w = synth.WORKLOADS[name]
+    t0, outs0 = _run_plan_mse(pab, w, w.ranges)
+    side = torch.cuda.Stream()
+    t1, outs1 = _run_plan_mse(pab, w, w.ranges, side=side)
+    assert np.array_equal(t0, t1)
+    for kind in synth.KINDS:
+        assert [i for i, _ in outs0[kind]] == [i for i, _ in outs1[kind]]
+        for (_, a), (_, b) in zip(outs0[kind], outs1[kind]):
+            assert torch.equal(a, b)
+
+
+def test_plan_diff_mse_stream_switch(pab):
+    """Switching between side-stream and in-line MSE launches mid-run gives
+    the same table (an in-line launch waits for the pending side-stream ones:
+    they share the plan's scratch)."""
+    w = synth.WORKLOADS["tiny"]
+    t0, _ = _run_plan_mse(pab, w, w.ranges)
+    side = torch.cuda.Stream()
+    plan = pab.Plan(w.T, w.H, w.W, w.heads, w.d, w.text_len, w.steps, w.ranges, dtype=w.torch_dtype)
+    table = torch.full((3, w.steps), -1.0, dtype=torch.float64, device="cuda")
+    plan.set_diff_mse(table)
+    x = synth.initial_inputs(w, device="cuda", seed=0)
+    g = synth.generator(1, "cuda")
+    edge = _edge(w)
+    for i in range(w.steps):
+        if i > 0:
+            synth.drift_(x, synth.sigma_at(w, i, edge), g)
+        plan.set_diff_mse_stream(side if i % 2 == 0 else None)
+        for kind in synth.KINDS:
+            plan.attention(kind, i, x[kind]["q"], x[kind]["k"], x[kind]["v"])
+    torch.cuda.synchronize()
+    plan.close()
+    assert np.array_equal(t0, table.cpu().numpy())
 
 
 @pytest.mark.parametrize("mode", ["window", "draft"])
