@@ -580,7 +580,8 @@ def run_ours(args):
                        mse="attention-difference MSE of every compute after a kind's first, one launch each "
                            "on a side stream (overlapping the next attention kernels)",
                        kernel_times="spatial: CUDA events around its launches in the timed region; the "
-                                    "other kernels: three more runs with every launch bracketed"),
+                                    "other kernels: three more runs with every launch bracketed; all of them "
+                                    "with the side-stream MSE launches overlapping"),
         "denoising_steps_per_s": world * w.steps / (ms * 1e-3),
         "executed_tflops": world * exec_flops / (ms * 1e-3) / 1e12,
         "computes": counts,
