@@ -67,7 +67,7 @@ def parse_args(argv=None):
     ap.add_argument("--workload", default="480p", choices=("480p", "720p", "temporal_heavy", "tiny", "sta_48x80", "draft_48x80"))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--e2e-steps", type=int, default=2)
+    ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--input-sets", type=int, default=8,
                     help="distinct drifted input sets cycled over the diffusion steps")
     ap.add_argument("--cpu-sample-s", type=float, default=15.0,

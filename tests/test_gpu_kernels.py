@@ -118,6 +118,26 @@ def test_cross_parity(pab, oracle_mod, R, Lt, heads, d):
                                   f"got {out[bad[:4, 0], bad[:4, 1]].tolist()} want {want1[bad[:4, 0], bad[:4, 1]].tolist()}")
 
 
+@pytest.mark.parametrize("R,Lt,heads,d", [
+    (86400, 256, 24, 128),  # 720p: every video token against 256 text tokens (the flash kernel)
+    (76800, 120, 16, 64),   # temporal-heavy: cross_tc at d = 64
+])
+def test_cross_full_size_sampled(pab, oracle_mod, R, Lt, heads, d):
+    """Full-size cross attention, checked on 1024 sampled query rows (rows
+    are independent, so the oracle of a row subset is the subset of the
+    oracle's output), spread over the whole range including the last row."""
+    C = heads * d
+    q = randn((R, C), 24)
+    kt, vt = randn((Lt, C), 25), randn((Lt, C), 26)
+    base, out = guarded_empty((R, C), torch.bfloat16)
+    pab.cross_attention(q, kt, vt, heads, out=out)
+    rows = torch.cat([torch.randperm(R - 1, generator=torch.Generator().manual_seed(27))[:1023],
+                      torch.tensor([R - 1])])
+    want = oracle_mod.cross_attention(to_f64(q[rows.cuda()]), to_f64(kt), to_f64(vt), heads)
+    assert_attn_close(out[rows.cuda()], want, f"cross full size R={R} Lt={Lt} h={heads} d={d}")
+    check_guards(base)
+
+
 def test_cross_row_order_is_kept(pab):
     R, Lt, heads, d = 500, 120, 4, 64
     C = heads * d
