@@ -87,7 +87,8 @@ def parse_args(argv=None):
     ap.add_argument("--sweep", action="store_true",
                     help="the 50-step sweep (480p shapes): every range set of the sweep workload timed, "
                          "with the per-step attention difference (MSE) of the all-compute run")
-    ap.add_argument("--kernel", choices=("spatial", "temporal", "temporal_sv", "cross", "layout", "mse"),
+    ap.add_argument("--kernel", choices=("spatial", "temporal", "temporal_sv", "cross", "layout", "mse",
+                                         "gemm_qkv", "gemm_mlp_in", "gemm_mlp_out"),
                     help="time one kernel alone on the workload's tensors (one input set, back-to-back "
                          "launches): the single-kernel view used for profiling")
     ap.add_argument("--dit", action="store_true",
@@ -1240,6 +1241,28 @@ def run_kernel(args):
         src = rnd(T, N, C)
         dst = torch.empty((N, T, C), dtype=torch.bfloat16, device=device)
         fn = lambda: pab.layout(src, True, out=dst)
+    elif kind.startswith("gemm"):
+        # the DiT block's projections on this workload's token rows: q | k | v
+        # (split into three outputs), the MLP's first GEMM with GELU, its
+        # second with the fp32 residual add
+        R = T * N
+        K, Nn, epi = {"gemm_qkv": (C, 3 * C, pab.GEMM_STORE), "gemm_mlp_in": (C, 4 * C, pab.GEMM_GELU),
+                      "gemm_mlp_out": (4 * C, C, pab.GEMM_RESID)}[kind]
+        A, B = rnd(R, K), (rnd(K, Nn) * K ** -0.5).to(torch.bfloat16)
+        if epi == pab.GEMM_RESID:
+            X = torch.zeros((R, Nn), dtype=torch.float32, device=device)
+            fn = lambda: pab.block_gemm(A, B, epi, X=X)
+            out_bytes = R * Nn * 4 * 2  # fp32 read and written
+        elif epi == pab.GEMM_STORE:
+            outs = [torch.empty((R, C), dtype=torch.bfloat16, device=device) for _ in range(3)]
+            fn = lambda: pab.block_gemm(A, B, epi, outs=outs)
+            out_bytes = R * Nn * 2
+        else:
+            outs = [torch.empty((R, Nn), dtype=torch.bfloat16, device=device)]
+            fn = lambda: pab.block_gemm(A, B, epi, outs=outs)
+            out_bytes = R * Nn * 2
+        flops[kind] = 2.0 * R * K * Nn
+        abytes[kind] = R * K * 2 + K * Nn * 2 + out_bytes
     else:
         a, b = rnd(T * N * C), rnd(T * N * C)
         res = torch.zeros(1, dtype=torch.float64, device=device)
