@@ -6,8 +6,12 @@
 // gemm_tc_kernel: D = epilogue(A B) on the 5th-generation tensor cores, A
 //   [M, K] bf16 row-major (K-major), B [K, N] bf16 row-major (the weights as
 //   [in, out], read MN-major), fp32 accumulators in TMEM.  Persistent CTAs
-//   walk 128 x BN output tiles (M fastest within an N column of tiles, so the
-//   CTAs running at one time share B and neighbouring A rows in L2):
+//   walk 128 x BN output tiles, the smaller operand's tile index fastest: M
+//   fastest within an N column of tiles when B is the larger operand (the
+//   CTAs running at one time share B and neighbouring A rows in L2), N
+//   fastest within an M row of tiles when A is (an A row block is read from
+//   HBM once and reused by the CTAs taking that row's N tiles, instead of A
+//   being streamed once per N column when it does not fit in L2):
 //     warp 4 (one thread)  TMA producer: a ring of NS stages of one
 //                          [128][64] A box and BN/64 [64][64] B boxes;
 //     warp 5               MMA issuer (warp-uniform, one elected lane), 4
@@ -52,6 +56,7 @@ struct GemmArgs {
     int M, N, K;
     int m_tiles, n_tiles;
     long long tiles;
+    int n_fast;  // tile t is (t / n_tiles, t % n_tiles) when set, else (t % m_tiles, t / m_tiles)
     // kStore: outputs out[0..2], each [M, split] row-major (split = N when one)
     __nv_bfloat16* out[3];
     int split;
@@ -124,7 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             long long it = 0;  // stage uses issued
             bool ok = true;
             for (long long t = blockIdx.x; t < g.tiles && ok; t += gridDim.x) {
-                const int mt = (int)(t % g.m_tiles), nt = (int)(t / g.m_tiles);
+                const int mt = g.n_fast ? (int)(t / g.n_tiles) : (int)(t % g.m_tiles);
+                const int nt = g.n_fast ? (int)(t % g.n_tiles) : (int)(t / g.m_tiles);
                 for (int k = 0; k < ksteps && ok; ++k, ++it) {
                     const int s = (int)(it % NS);
                     if (it >= NS) ok = gwait(&bars, &bars.empty[s], (uint32_t)(((it / NS) - 1) & 1));
@@ -180,7 +186,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         bool ok = true;
         for (long long t = blockIdx.x; t < g.tiles && ok; t += gridDim.x, ++i) {
             const int ab = i & 1;
-            const int mt = (int)(t % g.m_tiles), nt = (int)(t / g.m_tiles);
+            const int mt = g.n_fast ? (int)(t / g.n_tiles) : (int)(t % g.m_tiles);
+            const int nt = g.n_fast ? (int)(t % g.n_tiles) : (int)(t / g.m_tiles);
             ok = gwait(&bars, &bars.acc_full[ab], (uint32_t)((i >> 1) & 1));
             if (!ok) break;
             tc::fence_after_sync();
@@ -357,6 +364,7 @@ template <int EPI>
 cudaError_t launch_gemm_e(const CUtensorMap& ma, const CUtensorMap& mb, GemmArgs& g, int BN, cudaStream_t s) {
     g.n_tiles = (g.N + BN - 1) / BN;
     g.tiles = (long long)g.m_tiles * g.n_tiles;
+    g.n_fast = (long long)g.M * g.K > (long long)g.K * g.N ? 1 : 0;
     return BN == 256 ? launch_gemm_t<256, 4, EPI>(ma, mb, g, s) : launch_gemm_t<128, 6, EPI>(ma, mb, g, s);
 }
 
