@@ -804,7 +804,9 @@ def run_dit(args):
         torch.cuda.synchronize(device)
         ms = max_over_ranks(a.elapsed_time(b) / runs, device)
         counts = {k: sum(block.plan.is_compute(k, i) for i in range(w.steps)) for k in synth.KINDS}
-        res[label] = {"ms_per_run": ms, "computes": counts, "tflops": dit_flops(w, counts) / (ms * 1e-3) / 1e12}
+        tf = dit_flops(w, counts) / (ms * 1e-3) / 1e12
+        res[label] = {"ms_per_run": ms, "computes": counts, "tflops": tf,
+                      "frac_of_burst_bf16": tf / load_peaks()["tc"]}
         block.close()
     assert pab.device_errors() == 0
     if rank == 0:
