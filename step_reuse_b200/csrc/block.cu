@@ -6,7 +6,8 @@
 // gemm_tc_kernel: D = epilogue(A B) on the 5th-generation tensor cores, A
 //   [M, K] bf16 row-major (K-major), B [K, N] bf16 row-major (the weights as
 //   [in, out], read MN-major), fp32 accumulators in TMEM.  Persistent CTAs
-//   walk 128 x BN output tiles, the smaller operand's tile index fastest: M
+//   walk 128 x BN output tiles (BN = 256 unless N <= 128), the smaller
+//   operand's tile index fastest: M
 //   fastest within an N column of tiles when B is the larger operand (the
 //   CTAs running at one time share B and neighbouring A rows in L2), N
 //   fastest within an M row of tiles when A is (an A row block is read from
@@ -385,8 +386,9 @@ cudaError_t launch_gemm(const void* A, const void* B, int M, int N, int K, int e
     g.Y = static_cast<__nv_bfloat16*>(Y);
     CUtensorMap ma, mb;
     if (!make_map2d(&ma, A, M, K, kBM) || !make_map2d(&mb, B, K, N, kBK)) return cudaErrorInvalidValue;
-    // N a multiple of 256: 128 x 256 tiles; otherwise 128 x 128
-    const int BN = N % 256 == 0 ? 256 : 128;
+    // 128 x 256 tiles (a last partial N tile computes zero columns past N and
+    // stores nothing there); 128 x 128 only for N <= 128
+    const int BN = N > 128 ? 256 : 128;
     if (epi == kStore) return launch_gemm_e<kStore>(ma, mb, g, BN, s);
     if (epi == kGelu) return launch_gemm_e<kGelu>(ma, mb, g, BN, s);
     if (epi == kResid) return launch_gemm_e<kResid>(ma, mb, g, BN, s);
